@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark: forward pass of one MoE layer on B200, tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference] [--no-cpu-baseline]
+
+One step = route -> dispatch -> experts -> combine over one batch of the
+workload (default: the 64-expert builder layer, T=4096, H=4096, top-2,
+I=1408, bf16, Zipf(1.0)-skewed load), with inputs resident in HBM.  L2 is
+flushed (a 256 MiB write) before every timed step, outside the timed events.
+Each stage is bracketed by CUDA events on the launching stream, so the
+per-stage times and the grouped-GEMM roofline come from the same timed
+steps.  N > 1 (torchrun, one rank per GPU) runs independent replicas of the
+layer, each on its own token batch (weak scaling; the layer has no exchange
+step on one GPU's worth of experts), timed as the max over ranks.
+
+Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle instead (a bounded token sample per step; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_inputs import CONFIGS, make_layer, make_tokens  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1xB200; % of HBM or bf16 tensor roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+CPU_SAMPLE_TOKENS = 1024
+REF_SAMPLE_TOKENS = 256
+
+
+# ------------------------------------------------------------- helpers ---
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (6.65 TB/s, 1.59 PFLOP/s earlier pool measurement)"
+
+
+def expert_stage_work(cfg, counts):
+    """Algorithmic bytes and flops of the grouped-GEMM stage (both passes) for
+    the realised per-expert counts: weights of every expert with >= 1 row,
+    x_packed read, h written and read back, y_packed written, routing weights."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    active = sum(1 for c in counts if c > 0)
+    N = int(sum(counts))
+    H, I = cfg.H, cfg.I
+    wbytes = active * 3 * H * I * es
+    abytes = N * H * es + 2 * N * I * es + N * H * es + N * 4
+    flops = 2 * N * 3 * H * I
+    if cfg.shared_I:
+        wbytes += 3 * H * cfg.shared_I * es
+        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * es
+        flops += 2 * cfg.T * 3 * H * cfg.shared_I
+    return wbytes + abytes, flops
+
+
+def layer_work(cfg, counts):
+    """Algorithmic bytes / flops of the whole layer: activated expert weights,
+    router weights, x in, out out (the materialised packed intermediates are
+    not counted); flops of the router and the activated experts."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    active = sum(1 for c in counts if c > 0)
+    H, I, E, T = cfg.H, cfg.I, cfg.E, cfg.T
+    b = active * 3 * H * I * es + E * H * es + 2 * T * H * es
+    f = 2 * T * cfg.k * 3 * H * I + 2 * T * H * E
+    if cfg.shared_I:
+        b += 3 * H * cfg.shared_I * es + H * es
+        f += 2 * T * 3 * H * cfg.shared_I + 2 * T * H
+    return b, f
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_layer_44_b200", "csrc")
+    for name in ("experts_tc.cu", "sm100_ptx.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """Per-launch DRAM bytes of the grouped GEMM from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "grouped_gemm_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("per_step_bytes", {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while timing."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        props = torch.cuda.get_device_properties(device_index)
+        self.bus = None
+        try:
+            self.bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        except AttributeError:
+            pass
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.bus:
+            cmd += ["-i", self.bus]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------- CPU oracle ---
+
+def oracle_sample_run(cfg, p, ntok):
+    """The fp64 oracle, as it stands, on the first ``ntok`` tokens of the
+    workload (full router, dispatch, experts, merge for that sample)."""
+    import oracle.moe_oracle as O
+    sub = dict(p)
+    sub["x"] = p["x"][:ntok]
+    t0 = time.perf_counter()
+    O.moe_forward(sub, cfg.k, cfg.renormalize)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    p = make_layer(cfg, seed=0)
+    ntok = min(REF_SAMPLE_TOKENS, cfg.T)
+    for _ in range(args.warmup):
+        oracle_sample_run(cfg, p, ntok)
+    times = [oracle_sample_run(cfg, p, ntok) for _ in range(args.steps)]
+    total = sum(times)
+    value = ntok * args.steps / total
+    sample = (f"first {ntok} of the workload's {cfg.T} tokens per step (fp64 numpy oracle: "
+              f"router, dispatch, experts, merge), {args.steps} steps after {args.warmup} warm-up")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, counts):
+    c = {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I,
+         "renormalize": cfg.renormalize, "zipf_s": cfg.zipf_s, "empty_experts_forced": cfg.empty_tail,
+         "shared_I": cfg.shared_I, "seed": 0, "l2": "flushed: 256 MiB write before every timed step",
+         "parallelism": "replicas (one independent layer per GPU)"}
+    if counts is not None:
+        c["expert_counts"] = [int(x) for x in counts]
+    return c
+
+
+# ------------------------------------------------------------ GPU path ---
+
+def run_gpu(args, cfg):
+    import mixture_experts_layer_44_b200 as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    M.load_library()
+    dev = torch.device("cuda", local)
+
+    p = make_layer(cfg, seed=0)
+    if rank > 0:
+        p["x"] = make_tokens(cfg, seed=rank)
+    dp = {k: (v.to(dev) if v is not None else None) for k, v in p.items()}
+    buf = M.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.torch_dtype, device=dev,
+                            shared_I=cfg.shared_I)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    x = dp["x"]
+    E = cfg.E
+    shared = cfg.shared_I is not None
+    launches_per_step = M.KERNELS_PER_LAYER + (3 if shared else 0)
+
+    def step(ev=None):
+        # Each stage's events are recorded on the stream its kernels run on.
+        if ev:
+            ev[0].record(stream)
+        M.moe_route(x, dp["W_gate"], dp["bias"], cfg.k, cfg.renormalize, buf.logits, buf.ids,
+                    buf.w, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        M.moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
+                       buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status,
+                       stream=stream)
+        if ev:
+            ev[2].record(stream)
+        M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
+                      buf.y_packed, status=buf.status, stream=stream)
+        if shared:
+            M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
+            M.moe_experts(x, buf.sh_offsets, None, dp["w13s"].unsqueeze(0),
+                          dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, status=buf.status,
+                          stream=stream)
+        if ev:
+            ev[3].record(stream)
+        M.moe_combine(buf.y_packed, buf.inv_perm, cfg.T, cfg.k, buf.out,
+                      buf.sh_y if shared else None, buf.sg_logit if shared else None,
+                      status=buf.status, stream=stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if int(buf.status.item()) != 0:
+        raise SystemExit(f"device status {int(buf.status.item())} after warm-up")
+    counts = buf.counts.cpu().tolist()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    clock_info = clocks.stop()
+    if dist:
+        dist.barrier()
+    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
+    step_ms = [sum(s) for s in stage_ms]
+    ms = sum(step_ms) / args.steps
+    per_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(4)]
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    else:
+        ms_max = ms
+
+    # End to end through the public API with host buffers: pinned x in, out back.
+    x_host = p["x"].pin_memory()
+    out_host = torch.empty(cfg.T, cfg.H, dtype=cfg.torch_dtype).pin_memory()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps)
+    for _ in range(2):
+        M.moe_layer_forward_host(x_host, dp, cfg.k, cfg.renormalize, buf, out_host, stream=stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms_list = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        e_start.record(stream)
+        M.moe_layer_forward_host(x_host, dp, cfg.k, cfg.renormalize, buf, out_host, stream=stream)
+        e_end.record(stream)
+        e_end.synchronize()
+        e2e_ms_list.append(e_start.elapsed_time(e_end))
+    e2e_ms = sum(e2e_ms_list) / len(e2e_ms_list)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if int(buf.status.item()) != 0:
+        raise SystemExit(f"device status {int(buf.status.item())} after timing")
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        hbm = peaks["hbm_gbs"]
+        tf = peaks["bf16_tflops"]
+        bytes_x, flops_x = expert_stage_work(cfg, counts)
+        t_x = per_stage[2] / 1e3
+        ai = flops_x / bytes_x
+        ridge = tf * 1e12 / (hbm * 1e9)
+        if ai >= ridge:
+            roof = {"bound": "tensor", "achieved": flops_x / t_x / 1e12, "peak": tf,
+                    "unit": "TFLOP/s"}
+        else:
+            roof = {"bound": "hbm", "achieved": bytes_x / t_x / 1e9, "peak": hbm, "unit": "GB/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        tr = ncu_traffic(cfg.name)
+        roof["traffic"] = tr
+        roof["kernel"] = ("grouped_gemm_kernel (tcgen05), both passes of moe_experts: "
+                          f"{bytes_x/1e9:.3f} GB and {flops_x/1e9:.1f} GFLOP per step")
+        roof["peak_source"] = peak_src
+        lb, lf = layer_work(cfg, counts)
+        t_roof = max(lb / (hbm * 1e9), lf / (tf * 1e12))
+        cpu = None
+        if not args.no_cpu_baseline:
+            ntok = min(CPU_SAMPLE_TOKENS, cfg.T)
+            secs = oracle_sample_run(cfg, p, ntok)
+            cpu = {"value": ntok / secs, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                   "sample": f"first {ntok} of {cfg.T} tokens, fp64 numpy oracle (router, "
+                             f"dispatch, experts, merge), one run, {secs:.1f} s"}
+        es = 2 if cfg.dtype == "bf16" else 4
+        line = {
+            "metric": METRIC, "value": cfg.T * world / (ms_max / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights)",
+            "config": workload_config(cfg, counts),
+            "roofline": roof,
+            "layer_roofline": {"bytes": lb, "flops": lf, "t_roof_ms": t_roof * 1e3,
+                               "frac": t_roof / (ms / 1e3)},
+            "stage_ms": {"route": per_stage[0], "dispatch": per_stage[1],
+                         "experts": per_stage[2], "combine": per_stage[3]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": cfg.T * world / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": cfg.T * cfg.H * es,
+                    "d2h_bytes_per_step": cfg.T * cfg.H * es},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clock_info,
+            "gpu": torch.cuda.get_device_name(dev),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="builder_bf16", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    cfg = CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,204 @@
+/*
+ * moe_b200.h -- C ABI of libmoe_b200.so: the forward pass of one
+ * Mixture-of-Experts layer on one NVIDIA B200 (sm_100a).
+ *
+ * The four stage calls follow the stage contracts of the
+ * DWDP-Triton-MoE-Inference-Engine README: the Router ("Router Module"),
+ * the Dispatcher ("Dispatcher Module"), the Executor ("Executor Module")
+ * and the Merger ("Merger Module"), chained in the order its "Runtime
+ * Integration Layer" section gives.  Each stage reads only what the
+ * previous one wrote.
+ *
+ * Conventions shared by every call
+ *  - Pointers named as device pointers must point to device memory of the
+ *    current CUDA device; tensors are dense and row-major; bf16 means the
+ *    IEEE-like bfloat16 (1-8-7) bit pattern, fp32 means IEEE binary32.
+ *  - The caller owns every buffer.  The library allocates no device memory,
+ *    keeps no pointer after a call returns, and never synchronises the
+ *    stream on these calls.  All work is enqueued on `stream` (a
+ *    cudaStream_t; NULL = the legacy default stream) and runs asynchronously.
+ *  - Return value: MOE_OK, or a moe_status_t describing a host-side
+ *    argument check failure (nothing is enqueued) or a launch failure
+ *    (MOE_ERR_CUDA).  moe_last_error() then gives a one-line message.
+ *  - Errors found on the device (an expert id outside [0, E), an inverse
+ *    permutation entry outside [0, N), a bounded wait that ran out) are
+ *    written to the optional device word `status` (int32, caller-zeroed):
+ *    the first error code stays, later ones do not overwrite it.  Kernels
+ *    never trap: a bad entry is skipped and reported.  moe_read_status()
+ *    copies the word to the host.
+ *  - Sizes: 1 <= T; 1 <= E <= 256; 0 <= k <= min(E, 8) (k = 0 only in
+ *    moe_route, "logits only"); H, I >= 1 with H % 8 == 0 and I % 8 == 0
+ *    (whole 16-byte vectors); the bf16 tensor-core expert path also needs
+ *    H % 256 == 0 and I % 128 == 0, else moe_experts returns
+ *    MOE_ERR_UNSUPPORTED.  Activation and weight tensors must be 16-byte
+ *    aligned; index, weight and status arrays 4-byte aligned.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* bad size, null or misaligned pointer        */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented for this shape    */
+  MOE_ERR_CUDA = 3,         /* a CUDA launch / runtime call failed         */
+  MOE_ERR_TIMEOUT = 4,      /* (device status) a bounded wait ran out      */
+  MOE_ERR_BAD_INDEX = 5     /* (device status) an index was out of range   */
+} moe_status_t;
+
+typedef enum {
+  MOE_F32 = 0,   /* activations, weights and outputs in fp32              */
+  MOE_BF16 = 1   /* activations, weights and outputs in bf16, fp32 inside  */
+} moe_dtype_t;
+
+/* Version of this ABI (bumped on any signature change). */
+int moe_abi_version(void);
+
+/* Message for the last non-OK return on the calling thread ("" if none).
+ * The string stays valid until the next call on this thread. */
+const char* moe_last_error(void);
+
+/*
+ * moe_route -- Router.  DWDP README, "Router Module": router logits, routing
+ * probabilities, top-k expert indices and normalized routing weights;
+ * diffulex.moe API reference, "diffulex.moe.topk" (NaiveTopKRouter, the
+ * standard top-k router).
+ *
+ *   logits[t,e] = sum_h x[t,h] * W_gate[e,h] + bias[e]      (fp32 FMA)
+ *   p[t,:]      = softmax(logits[t,:]) over all E             (fp32)
+ *   topk_ids[t,j], j < k: the k experts with the largest logits, in
+ *               descending order; equal logits -> lower expert id first
+ *   topk_w[t,j] = p[t, topk_ids[t,j]]; if renormalize, divided by the
+ *               sum of the k selected probabilities
+ *
+ *   x        device [T,H] (dtype)          W_gate  device [E,H] (dtype)
+ *   bias     device [E] fp32, or NULL (no bias)
+ *   logits   device [T,E] fp32, written
+ *   topk_ids device [T,k] int32, written (may be NULL when k == 0)
+ *   topk_w   device [T,k] fp32, written  (may be NULL when k == 0)
+ *   k == 0 computes the logits only (e.g. a shared expert's scalar gate
+ *   logit with E == 1).  Inputs are assumed finite.
+ */
+int moe_route(const void* x, const void* W_gate, const float* bias,
+              int T, int H, int E, int k, int renormalize, int dtype,
+              float* logits, int32_t* topk_ids, float* topk_w, void* stream);
+
+/* Bytes of device scratch moe_dispatch needs for (T, k, E). */
+size_t moe_dispatch_workspace_bytes(int T, int k, int E);
+
+/*
+ * moe_dispatch -- Dispatcher.  DWDP README, "Dispatcher Module": converts
+ * token-major routing assignments into an expert-major layout with
+ * per-expert counts, expert offsets, token permutation, inverse permutation,
+ * packed token indices and packed routing weights; plus the Executor's
+ * "gather token activations" step ("Executor Module") into x_packed.
+ *
+ * Assignment f = t*k + j is entry j of token t (row-major [T,k], the flat
+ * order of metrale's ep_dispatch.rs, build_ep_routing_table).  N = T*k.
+ *   counts[e]      number of f with topk_ids[f] == e               [E]
+ *   offsets[e]     exclusive prefix sum of counts; offsets[E] = N  [E+1]
+ *   p(f)           offsets[e] + #{f' < f : topk_ids[f'] == e}  (stable:
+ *                  equal experts keep ascending f, i.e. token order)
+ *   perm[p(f)] = f,  inv_perm[f] = p(f),  packed_tok[p] = perm[p] / k,
+ *   packed_w[p] = topk_w[perm[p]],  x_packed[p,:] = x[packed_tok[p],:]
+ *
+ *   topk_ids device [T,k] int32     topk_w device [T,k] fp32 (or NULL: no
+ *   packed_w output)                 x device [T,H] (dtype), or NULL to
+ *   skip the gather (x_packed then unused)
+ *   counts, offsets, perm, inv_perm, packed_tok  device int32, written
+ *   packed_w  device [N] fp32, written (ignored if topk_w is NULL)
+ *   x_packed  device [N,H] (dtype), written
+ *   ws        device scratch of at least moe_dispatch_workspace_bytes()
+ *   status    device int32 or NULL.  An id outside [0,E) sets
+ *             MOE_ERR_BAD_INDEX; that assignment is left out of every
+ *             output (inv_perm[f] = -1) and offsets[E] < N.
+ */
+int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x,
+                 int T, int H, int E, int k, int dtype,
+                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                 int32_t* packed_tok, float* packed_w, void* x_packed,
+                 void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* Bytes of device scratch moe_experts needs (0 for the current kernels). */
+size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
+
+/*
+ * moe_experts -- Executor.  DWDP README, "Executor Module": for scheduled
+ * expert-major ranges, execute the expert modules, apply routing weights
+ * and write packed expert outputs.  Experts are SwiGLU MLPs whose gate and
+ * up projections are fused in one [E, 2I, H] buffer, gate (w1) in rows
+ * [0, I) and up (w3) in rows [I, 2I) of each expert's slot (the w13_weight
+ * layout of modelexpress-client's test_reshard_refit_moe_experts.py).
+ *
+ * For every expert e and every row p in [offsets[e], offsets[e+1]):
+ *   h[p,i]        = silu(x_packed[p,:] . w13[e,i,:]) * (x_packed[p,:] . w13[e,I+i,:])
+ *   y_packed[p,c] = packed_w[p] * (h[p,:] . w2[e,c,:])
+ * with silu(z) = z / (1 + exp(-z)), fp32 accumulation, and (bf16) h
+ * rounded to bf16 before the second product (it is the operand of a bf16
+ * tensor-core product).  y_packed is always fp32: the merger adds the k
+ * terms of a token before the output's one rounding.
+ *
+ *   x_packed device [N,H]       offsets device [E+1] int32 (read on the
+ *   device; the host never needs the split)
+ *   packed_w device [N] fp32, or NULL for all-ones (e.g. a shared expert)
+ *   w13 device [E,2I,H]         w2 device [E,H,I]
+ *   h        device [N,I] (dtype) scratch, written
+ *   y_packed device [N,H] fp32, written; rows outside every expert's
+ *            range are left untouched
+ *   ws/ws_bytes  device scratch (moe_experts_workspace_bytes; may be NULL/0
+ *            when that is 0)     status device int32 or NULL (timeouts)
+ * offsets must be non-decreasing with offsets[E] <= N (as moe_dispatch
+ * writes them); rows are trusted to lie in [0, N).
+ */
+int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
+                const void* w13, const void* w2, int N, int H, int I, int E, int dtype,
+                void* h, void* y_packed, void* ws, size_t ws_bytes,
+                int32_t* status, void* stream);
+
+/*
+ * moe_combine -- Merger.  DWDP README, "Merger Module": restore token-major
+ * assignment order, accumulate the top-k expert outputs and reshape back to
+ * the token layout.  Routing weights were already applied by moe_experts.
+ *
+ *   out[t,:] = sum_{j=0..k-1} y_packed[inv_perm[t*k+j],:]   (j in order,
+ *              fp32 sum, one rounding to the output type)
+ *            + sigmoid(shared_gate_logit[t]) * shared[t,:]   (if shared)
+ *
+ *   y_packed device [N,H] fp32, N = T*k      inv_perm device [N] int32
+ *   shared   device [T,H] fp32 or NULL (a moe_experts output with E = 1);
+ *            shared_gate_logit device [T] fp32 or NULL (gate 1 when shared
+ *            is given without it): the always-on shared expert of
+ *            diffulex.moe.layer (SharedExpertMLP)
+ *   dtype    type of `out` (MOE_BF16 or MOE_F32)
+ *   out      device [T,H] (dtype), written
+ *   status   device int32 or NULL: an inv_perm entry outside [0,N) sets
+ *            MOE_ERR_BAD_INDEX and contributes nothing.
+ */
+int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,
+                const float* shared, const float* shared_gate_logit, int dtype,
+                void* out, int32_t* status, void* stream);
+
+/* Copy the device status word to *host_status after the stream's prior work
+ * (synchronises `stream`).  Returns MOE_OK or MOE_ERR_CUDA. */
+int moe_read_status(const int32_t* status, void* stream, int32_t* host_status);
+
+/*
+ * moe_probe_wait_timeout -- self-test of the bounded-wait machinery every
+ * persistent kernel here uses.  Launches one CTA that waits on an mbarrier
+ * nothing ever arrives on, with a budget of `budget_us` microseconds
+ * (1..2,000,000); the wait gives up, writes MOE_ERR_TIMEOUT to `status`
+ * (device int32) and the kernel returns normally.  Used by the tests to
+ * check that a wait which runs out is reported, not hung.
+ */
+int moe_probe_wait_timeout(int32_t* status, int budget_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

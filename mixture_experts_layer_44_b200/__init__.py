@@ -1,0 +1,253 @@
+"""Python binding of libmoe_b200.so: one MoE layer's forward pass on a B200.
+
+The functions ``moe_route``, ``moe_dispatch``, ``moe_experts``,
+``moe_combine`` (and the helpers) carry the names of the C ABI in
+``include/moe_b200.h`` and only marshal arguments: every step of the layer
+runs in the library's CUDA kernels.  PyTorch supplies device memory and the
+stream.  There is no fallback: if the library is missing or was built for
+another GPU, the first call raises.
+
+``MoELayerBuffers`` / ``moe_layer_forward`` chain the four stages the way the
+DWDP README's "Runtime Integration Layer" orders them (router -> dispatcher
+-> executor -> merger), with caller-owned buffers allocated once.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MoEError", "lib_path", "load_library", "moe_abi_version", "moe_last_error",
+    "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_experts_workspace_bytes",
+    "moe_experts", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
+    "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
+    "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
+    "KERNELS_PER_LAYER", "moe_layer_forward_host",
+]
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
+MOE_F32, MOE_BF16 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[moe status {code}] {msg}")
+        self.code = code
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libmoe_b200.so")
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "moe_abi_version": (_I, []),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "moe_dispatch_workspace_bytes": (_SZ, [_I, _I, _I]),
+    "moe_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_experts_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "moe_experts": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
+    "moe_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
+    "moe_read_status": (_I, [_P, _P, _P]),
+    "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
+}
+
+# Kernels one moe_layer_forward launches: route 1, dispatch 4 (count, scan,
+# scatter, gather), experts 2 (w13 pass, w2 pass), combine 1.
+KERNELS_PER_LAYER = 8
+
+
+def load_library():
+    """Load libmoe_b200.so (once).  Raises if it is missing: no fallback exists."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m mixture_experts_layer_44_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    if t.dtype == torch.float32:
+        return MOE_F32
+    raise MoEError(MOE_ERR_INVALID_ARG, f"unsupported dtype {t.dtype}")
+
+
+def _check(code: int):
+    if code != MOE_OK:
+        raise MoEError(code, load_library().moe_last_error().decode())
+
+
+def moe_abi_version() -> int:
+    return load_library().moe_abi_version()
+
+
+def moe_last_error() -> str:
+    return load_library().moe_last_error().decode()
+
+
+def moe_route(x, W_gate, bias, k: int, renormalize: bool, logits, topk_ids=None, topk_w=None,
+              stream=None):
+    T, H = x.shape
+    E = W_gate.shape[0]
+    _check(load_library().moe_route(_ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k,
+                                    int(bool(renormalize)), _dtype_code(x), _ptr(logits),
+                                    _ptr(topk_ids), _ptr(topk_w), _stream(stream)))
+
+
+def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
+    return load_library().moe_dispatch_workspace_bytes(T, k, E)
+
+
+def moe_dispatch(topk_ids, topk_w, x, E: int, counts, offsets, perm, inv_perm, packed_tok,
+                 packed_w, x_packed, ws, status=None, stream=None):
+    T, k = topk_ids.shape
+    H = x.shape[1] if x is not None else 0
+    dt = _dtype_code(x) if x is not None else MOE_BF16
+    _check(load_library().moe_dispatch(
+        _ptr(topk_ids), _ptr(topk_w), _ptr(x), T, H, E, k, dt, _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w), _ptr(x_packed),
+        _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _ptr(status),
+        _stream(stream)))
+
+
+def moe_experts_workspace_bytes(N: int, H: int, I: int, E: int, dtype: int) -> int:
+    return load_library().moe_experts_workspace_bytes(N, H, I, E, dtype)
+
+
+def moe_experts(x_packed, offsets, packed_w, w13, w2, h, y_packed, ws=None, status=None,
+                stream=None):
+    N, H = x_packed.shape
+    E = w13.shape[0]
+    I = w13.shape[1] // 2
+    _check(load_library().moe_experts(
+        _ptr(x_packed), _ptr(offsets), _ptr(packed_w), _ptr(w13), _ptr(w2), N, H, I, E,
+        _dtype_code(x_packed), _ptr(h), _ptr(y_packed), _ptr(ws),
+        ws.numel() * ws.element_size() if ws is not None else 0, _ptr(status), _stream(stream)))
+
+
+def moe_combine(y_packed, inv_perm, T: int, k: int, out, shared=None, shared_gate_logit=None,
+                status=None, stream=None):
+    H = out.shape[1]
+    _check(load_library().moe_combine(
+        _ptr(y_packed), _ptr(inv_perm), T, H, k, _ptr(shared), _ptr(shared_gate_logit),
+        _dtype_code(out), _ptr(out), _ptr(status), _stream(stream)))
+
+
+def moe_read_status(status, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(load_library().moe_read_status(_ptr(status), _stream(stream), ctypes.byref(v)))
+    return int(v.value)
+
+
+def moe_probe_wait_timeout(status, budget_us: int, stream=None):
+    _check(load_library().moe_probe_wait_timeout(_ptr(status), budget_us, _stream(stream)))
+
+
+class MoELayerBuffers:
+    """Every device buffer one forward pass of a layer needs, allocated once.
+
+    Shapes follow the ABI: T tokens, N = T*k assignments.  With a shared
+    expert the buffers also hold its packed input/output and gate logit.
+    """
+
+    def __init__(self, T: int, H: int, E: int, k: int, I: int, dtype: torch.dtype,
+                 device="cuda", shared_I: Optional[int] = None):
+        N = T * k
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.T, self.H, self.E, self.k, self.I, self.N = T, H, E, k, I, N
+        self.logits = torch.empty(T, E, **f32)
+        self.ids = torch.empty(T, k, **i32)
+        self.w = torch.empty(T, k, **f32)
+        self.counts = torch.empty(E, **i32)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.perm = torch.empty(N, **i32)
+        self.inv_perm = torch.empty(N, **i32)
+        self.packed_tok = torch.empty(N, **i32)
+        self.packed_w = torch.empty(N, **f32)
+        self.x_packed = torch.empty(N, H, dtype=dtype, device=dev)
+        self.h = torch.empty(N, I, dtype=dtype, device=dev)
+        self.y_packed = torch.empty(N, H, **f32)        # packed expert outputs stay fp32
+        self.out = torch.empty(T, H, dtype=dtype, device=dev)
+        self.ws = torch.empty(max(1, moe_dispatch_workspace_bytes(T, k, E)), dtype=torch.uint8,
+                              device=dev)
+        self.status = torch.zeros(1, **i32)
+        self.shared_I = shared_I
+        if shared_I:
+            self.sg_logit = torch.empty(T, 1, **f32)
+            self.sh_offsets = torch.tensor([0, T], **i32)
+            self.sh_h = torch.empty(T, shared_I, dtype=dtype, device=dev)
+            self.sh_y = torch.empty(T, H, **f32)
+
+
+def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
+                      stream=None):
+    """Router -> dispatcher -> executor -> merger into ``buf.out`` (asynchronous).
+
+    ``params``: W_gate [E,H], bias [E] f32 or None, w13 [E,2I,H], w2 [E,H,I] and,
+    for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].
+    """
+    E = params["W_gate"].shape[0]
+    moe_route(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits, buf.ids,
+              buf.w, stream=stream)
+    moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
+                 buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
+    moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
+                buf.y_packed, status=buf.status, stream=stream)
+    shared = sg = None
+    if params.get("w13s") is not None:
+        moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
+        moe_experts(x, buf.sh_offsets, None, params["w13s"].unsqueeze(0),
+                    params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, status=buf.status,
+                    stream=stream)
+        shared, sg = buf.sh_y, buf.sg_logit
+    moe_combine(buf.y_packed, buf.inv_perm, buf.T, k, buf.out, shared, sg, status=buf.status,
+                stream=stream)
+    return buf.out
+
+
+def moe_layer_forward_host(x_host, params: dict, k: int, renormalize: bool,
+                           buf: MoELayerBuffers, out_host, stream=None):
+    """The same layer called with HOST activations: copy x (pinned host) to the
+    device, run the four stages, copy the output back into ``out_host``
+    (pinned), all on one stream; returns after the copy back is enqueued."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if not hasattr(buf, "x_dev"):
+        buf.x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device=buf.out.device)
+    with torch.cuda.stream(stream):
+        buf.x_dev.copy_(x_host, non_blocking=True)
+        moe_layer_forward(buf.x_dev, params, k, renormalize, buf, stream=stream)
+        out_host.copy_(buf.out, non_blocking=True)
+    return out_host

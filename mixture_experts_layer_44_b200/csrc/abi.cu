@@ -1,0 +1,207 @@
+// extern "C" entry points of libmoe_b200.so (declared in include/moe_b200.h):
+// host-side argument checks, then the stage launchers.  No call allocates
+// device memory or synchronises the stream (except moe_read_status).
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  g_err = std::string(where) + ": " + cudaGetErrorString(e);
+  return MOE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+#define REQ(cond, code, msg)                 \
+  do {                                       \
+    if (!(cond)) return fail(code, msg);   \
+  } while (0)
+
+int check_dtype(int dtype) {
+  if (dtype != MOE_F32 && dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "dtype must be MOE_F32 (0) or MOE_BF16 (1)");
+  return MOE_OK;
+}
+
+// Bounded-wait self-test: one thread waits on an mbarrier nothing arrives on.
+__global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = moe::smem_addr(&bar);
+  moe::mbar_init(b, 1);
+  moe::fence_barrier_init();
+  if (!moe::mbar_wait(b, 0, budget_ns)) moe::report(status, MOE_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+namespace moe_host {
+cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s) {
+  probe_wait_kernel<<<1, 32, 0, s>>>(status, static_cast<uint64_t>(budget_us) * 1000ull);
+  return cudaGetLastError();
+}
+}  // namespace moe_host
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+int moe_route(const void* x, const void* W_gate, const float* bias, int T, int H, int E, int k,
+              int renormalize, int dtype, float* logits, int32_t* topk_ids, float* topk_w,
+              void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(x && W_gate && logits, MOE_ERR_INVALID_ARG, "moe_route: null x, W_gate or logits");
+  REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_route: T and H must be >= 1");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_route: E must be in [1, 256]");
+  REQ(k >= 0 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
+      "moe_route: k must be in [0, min(E, 8)]");
+  REQ(k == 0 || (topk_ids && topk_w), MOE_ERR_INVALID_ARG, "moe_route: null topk_ids or topk_w");
+  REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_route: H must be a multiple of 8");
+  REQ(aligned16(x) && aligned16(W_gate), MOE_ERR_INVALID_ARG,
+      "moe_route: x and W_gate must be 16-byte aligned");
+  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias),
+      MOE_ERR_INVALID_ARG, "moe_route: outputs and bias must be 4-byte aligned");
+  REQ(static_cast<long long>(T) * (H > E ? H : E) < (1ll << 31), MOE_ERR_INVALID_ARG,
+      "moe_route: T*H too large");
+  cudaError_t e = moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
+                                         logits, topk_ids, topk_w,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+}
+
+size_t moe_dispatch_workspace_bytes(int T, int k, int E) {
+  if (T < 1 || k < 1 || E < 1) return 0;
+  return moe_host::dispatch_ws_bytes(T, k, E);
+}
+
+int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x, int T, int H, int E,
+                 int k, int dtype, int32_t* counts, int32_t* offsets, int32_t* perm,
+                 int32_t* inv_perm, int32_t* packed_tok, float* packed_w, void* x_packed,
+                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(topk_ids && counts && offsets && perm && inv_perm && packed_tok, MOE_ERR_INVALID_ARG,
+      "moe_dispatch: null ids or output");
+  REQ(!topk_w || packed_w, MOE_ERR_INVALID_ARG, "moe_dispatch: topk_w given but packed_w is null");
+  REQ(T >= 1, MOE_ERR_INVALID_ARG, "moe_dispatch: T must be >= 1");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_dispatch: E must be in [1, 256]");
+  REQ(k >= 1 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
+      "moe_dispatch: k must be in [1, min(E, 8)]");
+  REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG, "moe_dispatch: T*k too large");
+  REQ(aligned4(topk_ids) && aligned4(topk_w) && aligned4(counts) && aligned4(offsets) &&
+          aligned4(perm) && aligned4(inv_perm) && aligned4(packed_tok) && aligned4(packed_w),
+      MOE_ERR_INVALID_ARG, "moe_dispatch: index arrays must be 4-byte aligned");
+  REQ(aligned4(status), MOE_ERR_INVALID_ARG, "moe_dispatch: status must be 4-byte aligned");
+  if (x) {
+    REQ(x_packed, MOE_ERR_INVALID_ARG, "moe_dispatch: x given but x_packed is null");
+    REQ(H >= 1 && H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_dispatch: H must be a positive multiple of 8");
+    REQ(aligned16(x) && aligned16(x_packed), MOE_ERR_INVALID_ARG,
+        "moe_dispatch: x and x_packed must be 16-byte aligned");
+    REQ(static_cast<long long>(T) * k * H < (1ll << 40), MOE_ERR_INVALID_ARG,
+        "moe_dispatch: T*k*H too large");
+  }
+  const size_t need = moe_host::dispatch_ws_bytes(T, k, E);
+  REQ(ws && ws_bytes >= need && aligned16(ws), MOE_ERR_INVALID_ARG,
+      "moe_dispatch: workspace missing, misaligned or smaller than moe_dispatch_workspace_bytes()");
+  cudaError_t e = moe_host::launch_dispatch(topk_ids, topk_w, x, T, H, E, k, dtype, counts,
+                                            offsets, perm, inv_perm, packed_tok, packed_w,
+                                            x_packed, ws, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch launch");
+}
+
+size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype) {
+  (void)N; (void)H; (void)I; (void)E; (void)dtype;
+  return 0;
+}
+
+int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
+                const void* w13, const void* w2, int N, int H, int I, int E, int dtype, void* h,
+                void* y_packed, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  g_err.clear();
+  (void)ws; (void)ws_bytes;
+  if (int r = check_dtype(dtype)) return r;
+  REQ(N >= 0, MOE_ERR_INVALID_ARG, "moe_experts: N must be >= 0");
+  if (N == 0) return MOE_OK;
+  REQ(x_packed && offsets && w13 && w2 && h && y_packed, MOE_ERR_INVALID_ARG,
+      "moe_experts: null input or output");
+  REQ(H >= 1 && I >= 1, MOE_ERR_INVALID_ARG, "moe_experts: H and I must be >= 1");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_experts: E must be in [1, 256]");
+  REQ(H % 8 == 0 && I % 8 == 0, MOE_ERR_INVALID_ARG, "moe_experts: H and I must be multiples of 8");
+  REQ(aligned16(x_packed) && aligned16(w13) && aligned16(w2) && aligned16(h) && aligned16(y_packed),
+      MOE_ERR_INVALID_ARG, "moe_experts: tensors must be 16-byte aligned");
+  REQ(aligned4(offsets) && aligned4(packed_w) && aligned4(status), MOE_ERR_INVALID_ARG,
+      "moe_experts: offsets / packed_w / status must be 4-byte aligned");
+  REQ(static_cast<long long>(N) * (H > I ? H : I) < (1ll << 40) && N < (1 << 30),
+      MOE_ERR_INVALID_ARG, "moe_experts: N too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == MOE_BF16) {
+    REQ(H % 256 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
+        "moe_experts: the bf16 tensor-core path needs H % 256 == 0 and I % 128 == 0");
+    const char* why = "";
+    e = moe_host::launch_experts_tc(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h, y_packed,
+                                    status, s, &why);
+    if (e != cudaSuccess && why[0]) return fail(MOE_ERR_CUDA, std::string("moe_experts: ") + why);
+  } else {
+    e = moe_host::launch_experts_simt(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h,
+                                      y_packed, s);
+  }
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_experts launch");
+}
+
+int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,
+                const float* shared, const float* shared_gate_logit, int dtype, void* out,
+                int32_t* status, void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(y_packed && inv_perm && out, MOE_ERR_INVALID_ARG, "moe_combine: null y_packed, inv_perm or out");
+  REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_combine: T and H must be >= 1");
+  REQ(k >= 1 && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG, "moe_combine: k must be in [1, 8]");
+  REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_combine: H must be a multiple of 8");
+  REQ(aligned16(y_packed) && aligned16(out) && aligned16(shared), MOE_ERR_INVALID_ARG,
+      "moe_combine: y_packed, shared and out must be 16-byte aligned");
+  REQ(aligned4(inv_perm) && aligned4(shared_gate_logit) && aligned4(status), MOE_ERR_INVALID_ARG,
+      "moe_combine: inv_perm / gate / status must be 4-byte aligned");
+  REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG, "moe_combine: T*k too large");
+  cudaError_t e = moe_host::launch_combine(y_packed, inv_perm, T, H, k, shared, shared_gate_logit,
+                                           dtype, out, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
+}
+
+int moe_read_status(const int32_t* status, void* stream, int32_t* host_status) {
+  g_err.clear();
+  REQ(status && host_status, MOE_ERR_INVALID_ARG, "moe_read_status: null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(host_status, status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_read_status");
+}
+
+int moe_probe_wait_timeout(int32_t* status, int budget_us, void* stream) {
+  g_err.clear();
+  REQ(status && aligned4(status), MOE_ERR_INVALID_ARG, "moe_probe_wait_timeout: bad status pointer");
+  REQ(budget_us >= 1 && budget_us <= 2000000, MOE_ERR_INVALID_ARG,
+      "moe_probe_wait_timeout: budget_us must be in [1, 2000000]");
+  cudaError_t e = moe_host::launch_probe_wait_timeout(status, budget_us,
+                                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_probe_wait_timeout launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// Merger: inverse-permutation gather-reduce back to token order.
+//
+// DWDP-Triton-MoE-Inference-Engine README, "Merger Module": restore
+// token-major assignment order, accumulate the top-k expert outputs, reshape
+// to the token layout.  out[t] = sum_{j<k} y_packed[inv_perm[t*k+j]] in j
+// order with an fp32 accumulator (deterministic: no atomics), plus
+// sigmoid(gate_logit[t]) * shared[t] for the always-on shared expert
+// (diffulex.moe.layer, SharedExpertMLP).
+//
+// y_packed and the shared expert's output are fp32 (the executor keeps its
+// packed outputs in fp32), so the k terms and the shared term are added in
+// fp32 and rounded once, to the output type.
+//
+// One CTA per token at a time (grid-stride over tokens); each thread owns
+// 16-byte vectors of the hidden dimension, so every load and store is a
+// 128-bit access.  The k source rows of a token are independent loads that
+// are all in flight together.
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int CNT = 256;
+
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ y,
+                                                      const int32_t* __restrict__ inv_perm,
+                                                      int T, int H, int k, int N,
+                                                      const float* __restrict__ shared,
+                                                      const float* __restrict__ sgate,
+                                                      void* __restrict__ outv, int32_t* status) {
+  const int nvec = H / 8;                               // 8 outputs per thread step
+  __shared__ int rows[moe::kMaxTopK];
+  __shared__ float gate;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < k) {
+      int p = inv_perm[static_cast<size_t>(t) * k + threadIdx.x];
+      if (p < 0 || p >= N) {
+        moe::report(status, MOE_ERR_BAD_INDEX);
+        p = -1;
+      }
+      rows[threadIdx.x] = p;
+    }
+    if (threadIdx.x == 0) gate = shared ? (sgate ? 1.f / (1.f + expf(-sgate[t])) : 1.f) : 0.f;
+    __syncthreads();
+    for (int v = threadIdx.x; v < nvec; v += CNT) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int j = 0; j < k; ++j) {
+        const int p = rows[j];
+        if (p < 0) continue;
+        const float4* src = reinterpret_cast<const float4*>(y + static_cast<size_t>(p) * H) + 2 * v;
+        const float4 a = src[0], b = src[1];
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+      if (shared) {
+        const float g = gate;
+        const float4* src = reinterpret_cast<const float4*>(shared + static_cast<size_t>(t) * H) + 2 * v;
+        const float4 a = src[0], b = src[1];
+        acc[0] = fmaf(g, a.x, acc[0]); acc[1] = fmaf(g, a.y, acc[1]);
+        acc[2] = fmaf(g, a.z, acc[2]); acc[3] = fmaf(g, a.w, acc[3]);
+        acc[4] = fmaf(g, b.x, acc[4]); acc[5] = fmaf(g, b.y, acc[5]);
+        acc[6] = fmaf(g, b.z, acc[6]); acc[7] = fmaf(g, b.w, acc[7]);
+      }
+      if (OUT_BF16) {
+        reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(outv) + static_cast<size_t>(t) * H)[v] =
+            make_uint4(moe::pack_bf16x2(acc[0], acc[1]), moe::pack_bf16x2(acc[2], acc[3]),
+                       moe::pack_bf16x2(acc[4], acc[5]), moe::pack_bf16x2(acc[6], acc[7]));
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(outv) + static_cast<size_t>(t) * H) + 2 * v;
+        dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+namespace moe_host {
+
+cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
+                           const float* shared, const float* shared_gate, int dtype, void* out,
+                           int32_t* status, cudaStream_t s) {
+  const int grid = std::max(1, std::min(T, num_sms() * 8));
+  const int N = T * k;
+  if (dtype == MOE_BF16)
+    combine_kernel<true><<<grid, CNT, 0, s>>>(y, inv_perm, T, H, k, N, shared, shared_gate, out,
+                                              status);
+  else
+    combine_kernel<false><<<grid, CNT, 0, s>>>(y, inv_perm, T, H, k, N, shared, shared_gate, out,
+                                               status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe_host

@@ -1,0 +1,77 @@
+// Shared helpers of the libmoe_b200 kernels: status codes, bf16 conversion,
+// vector types and the bounded-wait clock.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// Largest sizes the kernels are written for (checked on the host).
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 8;
+
+// Budget of every bounded wait in a kernel (nanoseconds).  A correct kernel
+// waits microseconds at most; the budget only bounds a wait that would
+// otherwise never end, after which the kernel reports MOE_ERR_TIMEOUT.
+constexpr uint64_t kWaitBudgetNs = 2000ull * 1000ull * 1000ull;
+
+// Record the first device-side error in the caller's status word.
+__device__ __forceinline__ void report(int32_t* status, int32_t code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Unpack 8 bf16 (one 16-byte vector) into floats.
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+}  // namespace moe
+
+// Host-side internal launchers (one translation unit each).  They assume the
+// arguments were validated by the ABI layer and return a cudaError_t.
+namespace moe_host {
+cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, int T, int H,
+                         int E, int k, int renormalize, int dtype, float* logits,
+                         int32_t* ids, float* w, cudaStream_t s);
+size_t dispatch_ws_bytes(int T, int k, int E);
+cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, int T, int H,
+                            int E, int k, int dtype, int32_t* counts, int32_t* offsets,
+                            int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
+                            float* packed_w, void* x_packed, void* ws, int32_t* status,
+                            cudaStream_t s);
+cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
+                              const float* packed_w, const void* w13, const void* w2, int N,
+                              int H, int I, int E, void* h, void* y, int32_t* status,
+                              cudaStream_t s, const char** why);
+cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
+                                const float* packed_w, const void* w13, const void* w2, int N,
+                                int H, int I, int E, void* h, void* y, cudaStream_t s);
+cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
+                           const float* shared, const float* shared_gate, int dtype, void* out,
+                           int32_t* status, cudaStream_t s);
+cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s);
+int num_sms();
+}  // namespace moe_host

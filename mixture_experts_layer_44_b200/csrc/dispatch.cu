@@ -1,0 +1,280 @@
+// Dispatcher: token-major routing assignments -> expert-major layout.
+//
+// DWDP-Triton-MoE-Inference-Engine README, "Dispatcher Module": per-expert
+// counts, expert offsets, token permutation, inverse permutation, packed
+// token indices, packed routing weights; "Executor Module": gather token
+// activations for the expert ranges.  Assignment f = t*k + j (row-major
+// [T, k], the flat order of metrale's ep_dispatch.rs).
+//
+// Four launches:
+//   count   -- each CTA owns CHUNK consecutive assignments; each warp owns a
+//              contiguous CHUNK/8 slice and counts it per expert with
+//              __match_any_sync (one shared-memory add per distinct expert
+//              in a 32-lane round, no atomics); CTA totals go to ws[b][e].
+//   scan    -- one CTA: counts[e] = sum_b ws[b][e], offsets = exclusive scan
+//              over e, and ws[b][e] becomes the first position CTA b writes
+//              for expert e.
+//   scatter -- each CTA recounts its slice per warp, turns the counts into
+//              per-warp bases, and walks its assignments in order; inside a
+//              round a lane's rank among equal experts is the popcount of
+//              the lower lanes in its match mask.  Positions therefore grow
+//              with f inside an expert: the order is stable (bit-exact).
+//   gather  -- x_packed[p] = x[packed_tok[p]] with bulk asynchronous copies
+//              (global -> shared -> global on the TMA engine), one issuing
+//              lane per warp, a 4-row ring per warp.
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int CHUNK = 2048;        // assignments per CTA
+constexpr int DNT = 256;           // threads per CTA
+constexpr int DWARPS = DNT / 32;
+constexpr int PER_WARP = CHUNK / DWARPS;
+
+// Per-warp per-expert counts of this CTA's slice.  Invalid ids (outside
+// [0,E)) are reported and skipped.  wc: [DWARPS][E] in shared memory.
+__device__ __forceinline__ void warp_counts(const int32_t* __restrict__ ids, int N, int E,
+                                            int base, int* wc, int32_t* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < DWARPS * E; i += DNT) wc[i] = 0;
+  __syncthreads();
+  const int w0 = base + warp * PER_WARP;
+  for (int r = 0; r < PER_WARP; r += 32) {
+    const int f = w0 + r + lane;
+    int e = -1;
+    if (f < N) {
+      e = ids[f];
+      if (e < 0 || e >= E) {
+        moe::report(status, MOE_ERR_BAD_INDEX);
+        e = -1;
+      }
+    }
+    const unsigned valid = __ballot_sync(0xffffffffu, e >= 0);
+    // Lanes without a valid id get a unique key so they never match.
+    const int key = e >= 0 ? e : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers & valid);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* __restrict__ ids,
+                                                             int N, int E,
+                                                             int32_t* __restrict__ bc,
+                                                             int32_t* status) {
+  extern __shared__ int wc[];
+  warp_counts(ids, N, E, blockIdx.x * CHUNK, wc, status);
+  for (int e = threadIdx.x; e < E; e += DNT) {
+    int s = 0;
+#pragma unroll
+    for (int w = 0; w < DWARPS; ++w) s += wc[w * E + e];
+    bc[static_cast<size_t>(blockIdx.x) * E + e] = s;
+  }
+}
+
+// One CTA of 256 threads (E <= 256).
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict__ bc, int B,
+                                                            int E, int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int s_scan[256];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int b = 0; b < B; ++b) total += bc[static_cast<size_t>(b) * E + e];
+  // Exclusive scan over experts (Hillis-Steele on 256 entries).
+  s_scan[e] = total;
+  __syncthreads();
+  for (int o = 1; o < 256; o <<= 1) {
+    const int v = e >= o ? s_scan[e - o] : 0;
+    __syncthreads();
+    s_scan[e] += v;
+    __syncthreads();
+  }
+  const int excl = s_scan[e] - total;
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = excl;
+    int run = excl;
+    for (int b = 0; b < B; ++b) {
+      const size_t i = static_cast<size_t>(b) * E + e;
+      const int c = bc[i];
+      bc[i] = run;
+      run += c;
+    }
+  }
+  if (e == 255) offsets[E] = s_scan[255];
+}
+
+__global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int N, int E, int k,
+    const int32_t* __restrict__ bc, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+    int32_t* __restrict__ packed_tok, float* __restrict__ packed_w, int32_t* status) {
+  extern __shared__ int wc[];  // [DWARPS][E] counts, then bases
+  const int base = blockIdx.x * CHUNK;
+  warp_counts(ids, N, E, base, wc, nullptr);
+  for (int e = threadIdx.x; e < E; e += DNT) {
+    int run = bc[static_cast<size_t>(blockIdx.x) * E + e];
+#pragma unroll
+    for (int ww = 0; ww < DWARPS; ++ww) {
+      const int c = wc[ww * E + e];
+      wc[ww * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int w0 = base + warp * PER_WARP;
+  for (int r = 0; r < PER_WARP; r += 32) {
+    const int f = w0 + r + lane;
+    int e = -1;
+    if (f < N) {
+      e = ids[f];
+      if (e < 0 || e >= E) {
+        e = -1;
+        inv_perm[f] = -1;
+      }
+    }
+    const int key = e >= 0 ? e : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (e >= 0) {
+      const int p = wc[warp * E + e] + __popc(peers & lt);
+      perm[p] = f;
+      inv_perm[f] = p;
+      packed_tok[p] = f / k;
+      if (packed_w) packed_w[p] = w[f];
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------- gather ---
+
+constexpr int GW = 4;      // warps per CTA, each an independent copy engine client
+constexpr int GSLOTS = 4;  // rows in flight per warp
+
+__global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
+    const uint8_t* __restrict__ x, const int32_t* __restrict__ packed_tok,
+    const int32_t* __restrict__ offsets, int E, int row_bytes, uint8_t* __restrict__ xp,
+    int32_t* status) {
+  extern __shared__ __align__(128) uint8_t gsm[];
+  __shared__ __align__(8) uint64_t bars[GW][GSLOTS];
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) != 0) return;
+  uint8_t* ring = gsm + static_cast<size_t>(warp) * GSLOTS * row_bytes;
+  for (int s = 0; s < GSLOTS; ++s) moe::mbar_init(moe::smem_addr(&bars[warp][s]), 1);
+  moe::fence_barrier_init();
+
+  const int nrows = offsets[E];            // valid rows (assignments with a valid id)
+  const int stride = gridDim.x * GW;
+  const int first = blockIdx.x * GW + warp;
+  const int mine = first < nrows ? (nrows - first + stride - 1) / stride : 0;
+  auto issue = [&](int i) {
+    const int p = first + i * stride;
+    const int s = i % GSLOTS;
+    const uint32_t bar = moe::smem_addr(&bars[warp][s]);
+    moe::mbar_arrive_expect_tx(bar, row_bytes);
+    moe::bulk_g2s(moe::smem_addr(ring + static_cast<size_t>(s) * row_bytes),
+                  x + static_cast<size_t>(packed_tok[p]) * row_bytes, row_bytes, bar);
+  };
+  const int prologue = mine < GSLOTS ? mine : GSLOTS;
+  for (int i = 0; i < prologue; ++i) issue(i);
+  for (int i = 0; i < mine; ++i) {
+    const int s = i % GSLOTS;
+    const int p = first + i * stride;
+    if (!moe::mbar_wait(moe::smem_addr(&bars[warp][s]), (i / GSLOTS) & 1)) {
+      moe::report(status, MOE_ERR_TIMEOUT);
+      // Let every load already issued land before the CTA leaves.
+      const int last = mine < i + GSLOTS ? mine : i + GSLOTS;
+      for (int j = i + 1; j < last; ++j)
+        moe::mbar_wait(moe::smem_addr(&bars[warp][j % GSLOTS]), (j / GSLOTS) & 1);
+      break;
+    }
+    moe::bulk_s2g(xp + static_cast<size_t>(p) * row_bytes,
+                  moe::smem_addr(ring + static_cast<size_t>(s) * row_bytes), row_bytes);
+    moe::bulk_commit();
+    if (i + GSLOTS < mine) {
+      moe::bulk_wait_read_all();   // this slot's store has read its bytes
+      issue(i + GSLOTS);
+    }
+  }
+  moe::bulk_wait_all();
+}
+
+// Rows too large for the shared-memory ring: one warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ packed_tok,
+    const int32_t* __restrict__ offsets, int E, int row_vecs, uint4* __restrict__ xp) {
+  const int nrows = offsets[E];
+  const int lane = threadIdx.x & 31;
+  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < nrows;
+       p += (gridDim.x * blockDim.x) >> 5) {
+    const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
+    uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
+    for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+  }
+}
+
+}  // namespace
+
+namespace moe_host {
+
+size_t dispatch_ws_bytes(int T, int k, int E) {
+  const size_t N = static_cast<size_t>(T) * k;
+  const size_t B = (N + CHUNK - 1) / CHUNK;
+  return std::max<size_t>(B * E * sizeof(int32_t), 256);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, int T, int H,
+                            int E, int k, int dtype, int32_t* counts, int32_t* offsets,
+                            int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
+                            float* packed_w, void* x_packed, void* ws, int32_t* status,
+                            cudaStream_t s) {
+  const int N = T * k;
+  const int B = (N + CHUNK - 1) / CHUNK;
+  int32_t* bc = static_cast<int32_t*>(ws);
+  const size_t wsm = sizeof(int) * DWARPS * E;
+  dispatch_count_kernel<<<B, DNT, wsm, s>>>(ids, N, E, bc, status);
+  dispatch_scan_kernel<<<1, 256, 0, s>>>(bc, B, E, counts, offsets);
+  dispatch_scatter_kernel<<<B, DNT, wsm, s>>>(ids, w, N, E, k, bc, perm, inv_perm, packed_tok,
+                                              w ? packed_w : nullptr, status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess || x == nullptr) return err;
+  const int es = dtype == MOE_BF16 ? 2 : 4;
+  const int row_bytes = H * es;
+  const size_t gsm = static_cast<size_t>(GW) * GSLOTS * row_bytes;
+  if (gsm > 200 * 1024) {
+    const int grid = std::max(1, std::min((N + 7) / 8, num_sms() * 8));
+    dispatch_gather_vec_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), packed_tok,
+                                                     offsets, E, row_bytes / 16,
+                                                     static_cast<uint4*>(x_packed));
+    return cudaGetLastError();
+  }
+  err = cudaFuncSetAttribute(dispatch_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gsm));
+  if (err != cudaSuccess) return err;
+  const int ctas_per_sm = std::max(1, static_cast<int>((200 * 1024) / gsm));
+  const int grid = std::max(1, std::min((N + GW - 1) / GW, num_sms() * ctas_per_sm));
+  dispatch_gather_kernel<<<grid, GW * 32, gsm, s>>>(static_cast<const uint8_t*>(x), packed_tok,
+                                                     offsets, E, row_bytes,
+                                                     static_cast<uint8_t*>(x_packed), status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe_host

@@ -1,0 +1,419 @@
+// Executor, bf16: persistent grouped GEMM on the 5th-generation tensor cores.
+//
+// DWDP-Triton-MoE-Inference-Engine README, "Executor Module": execute the
+// expert modules over expert-major ranges, apply routing weights, write
+// packed expert outputs.  Experts are SwiGLU MLPs with the fused gate/up
+// buffer w13 [E, 2I, H] (gate w1 rows [0,I), up w3 rows [I,2I): the
+// w13_weight layout of modelexpress-client's test_reshard_refit_moe_experts.py)
+// and w2 [E, H, I].
+//
+// Two launches of one kernel template:
+//   pass 1 (EPI_SWIGLU): A = x_packed [N,H], B = w13[e];
+//                        h[p, f] = silu(gate) * up   (bf16 out)
+//   pass 2 (EPI_SCALE):  A = h [N,I],        B = w2[e];
+//                        y_packed[p, c] = packed_w[p] * acc  (fp32 out, so the
+//                        merger adds the k terms before the one bf16 rounding)
+//
+// Tile = 128 packed rows (tokens of one expert; MMA M) x 256 weight rows
+// (MMA N) x the whole K.  In pass 1 the 256 weight rows are 128 gate rows and
+// the 128 matching up rows (one 3-D TMA box over [2E, I, H]), so column c and
+// column 128 + c of the accumulator are the gate and up value of the same
+// feature and the SwiGLU is thread-local.  The tile list is derived on the
+// device from `offsets` (the scheduler of the README's "Scheduler Module",
+// folded into the kernel): expert e owns ceil(count_e / 128) token tiles x
+// (rows / 256) weight tiles, token tiles fastest, so CTAs running at the same
+// time share a weight tile through L2.  Experts with no rows own no tiles.
+//
+// CTA = 6 warps, one CTA per SM, persistent over tiles:
+//   warp 0   TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
+//   warp 1   MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
+//   warps 2-5 epilogue      (tcgen05.ld from the TMEM accumulator, math, store)
+// The two 256-column fp32 accumulators are double-buffered in TMEM, so the
+// epilogue of one tile overlaps the MMAs of the next.  Every wait is bounded;
+// a wait that runs out reports MOE_ERR_TIMEOUT, the CTA drains what it issued
+// and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NTHREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
+
+enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int offs[moe::kMaxExperts + 1];
+  int tstart[moe::kMaxExperts + 1];   // first tile of expert e (tiles = token tiles x NTW)
+};
+
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+
+struct TileCoord {
+  int e, nt, mt;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const Ctl& c, int E, int ntw, int t) {
+  // largest e with tstart[e] <= t (experts without tiles share their successor's start)
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (c.tstart[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  const int e = lo;
+  const int mte = (c.offs[e + 1] - c.offs[e] + BM - 1) / BM;
+  const int local = t - c.tstart[e];
+  TileCoord r;
+  r.e = e;
+  r.nt = local / mte;
+  r.mt = local - r.nt * mte;
+  (void)ntw;
+  return r;
+}
+
+__device__ __forceinline__ void set_abort(Ctl& c, int32_t* status) {
+  moe::report(status, MOE_ERR_TIMEOUT);
+  *reinterpret_cast<volatile int*>(&c.abort) = 1;
+}
+
+__device__ __forceinline__ bool aborted(const Ctl& c) {
+  return *reinterpret_cast<const volatile int*>(&c.abort) != 0;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB,
+                        const int32_t* __restrict__ offsets, int E, int K, int ntw,
+                        int rows_per_expert, const float* __restrict__ packed_w,
+                        void* __restrict__ out, int ldo, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      moe::mbar_init(moe::smem_addr(&c.full[s]), 1);
+      moe::mbar_init(moe::smem_addr(&c.empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      moe::mbar_init(moe::smem_addr(&c.tfull[b]), 1);
+      moe::mbar_init(moe::smem_addr(&c.tempty[b]), 4);
+    }
+    moe::mbar_init(moe::smem_addr(&c.drain), 1);
+    c.abort = 0;
+    moe::fence_barrier_init();
+    moe::prefetch_tmap(&tmA);
+    moe::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
+    moe::tmem_relinquish();
+  }
+  if (warp == 2) {
+    // Tile table: per-expert token-tile counts, exclusive scan, x ntw.
+    // Lane l owns experts [8l, 8l+8); lane 31 also writes the end entries.
+    int cnt[8];
+    int local = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      int m = 0;
+      if (e < E) {
+        c.offs[e] = offsets[e];
+        m = (offsets[e + 1] - offsets[e] + BM - 1) / BM;
+      }
+      cnt[j] = m;
+      local += m;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) c.tstart[e] = run * ntw;
+      run += cnt[j];
+    }
+    if (lane == 31) {
+      c.offs[E] = offsets[E];
+      c.tstart[E] = incl * ntw;
+    }
+  }
+  moe::tc_fence_before();
+  __syncthreads();
+  moe::tc_fence_after();
+
+  const int total = c.tstart[E];
+  const int kblocks = K / BK;
+  const uint32_t tmem = c.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ producer ---
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[STAGES] = {0, 0, 0, 0};
+      for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x) {
+        const TileCoord tc = decode_tile(c, E, ntw, t);
+        const int arow = c.offs[tc.e] + tc.mt * BM;
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
+            set_abort(c, status);
+            ok = false;
+            break;
+          }
+          const uint32_t fb = moe::smem_addr(&c.full[stage]);
+          const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
+          moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          moe::tma_load_2d(sa, &tmA, fb, kb * BK, arow);
+          if (EPI == EPI_SWIGLU)
+            moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, tc.nt * (BN / 2), 2 * tc.e);
+          else
+            moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, tc.e * rows_per_expert + tc.nt * BN);
+          ++issued[stage];
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      // Drain: every load issued has landed before the CTA can leave.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > 0) moe::mbar_wait(moe::smem_addr(&c.full[s]), (issued[s] - 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA ---
+      int stage = 0;
+      uint32_t phase = 0;
+      int i = 0;
+      for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
+          set_abort(c, status);
+          break;
+        }
+        moe::tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
+        bool ok = true;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase)) {
+            set_abort(c, status);
+            ok = false;
+            break;
+          }
+          moe::tc_fence_after();
+          const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = moe::sw128_kmajor_desc(sa + kk * 32);
+            const uint64_t bd = moe::sw128_kmajor_desc(sa + A_BYTES + kk * 32);
+            moe::tc_mma_f16(d, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          moe::tc_commit(moe::smem_addr(&c.empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        moe::tc_commit(moe::smem_addr(&c.tfull[buf]));
+      }
+      // Drain: all MMAs this thread issued have completed.
+      moe::tc_commit(moe::smem_addr(&c.drain));
+      moe::mbar_wait(moe::smem_addr(&c.drain), 0);
+    }
+  } else {
+    // ------------------------------------------------------- epilogue ---
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;          // row of the tile owned by this thread
+    int i = 0;
+    for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x, ++i) {
+      const int buf = i & 1;
+      if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1)) {
+        set_abort(c, status);
+        break;
+      }
+      moe::tc_fence_after();
+      const TileCoord tc = decode_tile(c, E, ntw, t);
+      const int rows_valid = c.offs[tc.e + 1] - c.offs[tc.e] - tc.mt * BM;
+      const bool live = row < rows_valid;
+      const size_t grow = static_cast<size_t>(c.offs[tc.e] + tc.mt * BM + row);
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(buf * BN);
+      if (EPI == EPI_SWIGLU) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + grow * ldo + tc.nt * (BN / 2);
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 2; cc += 16) {
+          uint32_t g[16], u[16];
+          moe::tmem_ld16(taddr + cc, g);
+          moe::tmem_ld16(taddr + BN / 2 + cc, u);
+          moe::tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
+            const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
+            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+            pk[j] = moe::pack_bf16x2(h0, h1);
+          }
+          if (live) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+        const float sc = live ? (packed_w ? packed_w[grow] : 1.f) : 0.f;
+        float* dst = static_cast<float*>(out) + grow * ldo + tc.nt * BN;
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          uint32_t a[16], b[16];
+          moe::tmem_ld16(taddr + cc, a);
+          moe::tmem_ld16(taddr + cc + 16, b);
+          moe::tmem_ld_wait();
+          if (live) {
+            float4* d4 = reinterpret_cast<float4*>(dst + cc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              d4[j] = make_float4(__uint_as_float(a[4 * j]) * sc, __uint_as_float(a[4 * j + 1]) * sc,
+                                  __uint_as_float(a[4 * j + 2]) * sc, __uint_as_float(a[4 * j + 3]) * sc);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              d4[4 + j] = make_float4(__uint_as_float(b[4 * j]) * sc, __uint_as_float(b[4 * j + 1]) * sc,
+                                      __uint_as_float(b[4 * j + 2]) * sc, __uint_as_float(b[4 * j + 3]) * sc);
+          }
+        }
+      }
+      moe::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
+    }
+  }
+
+  moe::tc_fence_before();
+  __syncthreads();
+  moe::tc_fence_after();
+  if (warp == 1) moe::tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------ tensor maps ---
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  auto fn = get_encode();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+                  strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Activations [rows, K] bf16, box 64 x 128.
+bool map_rows(CUtensorMap* m, const void* p, int rows, int K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {BK, BM};
+  return encode(m, p, 2, dims, str, box);
+}
+
+}  // namespace
+
+namespace moe_host {
+
+cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
+                              const float* packed_w, const void* w13, const void* w2, int N,
+                              int H, int I, int E, void* h, void* y, int32_t* status,
+                              cudaStream_t s, const char** why) {
+  cudaError_t e1 = cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(SMEM_BYTES));
+  if (e1 != cudaSuccess) return e1;
+  e1 = cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                            static_cast<int>(SMEM_BYTES));
+  if (e1 != cudaSuccess) return e1;
+  CUtensorMap mA1, mB1, mA2, mB2;
+  bool ok = map_rows(&mA1, x_packed, N, H) && map_rows(&mA2, h, N, I);
+  {
+    // w13 as [2E][I][H]: one box = 128 gate rows + the matching 128 up rows.
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
+                                static_cast<cuuint64_t>(2) * E};
+    const cuuint64_t str[2] = {static_cast<cuuint64_t>(H) * 2,
+                               static_cast<cuuint64_t>(I) * H * 2};
+    const cuuint32_t box[3] = {BK, BN / 2, 2};
+    ok = ok && encode(&mB1, w13, 3, dims, str, box);
+  }
+  {
+    // w2 as [E*H][I]
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(E) * H};
+    const cuuint64_t str[1] = {static_cast<cuuint64_t>(I) * 2};
+    const cuuint32_t box[2] = {BK, BN};
+    ok = ok && encode(&mB2, w2, 2, dims, str, box);
+  }
+  if (!ok) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
+    return cudaErrorInvalidValue;
+  }
+  const int mt_bound = (N + BM - 1) / BM + E;
+  const int ntw1 = I / (BN / 2);
+  const int ntw2 = H / BN;
+  const int sms = num_sms();
+  const int g1 = std::max(1, std::min(sms, mt_bound * ntw1));
+  const int g2 = std::max(1, std::min(sms, mt_bound * ntw2));
+  grouped_gemm_kernel<EPI_SWIGLU><<<g1, NTHREADS, SMEM_BYTES, s>>>(
+      mA1, mB1, offsets, E, H, ntw1, 2 * I, nullptr, h, I, status);
+  grouped_gemm_kernel<EPI_SCALE><<<g2, NTHREADS, SMEM_BYTES, s>>>(
+      mA2, mB2, offsets, E, I, ntw2, H, packed_w, y, H, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe_host

@@ -1,0 +1,129 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import mixture_experts_layer_44_b200 as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(M.lib_path()):
+        from mixture_experts_layer_44_b200 import build
+        build.build()
+    return M.load_library()
+
+
+def test_header_declares_the_stage_calls():
+    names = _declared()
+    for n in ("moe_route", "moe_dispatch", "moe_experts", "moe_combine",
+              "moe_dispatch_workspace_bytes", "moe_experts_workspace_bytes", "moe_read_status",
+              "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", M.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", out, flags=re.M))
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_library_is_built_for_sm100a_only():
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", M.lib_path()],
+                         capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+    assert "sm_90" not in out and "sm_80" not in out
+
+
+def test_abi_version_and_workspace_queries(lib):
+    assert M.moe_abi_version() == 1
+    ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
+    assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
+    assert M.moe_dispatch_workspace_bytes(0, 2, 8) == 0
+    assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_BF16) == 0
+
+
+NULL = None
+P = ctypes.c_void_p(16)   # an aligned non-null address that is never dereferenced
+
+
+def _err(lib):
+    return lib.moe_last_error().decode()
+
+
+def test_route_rejects_bad_arguments_on_the_host(lib):
+    r = lib.moe_route(P, P, NULL, 0, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "T and H" in _err(lib)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 9, 1, M.MOE_BF16, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "k must be" in _err(lib)
+    r = lib.moe_route(P, P, NULL, 4, 64, 300, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "E must be" in _err(lib)
+    r = lib.moe_route(P, P, NULL, 4, 60, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "multiple of 8" in _err(lib)
+    r = lib.moe_route(ctypes.c_void_p(24), P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "aligned" in _err(lib)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, 7, P, P, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG and "dtype" in _err(lib)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, NULL, P, NULL)
+    assert r == M.MOE_ERR_INVALID_ARG
+
+
+def test_dispatch_rejects_bad_arguments_on_the_host(lib):
+    args = [P, P, P, 4, 64, 8, 2, M.MOE_BF16, P, P, P, P, P, P, P, P, 4096, NULL, NULL]
+    a = list(args); a[6] = 0
+    assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(args); a[15] = NULL          # ws missing
+    assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "workspace" in _err(lib)
+    a = list(args); a[16] = 4             # ws too small
+    assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(args); a[14] = NULL          # x given but no x_packed
+    assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "x_packed" in _err(lib)
+    a = list(args); a[13] = NULL          # topk_w given but no packed_w
+    assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG
+
+
+def test_experts_rejects_bad_arguments_on_the_host(lib):
+    base = [P, P, P, P, P, 100, 256, 128, 4, M.MOE_BF16, P, P, NULL, 0, NULL, NULL]
+    a = list(base); a[6] = 200            # H not a multiple of 256 on the bf16 path
+    assert lib.moe_experts(*a) == M.MOE_ERR_UNSUPPORTED and "H % 256" in _err(lib)
+    a = list(base); a[7] = 100            # I not a multiple of 8
+    assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[8] = 0
+    assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[5] = 0              # nothing to do: OK without touching the GPU
+    assert lib.moe_experts(*a) == M.MOE_OK
+    a = list(base); a[3] = NULL
+    assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+
+
+def test_combine_and_status_reject_bad_arguments_on_the_host(lib):
+    assert lib.moe_combine(P, P, 4, 64, 0, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(P, P, 4, 63, 2, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(NULL, P, 4, 64, 2, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    v = ctypes.c_int32(0)
+    assert lib.moe_read_status(NULL, NULL, ctypes.byref(v)) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_probe_wait_timeout(P, 0, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_probe_wait_timeout(P, 3_000_000, NULL) == M.MOE_ERR_INVALID_ARG
+
+
+def test_python_binding_raises_with_the_library_message(lib):
+    import torch
+    x = torch.empty(0, 64)
+    with pytest.raises(M.MoEError, match="moe_route: "):
+        M.moe_route(x, torch.empty(8, 64), None, 2, True, torch.empty(0, 8), stream=0)

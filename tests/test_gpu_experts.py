@@ -1,0 +1,104 @@
+"""Executor parity: GPU moe_experts against the oracle's experts().
+
+Same x_packed, offsets and packed_w on both sides.  bf16 path (tcgen05):
+y_packed (fp32) within 2e-2 of the fp64 oracle (max |err| / rms) and h (a
+bf16 tensor) within 2e-2 beyond its own final rounding; fp32 path: both
+within 1e-5.  Shapes span several tiles, ragged tails, empty experts and
+rows beyond the last expert's range (which must stay untouched).
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_44_b200 as M
+import oracle.moe_oracle as O
+from tests.gpu_util import DEV, TOL, dev, err_bf16_out, rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _make(counts, H, I, dtype, seed=0, N=None, with_w=True):
+    g = torch.Generator().manual_seed(seed)
+    E = len(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    N = int(offs[-1]) if N is None else N
+    x = torch.randn(N, H, generator=g).to(dtype)
+    w13 = (torch.randn(E, 2 * I, H, generator=g) / H ** 0.5).to(dtype)
+    w2 = (torch.randn(E, H, I, generator=g) / I ** 0.5).to(dtype)
+    pw = torch.rand(N, generator=g) if with_w else None
+    return x, torch.tensor(offs), pw, w13, w2
+
+
+def _run(x, offs, pw, w13, w2, canary=True):
+    N, H = x.shape
+    I = w13.shape[1] // 2
+    fill = 1234.5 if canary else 0.0
+    h = torch.full((N, I), fill, dtype=x.dtype, device=DEV)
+    y = torch.full((N, H), fill, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    M.moe_experts(dev(x), dev(offs), dev(pw), dev(w13), dev(w2), h, y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return h.cpu(), y.cpu()
+
+
+def _check(x, offs, pw, w13, w2, tol):
+    h, y = _run(x, offs, pw, w13, w2)
+    hn = int(offs[-1])
+    ho, yo = O.experts(x[:hn], offs.numpy(), None if pw is None else pw[:hn], w13, w2)
+    eh = err_bf16_out(h[:hn], ho) if h.dtype == torch.bfloat16 else rel(h[:hn], ho)
+    assert eh <= tol, eh
+    assert y.dtype == torch.float32
+    assert rel(y[:hn], yo) <= tol, rel(y[:hn], yo)
+    # rows outside every expert's range are untouched
+    assert (h[hn:].float() == 1234.5).all() and (y[hn:].float() == 1234.5).all()
+    return h, y
+
+
+@pytest.mark.parametrize("counts,H,I", [
+    ([0, 1, 127, 300], 256, 128),            # empty, single row, one short of a tile, ragged
+    ([200], 512, 256),                       # one expert, K loop wraps the 4-stage ring
+    ([0, 0, 5], 256, 128),                   # N below one tile: TMA zero-fills past N
+    ([128, 128, 256, 0, 129], 768, 384),     # exact tiles, then one row over
+])
+def test_experts_bf16_tiles(counts, H, I):
+    _check(*_make(counts, H, I, torch.bfloat16, seed=sum(counts)), tol=TOL["bf16"])
+
+
+def test_experts_bf16_many_tiles_per_cta():
+    rng = np.random.default_rng(0)
+    counts = rng.multinomial(16384, rng.dirichlet(np.ones(8)))
+    _check(*_make(list(counts), 512, 512, torch.bfloat16, seed=1), tol=TOL["bf16"])
+
+
+def test_experts_bf16_rows_beyond_last_expert_untouched():
+    x, offs, pw, w13, w2 = _make([40, 0, 250], 256, 128, torch.bfloat16, seed=3, N=300)
+    _check(x, offs, pw, w13, w2, tol=TOL["bf16"])
+
+
+def test_experts_bf16_unit_weights_for_a_shared_expert():
+    x, offs, _, w13, w2 = _make([333], 256, 256, torch.bfloat16, seed=4, with_w=False)
+    _check(x, offs, None, w13, w2, tol=TOL["bf16"])
+
+
+def test_experts_bf16_qwen3_shape_slice():
+    # I = 768, H = 2048 (the Qwen3-30B-A3B expert shape) with a skewed split
+    counts = [900, 0, 37, 260, 1, 0, 0, 130]
+    _check(*_make(counts, 2048, 768, torch.bfloat16, seed=5), tol=TOL["bf16"])
+
+
+@pytest.mark.parametrize("counts,H,I", [
+    ([10, 30, 0, 24, 16, 8, 40, 0], 128, 256),   # the tiny fp32 workload's shape
+    ([65, 0, 3], 72, 40),                        # ragged H, I vs the 64 x 64 x 16 tiles
+    ([1], 8, 8),
+])
+def test_experts_f32_simt(counts, H, I):
+    _check(*_make(counts, H, I, torch.float32, seed=sum(counts) + H), tol=TOL["f32"])
+
+
+def test_experts_deterministic():
+    args = _make([300, 17, 0, 500], 512, 256, torch.bfloat16, seed=7)
+    h1, y1 = _run(*args)
+    h2, y2 = _run(*args)
+    assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))

@@ -1,0 +1,106 @@
+"""Router parity: GPU moe_route against the fp64 oracle.
+
+Logits (fp32) within 1e-5 of the oracle's fp64 logits (relative to their
+RMS).  Given the GPU's own logits, the oracle's top-k ids must match bit for
+bit and its weights within 1e-5 relative, element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_layer_44_b200 as M
+import oracle.moe_oracle as O
+from moe_inputs import CONFIGS, LayerConfig, make_layer
+from tests.gpu_util import DEV, dev, rel
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, W, b, k, renorm):
+    T, E = x.shape[0], W.shape[0]
+    logits = torch.empty(T, E, device=DEV)
+    ids = torch.empty(T, max(k, 1), dtype=torch.int32, device=DEV)
+    w = torch.empty(T, max(k, 1), device=DEV)
+    M.moe_route(dev(x), dev(W), dev(b), k, renorm, logits, ids if k else None, w if k else None)
+    torch.cuda.synchronize()
+    return logits.cpu(), ids.cpu()[:, :k], w.cpu()[:, :k]
+
+
+def _check(x, W, b, k, renorm, logit_tol=1e-5):
+    logits, ids, w = _run(x, W, b, k, renorm)
+    l64 = O.router_logits(x, W, b)
+    assert rel(logits, l64) <= logit_tol
+    if k == 0:
+        return
+    ids_o, w_o = O.route_from_logits(logits, k, renorm)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    np.testing.assert_allclose(w.numpy(), w_o, rtol=1e-5, atol=0)
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "builder_bf16", "qwen15_t32", "qwen3_t16384",
+                                  "decode_t1", "decode_t64"])
+def test_route_configs(name):
+    cfg = CONFIGS[name]
+    # Router-only draw: the expert weights are not needed here, so draw a
+    # narrow layer with the same T, H, E, k and bias recipe.
+    small = LayerConfig("r", T=cfg.T, H=cfg.H, E=cfg.E, k=cfg.k, I=8, dtype=cfg.dtype,
+                        renormalize=cfg.renormalize, zipf_s=cfg.zipf_s, empty_tail=cfg.empty_tail)
+    p = make_layer(small, seed=0)
+    _check(p["x"], p["W_gate"], p["bias"], cfg.k, cfg.renormalize)
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (3, 2), (8, 8), (60, 4), (64, 2), (65, 3), (128, 8),
+                                 (200, 5), (256, 8)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("H", [72, 96])
+def test_route_shapes(E, k, dtype, H):
+    cfg = LayerConfig("r", T=131, H=H, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 2 == 0))
+    p = make_layer(cfg, seed=E + k)
+    _check(p["x"], p["W_gate"], None, k, cfg.renormalize)
+
+
+def test_route_with_bias_and_no_renorm():
+    rng = np.random.default_rng(5)
+    x = torch.randn(77, 256, generator=torch.Generator().manual_seed(1))
+    W = torch.randn(40, 256, generator=torch.Generator().manual_seed(2)) / 16
+    b = torch.tensor(rng.standard_normal(40), dtype=torch.float32)
+    _check(x, W, b, 6, False)
+
+
+def test_route_ties_go_to_lower_expert_id():
+    # Duplicate W_gate rows give bit-identical logits: the lower id must win.
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(50, 64, generator=g)
+    W = torch.randn(16, 64, generator=g)
+    W[9] = W[2]
+    W[12] = W[2]
+    W[5] = W[14]
+    logits, ids, _ = _run(x, W, None, 4, True)
+    assert torch.equal(logits[:, 9], logits[:, 2]) and torch.equal(logits[:, 12], logits[:, 2])
+    ids_o, _ = O.route_from_logits(logits, 4, True)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    for t in range(50):
+        row = ids[t].tolist()
+        if 9 in row or 12 in row:
+            assert 2 in row and row.index(2) < row.index(9 if 9 in row else 12)
+    # All-equal logits: ids are 0..k-1 in order, weights uniform.
+    logits, ids, w = _run(torch.zeros(3, 64), torch.randn(10, 64, generator=g), None, 3, True)
+    assert ids.tolist() == [[0, 1, 2]] * 3
+    np.testing.assert_allclose(w.numpy(), 1 / 3, rtol=1e-6)
+
+
+def test_route_logits_only_for_a_shared_gate():
+    g = torch.Generator().manual_seed(4)
+    x = torch.randn(33, 128, generator=g).to(torch.bfloat16)
+    wsg = (torch.randn(1, 128, generator=g) / 11).to(torch.bfloat16)
+    _check(x, wsg, None, 0, False)
+
+
+def test_route_k_equals_E_is_the_full_softmax():
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(20, 64, generator=g)
+    W = torch.randn(8, 64, generator=g) / 8
+    logits, ids, w = _run(x, W, None, 8, False)
+    full = torch.zeros(20, 8)
+    full.scatter_(1, ids.long(), w)
+    np.testing.assert_allclose(full.numpy(), O.softmax_rows(O.to_f64(logits)), rtol=1e-5)
