@@ -109,6 +109,48 @@ def ncu_traffic(workload):
     return d.get("per_step_bytes", {}).get(workload)
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest ``value`` over all ranks (torch.distributed MAX all-reduce);
+    the value itself when no process group is initialised."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_inputs(cfg, rank: int) -> dict:
+    """One replica's layer: the same seeded weights on every rank, and the
+    workload's own tokens on rank 0, a fresh seeded batch on rank r > 0."""
+    p = make_layer(cfg, seed=0)
+    if rank > 0:
+        p["x"] = make_tokens(cfg, seed=rank)
+    return p
+
+
+def parse_clock_samples(text: str) -> dict:
+    """Median SM clock, max clock and the throttle reasons seen in
+    ``nvidia-smi --query-gpu=...`` CSV rows (the ClockSampler query)."""
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in text.strip().splitlines():
+        f = [x.strip() for x in line.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1]))
+            smax.append(float(f[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, f[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while timing."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -143,23 +185,7 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return parse_clock_samples(out)
 
 
 # ---------------------------------------------------------- CPU oracle ---
@@ -239,9 +265,7 @@ def run_gpu(args, cfg):
     M.load_library()
     dev = torch.device("cuda", local)
 
-    p = make_layer(cfg, seed=0)
-    if rank > 0:
-        p["x"] = make_tokens(cfg, seed=rank)
+    p = rank_inputs(cfg, rank)
     dp = {k: (v.to(dev) if v is not None else None) for k, v in p.items()}
     buf = M.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.torch_dtype, device=dev,
                             shared_I=cfg.shared_I)
@@ -306,12 +330,7 @@ def run_gpu(args, cfg):
     step_ms = [sum(s) for s in stage_ms]
     ms = sum(step_ms) / args.steps
     per_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(4)]
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    else:
-        ms_max = ms
+    ms_max = max_over_ranks(ms, dev)
 
     # End to end through the public API with host buffers: pinned x in, out back.
     x_host = p["x"].pin_memory()
@@ -331,10 +350,7 @@ def run_gpu(args, cfg):
         e_end.synchronize()
         e2e_ms_list.append(e_start.elapsed_time(e_end))
     e2e_ms = sum(e2e_ms_list) / len(e2e_ms_list)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     if int(buf.status.item()) != 0:
         raise SystemExit(f"device status {int(buf.status.item())} after timing")
 
@@ -401,10 +417,17 @@ def main():
     ap.add_argument("--workload", default="builder_bf16", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="the workload with E=16 experts and T=1024 tokens (weights 0.55 GB, "
+                         "still above L2): the case detailed ncu captures run on")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     cfg = CONFIGS[args.workload]
+    if args.profile_small:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, name=cfg.name + "_e16_t1024", E=min(cfg.E, 16),
+                                  T=min(cfg.T, 1024))
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_gpu(args, cfg)

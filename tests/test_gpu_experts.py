@@ -32,7 +32,7 @@ def _make(counts, H, I, dtype, seed=0, N=None, with_w=True):
 def _run(x, offs, pw, w13, w2, canary=True):
     N, H = x.shape
     I = w13.shape[1] // 2
-    fill = 1234.5 if canary else 0.0
+    fill = 1536.0 if canary else 0.0
     h = torch.full((N, I), fill, dtype=x.dtype, device=DEV)
     y = torch.full((N, H), fill, dtype=torch.float32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
@@ -51,7 +51,7 @@ def _check(x, offs, pw, w13, w2, tol):
     assert y.dtype == torch.float32
     assert rel(y[:hn], yo) <= tol, rel(y[:hn], yo)
     # rows outside every expert's range are untouched
-    assert (h[hn:].float() == 1234.5).all() and (y[hn:].float() == 1234.5).all()
+    assert (h[hn:].float() == 1536.0).all() and (y[hn:].float() == 1536.0).all()
     return h, y
 
 
