@@ -125,6 +125,36 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x,
                  int32_t* packed_tok, float* packed_w, void* x_packed,
                  void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
+/*
+ * moe_dispatch_noalloc -- moe_dispatch for callers that cannot allocate
+ * device memory at the point where they dispatch: a C host program whose GPU
+ * memory is carved up by someone else, a plugin of a framework that does not
+ * expose its allocator, or a serving loop that forbids allocation once it is
+ * running.  The pages have no counterpart; it exists only so that such a
+ * caller needs no workspace.
+ *
+ * Same arguments, outputs, ordering and status reporting as moe_dispatch,
+ * without `ws` / `ws_bytes`: the per-block count table lives in one fixed
+ * array of the library (a file-scope __device__ array of 128 KiB that every
+ * GPU which loads the library holds until the process exits).  The call
+ * allocates nothing.
+ *   - Limit: ceil(T*k / 2048) * E <= 32768 (e.g. T*k <= 524288 at E = 128);
+ *     larger problems return MOE_ERR_INVALID_ARG with a message naming the
+ *     limit.  Use moe_dispatch with a workspace for them.
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, then cached), so make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Two calls whose work overlaps
+ *     on the GPU (different streams, or different host threads) race on it:
+ *     order them on one stream.
+ */
+int moe_dispatch_noalloc(const int32_t* topk_ids, const float* topk_w, const void* x,
+                         int T, int H, int E, int k, int dtype,
+                         int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                         int32_t* packed_tok, float* packed_w, void* x_packed,
+                         int32_t* status, void* stream);
+
 /* Bytes of device scratch moe_experts needs (0 for the current kernels). */
 size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
 

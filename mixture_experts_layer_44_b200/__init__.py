@@ -21,7 +21,8 @@ import torch
 
 __all__ = [
     "MoEError", "lib_path", "load_library", "moe_abi_version", "moe_last_error",
-    "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_experts_workspace_bytes",
+    "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_dispatch_noalloc",
+    "moe_experts_workspace_bytes",
     "moe_experts", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
@@ -55,6 +56,7 @@ _SIGS = {
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "moe_dispatch_workspace_bytes": (_SZ, [_I, _I, _I]),
     "moe_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_dispatch_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_experts_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_experts": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
     "moe_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
@@ -138,6 +140,20 @@ def moe_dispatch(topk_ids, topk_w, x, E: int, counts, offsets, perm, inv_perm, p
         _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w), _ptr(x_packed),
         _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _ptr(status),
         _stream(stream)))
+
+
+def moe_dispatch_noalloc(topk_ids, topk_w, x, E: int, counts, offsets, perm, inv_perm,
+                         packed_tok, packed_w, x_packed, status=None, stream=None):
+    """moe_dispatch without a workspace, for callers that cannot allocate: the
+    count table lives in a fixed array inside the library (limit
+    ceil(T*k/2048)*E <= 32768).  Calls that overlap on the GPU race on it."""
+    T, k = topk_ids.shape
+    H = x.shape[1] if x is not None else 0
+    dt = _dtype_code(x) if x is not None else MOE_BF16
+    _check(load_library().moe_dispatch_noalloc(
+        _ptr(topk_ids), _ptr(topk_w), _ptr(x), T, H, E, k, dt, _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w), _ptr(x_packed),
+        _ptr(status), _stream(stream)))
 
 
 def moe_experts_workspace_bytes(N: int, H: int, I: int, E: int, dtype: int) -> int:

@@ -50,6 +50,8 @@ __global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
 }  // namespace
 
 namespace moe_host {
+void set_last_error(const std::string& msg) { g_err = msg; }
+
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s) {
   probe_wait_kernel<<<1, 32, 0, s>>>(status, static_cast<uint64_t>(budget_us) * 1000ull);
   return cudaGetLastError();

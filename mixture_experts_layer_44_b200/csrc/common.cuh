@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <string>
+
 #include "../../include/moe_b200.h"
 
 namespace moe {
@@ -74,4 +76,5 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
                            int32_t* status, cudaStream_t s);
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s);
 int num_sms();
+void set_last_error(const std::string& msg);   // the message moe_last_error() returns
 }  // namespace moe_host

@@ -23,6 +23,8 @@
 //              (global -> shared -> global on the TMA engine), one issuing
 //              lane per warp, a 4-row ring per warp.
 #include <algorithm>
+#include <mutex>
+#include <string>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -278,3 +280,83 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
 }
 
 }  // namespace moe_host
+
+// ----------------------------------------------- allocation-free variant ---
+//
+// moe_dispatch_noalloc runs the same four kernels as moe_dispatch, but its
+// per-CTA count table lives in the fixed array below instead of a
+// caller-allocated workspace.  It is for callers that cannot call
+// cudaMalloc (or any allocator) at the point where they dispatch: a C host
+// program whose device memory is carved up by someone else, a plugin of a
+// framework that does not expose its allocator, or a serving loop that
+// forbids allocation after start-up.  Every GPU that loads this library
+// holds the array (128 KiB) until the process exits.
+
+namespace {
+constexpr int kNoAllocScratchInts = 32768;   // 128 KiB: ceil(T*k / 2048) * E entries
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocScratchInts];
+
+namespace {
+
+// Device address of g_dispatch_scratch on the current device.  In host code
+// the array's name only stands in for the symbol; the address a kernel may
+// use comes from cudaGetSymbolAddress, called once per device (with that
+// device current) and cached.
+cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* cached[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = p;
+  }
+  *out = cached[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int moe_dispatch_noalloc(const int32_t* topk_ids, const float* topk_w, const void* x,
+                                    int T, int H, int E, int k, int dtype, int32_t* counts,
+                                    int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                                    int32_t* packed_tok, float* packed_w, void* x_packed,
+                                    int32_t* status, void* stream) {
+  moe_host::set_last_error("");
+  if (T < 1 || k < 1 || E < 1 || E > moe::kMaxExperts || k > E || k > moe::kMaxTopK) {
+    moe_host::set_last_error("moe_dispatch_noalloc: need T >= 1, 1 <= k <= min(E, 8), 1 <= E <= 256");
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(T) * k >= (1ll << 30)) {
+    moe_host::set_last_error("moe_dispatch_noalloc: T*k too large");
+    return MOE_ERR_INVALID_ARG;
+  }
+  const size_t need = moe_host::dispatch_ws_bytes(T, k, E);
+  if (need > sizeof(int32_t) * kNoAllocScratchInts) {
+    moe_host::set_last_error(
+        "moe_dispatch_noalloc: ceil(T*k/2048)*E = " + std::to_string(need / sizeof(int32_t)) +
+        " count entries exceed the fixed scratch of 32768 (128 KiB); use moe_dispatch with a "
+        "workspace");
+    return MOE_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) {
+    moe_host::set_last_error(std::string("moe_dispatch_noalloc: cudaGetSymbolAddress: ") +
+                             cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  // The remaining argument checks and the launches are those of moe_dispatch
+  // (which sets moe_last_error() itself).
+  return moe_dispatch(topk_ids, topk_w, x, T, H, E, k, dtype, counts, offsets, perm, inv_perm,
+                      packed_tok, packed_w, x_packed, scratch,
+                      sizeof(int32_t) * kNoAllocScratchInts, status, stream);
+}
