@@ -7,7 +7,9 @@
 One step = route -> dispatch -> experts -> combine over one batch of the
 workload (default: the 64-expert builder layer, T=4096, H=4096, top-2,
 I=1408, bf16, Zipf(1.0)-skewed load), with inputs resident in HBM.  L2 is
-flushed (a 256 MiB write) before every timed step, outside the timed events.
+flushed before every timed step, outside the timed events: a 256 MiB write,
+then a read of the same buffer, so that the timed step does not start by
+writing back a cache full of dirty lines.
 Each stage is bracketed by CUDA events on the launching stream, so the
 per-stage times and the grouped-GEMM roofline come from the same timed
 steps.  N > 1 (torchrun, one rank per GPU) runs independent replicas of the
@@ -238,7 +240,7 @@ def run_reference(args, cfg):
 def workload_config(cfg, counts):
     c = {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.k, "I": cfg.I,
          "renormalize": cfg.renormalize, "zipf_s": cfg.zipf_s, "empty_experts_forced": cfg.empty_tail,
-         "shared_I": cfg.shared_I, "seed": 0, "l2": "flushed: 256 MiB write before every timed step",
+         "shared_I": cfg.shared_I, "seed": 0, "l2": "flushed before every timed step: 256 MiB write, then read back",
          "parallelism": "replicas (one independent layer per GPU)"}
     if counts is not None:
         c["expert_counts"] = [int(x) for x in counts]
@@ -290,12 +292,12 @@ def run_gpu(args, cfg):
         if ev:
             ev[2].record(stream)
         M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
-                      buf.y_packed, status=buf.status, stream=stream)
+                      buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
         if shared:
             M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
             M.moe_experts(x, buf.sh_offsets, None, dp["w13s"].unsqueeze(0),
-                          dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, status=buf.status,
-                          stream=stream)
+                          dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
+                          status=buf.status, stream=stream)
         if ev:
             ev[3].record(stream)
         M.moe_combine(buf.y_packed, buf.inv_perm, cfg.T, cfg.k, buf.out,
@@ -304,8 +306,12 @@ def run_gpu(args, cfg):
         if ev:
             ev[4].record(stream)
 
+    def flush_l2():
+        flush.zero_()                 # write > L2 ...
+        flush.sum()                   # ... then read it, leaving clean lines only
+
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2()
         step()
     torch.cuda.synchronize(dev)
     if int(buf.status.item()) != 0:
@@ -319,9 +325,15 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.3)
-    for i in range(args.steps):
-        flush.zero_()
-        step(evs[i])
+    # Steps are enqueued in groups behind a short GPU spin (outside every timed
+    # bracket), so the GPU runs each group back to back and no stage bracket
+    # contains time spent waiting for the host to issue the next launch.
+    GROUP = 8
+    for g0 in range(0, args.steps, GROUP):
+        torch.cuda._sleep(int(20e6))            # ~10 ms of GPU spin while the host enqueues
+        for i in range(g0, min(args.steps, g0 + GROUP)):
+            flush_l2()
+            step(evs[i])
     torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
     if dist:
@@ -343,7 +355,7 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     e2e_ms_list = []
     for _ in range(e2e_steps):
-        flush.zero_()
+        flush_l2()
         e_start.record(stream)
         M.moe_layer_forward_host(x_host, dp, cfg.k, cfg.renormalize, buf, out_host, stream=stream)
         e_end.record(stream)

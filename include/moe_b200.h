@@ -155,7 +155,8 @@ int moe_dispatch_noalloc(const int32_t* topk_ids, const float* topk_w, const voi
                          int32_t* packed_tok, float* packed_w, void* x_packed,
                          int32_t* status, void* stream);
 
-/* Bytes of device scratch moe_experts needs (0 for the current kernels). */
+/* Bytes of device scratch moe_experts can use (bf16 path: per-tile counters
+ * plus 128 KiB partial slots, 4 per SM; fp32 path: 0). */
 size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
 
 /*
@@ -181,8 +182,13 @@ size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
  *   h        device [N,I] (dtype) scratch, written
  *   y_packed device [N,H] fp32, written; rows outside every expert's
  *            range are left untouched
- *   ws/ws_bytes  device scratch (moe_experts_workspace_bytes; may be NULL/0
- *            when that is 0)     status device int32 or NULL (timeouts)
+ *   ws/ws_bytes  device scratch of moe_experts_workspace_bytes() bytes,
+ *            ZERO-FILLED before its first use (the kernels leave it zeroed
+ *            again; re-zero it after a MOE_ERR_TIMEOUT).  With it, a pass with
+ *            fewer tiles than two per SM splits K and reduces the fp32
+ *            partials in a fixed order (deterministic).  NULL / 0 is allowed:
+ *            no split.  Calls that share one ws must not overlap on the GPU.
+ *   status   device int32 or NULL (timeouts)
  * offsets must be non-decreasing with offsets[E] <= N (as moe_dispatch
  * writes them); rows are trusted to lie in [0, N).
  */

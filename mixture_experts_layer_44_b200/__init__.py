@@ -218,6 +218,10 @@ class MoELayerBuffers:
         self.out = torch.empty(T, H, dtype=dtype, device=dev)
         self.ws = torch.empty(max(1, moe_dispatch_workspace_bytes(T, k, E)), dtype=torch.uint8,
                               device=dev)
+        # zero-filled once; the split-K counters return to zero after every call
+        self.ws_experts = torch.zeros(
+            max(16, moe_experts_workspace_bytes(N, H, I, E, MOE_BF16 if dtype == torch.bfloat16
+                                                else MOE_F32)), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
         self.shared_I = shared_I
         if shared_I:
@@ -240,13 +244,13 @@ def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerB
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
     moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
-                buf.y_packed, status=buf.status, stream=stream)
+                buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
     shared = sg = None
     if params.get("w13s") is not None:
         moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
         moe_experts(x, buf.sh_offsets, None, params["w13s"].unsqueeze(0),
-                    params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, status=buf.status,
-                    stream=stream)
+                    params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
+                    status=buf.status, stream=stream)
         shared, sg = buf.sh_y, buf.sg_logit
     moe_combine(buf.y_packed, buf.inv_perm, buf.T, k, buf.out, shared, sg, status=buf.status,
                 stream=stream)

@@ -4,7 +4,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
 #include <string>
+#include <tuple>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -51,6 +54,21 @@ __global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
 
 namespace moe_host {
 void set_last_error(const std::string& msg) { g_err = msg; }
+
+cudaError_t ensure_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*>, int> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_tuple(dev, kernel);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
 
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s) {
   probe_wait_kernel<<<1, 32, 0, s>>>(status, static_cast<uint64_t>(budget_us) * 1000ull);
@@ -129,15 +147,14 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x, in
 }
 
 size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype) {
-  (void)N; (void)H; (void)I; (void)E; (void)dtype;
-  return 0;
+  (void)N; (void)H; (void)I; (void)E;
+  return dtype == MOE_BF16 ? moe_host::experts_ws_bytes() : 0;
 }
 
 int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
                 const void* w13, const void* w2, int N, int H, int I, int E, int dtype, void* h,
                 void* y_packed, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   g_err.clear();
-  (void)ws; (void)ws_bytes;
   if (int r = check_dtype(dtype)) return r;
   REQ(N >= 0, MOE_ERR_INVALID_ARG, "moe_experts: N must be >= 0");
   if (N == 0) return MOE_OK;
@@ -150,6 +167,7 @@ int moe_experts(const void* x_packed, const int32_t* offsets, const float* packe
       MOE_ERR_INVALID_ARG, "moe_experts: tensors must be 16-byte aligned");
   REQ(aligned4(offsets) && aligned4(packed_w) && aligned4(status), MOE_ERR_INVALID_ARG,
       "moe_experts: offsets / packed_w / status must be 4-byte aligned");
+  REQ(aligned16(ws), MOE_ERR_INVALID_ARG, "moe_experts: ws must be 16-byte aligned");
   REQ(static_cast<long long>(N) * (H > I ? H : I) < (1ll << 40) && N < (1 << 30),
       MOE_ERR_INVALID_ARG, "moe_experts: N too large");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -159,7 +177,7 @@ int moe_experts(const void* x_packed, const int32_t* offsets, const float* packe
         "moe_experts: the bf16 tensor-core path needs H % 256 == 0 and I % 128 == 0");
     const char* why = "";
     e = moe_host::launch_experts_tc(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h, y_packed,
-                                    status, s, &why);
+                                    ws, ws_bytes, status, s, &why);
     if (e != cudaSuccess && why[0]) return fail(MOE_ERR_CUDA, std::string("moe_experts: ") + why);
   } else {
     e = moe_host::launch_experts_simt(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h,

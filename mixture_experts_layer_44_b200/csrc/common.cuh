@@ -64,10 +64,11 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
                             int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
                             float* packed_w, void* x_packed, void* ws, int32_t* status,
                             cudaStream_t s);
+size_t experts_ws_bytes();
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, int32_t* status,
-                              cudaStream_t s, const char** why);
+                              int H, int I, int E, void* h, void* y, void* ws, size_t ws_bytes,
+                              int32_t* status, cudaStream_t s, const char** why);
 cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
                                 const float* packed_w, const void* w13, const void* w2, int N,
                                 int H, int I, int E, void* h, void* y, cudaStream_t s);
@@ -77,4 +78,6 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s);
 int num_sms();
 void set_last_error(const std::string& msg);   // the message moe_last_error() returns
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel, size).
+cudaError_t ensure_smem(const void* kernel, int bytes);
 }  // namespace moe_host

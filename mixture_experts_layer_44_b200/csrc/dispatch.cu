@@ -6,7 +6,10 @@
 // activations for the expert ranges.  Assignment f = t*k + j (row-major
 // [T, k], the flat order of metrale's ep_dispatch.rs).
 //
-// Four launches:
+// Small batches (N <= 8192 assignments) take one CTA of 32 warps through
+// count, scan and scatter in a single launch (the same warp-slice algorithm
+// as below), and also gather the rows when they total at most 1 MiB (decode);
+// larger gathers use the bulk-copy kernel.  Larger N takes four launches:
 //   count   -- each CTA owns CHUNK consecutive assignments; each warp owns a
 //              contiguous CHUNK/8 slice and counts it per expert with
 //              __match_any_sync (one shared-memory add per distinct expert
@@ -155,6 +158,101 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
   }
 }
 
+// ------------------------------------------------- single-CTA variant ---
+
+constexpr int SMALL_WARPS = 32;
+constexpr int SMALL_PER_WARP = 256;
+constexpr int SMALL_N = SMALL_WARPS * SMALL_PER_WARP;   // 8192 assignments
+
+__global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, const float* __restrict__ w, int N, int E, int k,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, int32_t* __restrict__ packed_tok,
+    float* __restrict__ packed_w, const uint4* __restrict__ x, int row_vecs,
+    uint4* __restrict__ xp, int32_t* status) {
+  extern __shared__ int wc[];                  // [SMALL_WARPS][E]
+  __shared__ int s_scan[moe::kMaxExperts];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i = threadIdx.x; i < SMALL_WARPS * E; i += blockDim.x) wc[i] = 0;
+  __syncthreads();
+  const int per = (N + SMALL_WARPS - 1) / SMALL_WARPS;
+  const int w0 = warp * per, w1 = min(N, w0 + per);
+  // 1. per-warp counts over this warp's contiguous slice
+  for (int r = w0; r < w1; r += 32) {
+    const int f = r + lane;
+    int e = -1;
+    if (f < w1) {
+      e = ids[f];
+      if (e < 0 || e >= E) {
+        moe::report(status, MOE_ERR_BAD_INDEX);
+        inv_perm[f] = -1;
+        e = -1;
+      }
+    }
+    const int key = e >= 0 ? e : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
+  }
+  __syncthreads();
+  // 2. counts, exclusive scan over experts, per-warp bases
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int ww = 0; ww < SMALL_WARPS; ++ww) total += wc[ww * E + e];
+  if (e < moe::kMaxExperts) s_scan[e] = total;
+  __syncthreads();
+  for (int o = 1; o < moe::kMaxExperts; o <<= 1) {
+    const int v = (e < moe::kMaxExperts && e >= o) ? s_scan[e - o] : 0;
+    __syncthreads();
+    if (e < moe::kMaxExperts) s_scan[e] += v;
+    __syncthreads();
+  }
+  if (e < E) {
+    const int excl = s_scan[e] - total;
+    counts[e] = total;
+    offsets[e] = excl;
+    int run = excl;
+    for (int ww = 0; ww < SMALL_WARPS; ++ww) {
+      const int c = wc[ww * E + e];
+      wc[ww * E + e] = run;
+      run += c;
+    }
+  }
+  if (e == 0) offsets[E] = s_scan[moe::kMaxExperts - 1];
+  __syncthreads();
+  // 3. stable scatter: slices in warp order, rounds in order, lanes in order
+  for (int r = w0; r < w1; r += 32) {
+    const int f = r + lane;
+    int ex = -1;
+    if (f < w1) {
+      ex = ids[f];
+      if (ex < 0 || ex >= E) ex = -1;
+    }
+    const int key = ex >= 0 ? ex : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (ex >= 0) {
+      const int p = wc[warp * E + ex] + __popc(peers & lt);
+      perm[p] = f;
+      inv_perm[f] = p;
+      packed_tok[p] = f / k;
+      if (packed_w) packed_w[p] = w[f];
+    }
+    __syncwarp();
+    if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
+    __syncwarp();
+  }
+  if (x == nullptr) return;
+  __syncthreads();
+  // 4. gather (small total): one warp per row, 16-byte vectors
+  const int nrows = s_scan[moe::kMaxExperts - 1];
+  for (int p = warp; p < nrows; p += SMALL_WARPS) {
+    const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
+    uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
+    for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+  }
+}
+
 // ------------------------------------------------------------- gather ---
 
 constexpr int GW = 4;      // warps per CTA, each an independent copy engine client
@@ -249,17 +347,29 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
                             float* packed_w, void* x_packed, void* ws, int32_t* status,
                             cudaStream_t s) {
   const int N = T * k;
-  const int B = (N + CHUNK - 1) / CHUNK;
-  int32_t* bc = static_cast<int32_t*>(ws);
-  const size_t wsm = sizeof(int) * DWARPS * E;
-  dispatch_count_kernel<<<B, DNT, wsm, s>>>(ids, N, E, bc, status);
-  dispatch_scan_kernel<<<1, 256, 0, s>>>(bc, B, E, counts, offsets);
-  dispatch_scatter_kernel<<<B, DNT, wsm, s>>>(ids, w, N, E, k, bc, perm, inv_perm, packed_tok,
-                                              w ? packed_w : nullptr, status);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess || x == nullptr) return err;
   const int es = dtype == MOE_BF16 ? 2 : 4;
   const int row_bytes = H * es;
+  if (N <= SMALL_N) {
+    const bool fuse_gather =
+        x != nullptr && static_cast<size_t>(N) * row_bytes <= (static_cast<size_t>(1) << 20);
+    dispatch_small_kernel<<<1, SMALL_WARPS * 32, sizeof(int) * SMALL_WARPS * E, s>>>(
+        ids, w, N, E, k, counts, offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,
+        fuse_gather ? static_cast<const uint4*>(x) : nullptr, row_bytes / 16,
+        static_cast<uint4*>(x_packed), status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || x == nullptr || fuse_gather) return err;
+  } else {
+    const int B = (N + CHUNK - 1) / CHUNK;
+    int32_t* bc = static_cast<int32_t*>(ws);
+    const size_t wsm = sizeof(int) * DWARPS * E;
+    dispatch_count_kernel<<<B, DNT, wsm, s>>>(ids, N, E, bc, status);
+    dispatch_scan_kernel<<<1, 256, 0, s>>>(bc, B, E, counts, offsets);
+    dispatch_scatter_kernel<<<B, DNT, wsm, s>>>(ids, w, N, E, k, bc, perm, inv_perm, packed_tok,
+                                                w ? packed_w : nullptr, status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess || x == nullptr) return err;
+  }
+  cudaError_t err;
   const size_t gsm = static_cast<size_t>(GW) * GSLOTS * row_bytes;
   if (gsm > 200 * 1024) {
     const int grid = std::max(1, std::min((N + 7) / 8, num_sms() * 8));
@@ -268,8 +378,7 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
                                                      static_cast<uint4*>(x_packed));
     return cudaGetLastError();
   }
-  err = cudaFuncSetAttribute(dispatch_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gsm));
+  err = ensure_smem(reinterpret_cast<const void*>(dispatch_gather_kernel), static_cast<int>(gsm));
   if (err != cudaSuccess) return err;
   const int ctas_per_sm = std::max(1, static_cast<int>((200 * 1024) / gsm));
   const int grid = std::max(1, std::min((N + GW - 1) / GW, num_sms() * ctas_per_sm));

@@ -15,27 +15,36 @@
 //                        merger adds the k terms before the one bf16 rounding)
 //
 // Tile = 128 packed rows (tokens of one expert; MMA M) x 256 weight rows
-// (MMA N) x the whole K.  In pass 1 the 256 weight rows are 128 gate rows and
-// the 128 matching up rows (one 3-D TMA box over [2E, I, H]), so column c and
-// column 128 + c of the accumulator are the gate and up value of the same
-// feature and the SwiGLU is thread-local.  The tile list is derived on the
-// device from `offsets` (the scheduler of the README's "Scheduler Module",
-// folded into the kernel): expert e owns ceil(count_e / 128) token tiles x
-// (rows / 256) weight tiles, token tiles fastest, so CTAs running at the same
-// time share a weight tile through L2.  Experts with no rows own no tiles.
+// (MMA N) x K.  In pass 1 the 256 weight rows are 128 gate rows and the 128
+// matching up rows (one 3-D TMA box over [2E, I, H]), so column c and column
+// 128 + c of the accumulator are the gate and up value of the same feature
+// and the SwiGLU is thread-local.  The tile list is derived on the device from
+// `offsets` (the scheduler of the README's "Scheduler Module", folded into
+// the kernel): expert e owns ceil(count_e / 128) token tiles x (rows / 256)
+// weight tiles, token tiles fastest, so CTAs running at the same time share a
+// weight tile through L2.  Experts with no rows own no tiles.
 //
-// CTA = 6 warps, one CTA per SM, persistent over tiles:
-//   warp 0   TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
-//   warp 1   MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
-//   warps 2-5 epilogue      (tcgen05.ld from the TMEM accumulator, math, store)
+// Split-K.  When a pass has fewer tiles than two per CTA (decode batches, a
+// shared expert, a long K), every CTA derives the same split count S from the
+// tile count, the grid and K, and the work unit becomes (tile, K-slice).  A
+// unit stores the valid rows of its fp32 partial in the workspace; the last
+// unit of a tile to finish (a per-tile arrival counter) adds the S partials in
+// slice order (deterministic) and applies the epilogue.  The counter returns
+// to zero for the next call.
+//
+// CTA = 6 warps, one CTA per SM, persistent over units:
+//   warp 0    TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
+//   warp 1    MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
+//   warps 2-5 epilogue       (tcgen05.ld from the TMEM accumulator, math, store)
 // The two 256-column fp32 accumulators are double-buffered in TMEM, so the
-// epilogue of one tile overlaps the MMAs of the next.  Every wait is bounded;
+// epilogue of one unit overlaps the MMAs of the next.  Every wait is bounded;
 // a wait that runs out reports MOE_ERR_TIMEOUT, the CTA drains what it issued
 // and frees its TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -53,6 +62,9 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NTHREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
+constexpr int MAX_SPLITS = 16;
+constexpr int COUNTER_INTS = 4096;                        // per-tile arrival counters
+constexpr size_t PARTIAL_BYTES = sizeof(float) * BM * BN;  // one unit's partial slot
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
 
@@ -64,32 +76,60 @@ struct Ctl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int splits;          // S: K-slices per tile (1 = no split)
+  int last_flag;       // epilogue: this unit is the last of its tile
   int offs[moe::kMaxExperts + 1];
   int tstart[moe::kMaxExperts + 1];   // first tile of expert e (tiles = token tiles x NTW)
 };
 
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
 
-struct TileCoord {
-  int e, nt, mt;
+struct Unit {
+  int tile, e, nt, mt, ks, kb0, kb1;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const Ctl& c, int E, int ntw, int t) {
-  // largest e with tstart[e] <= t (experts without tiles share their successor's start)
+__device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, int u) {
+  Unit r;
+  const int S = c.splits;
+  r.tile = u / S;
+  r.ks = u - r.tile * S;
+  r.kb0 = (r.ks * kblocks) / S;
+  r.kb1 = ((r.ks + 1) * kblocks) / S;
+  // largest e with tstart[e] <= tile (experts without tiles share their successor's start)
   int lo = 0, hi = E - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (c.tstart[mid] <= t) lo = mid; else hi = mid - 1;
+    if (c.tstart[mid] <= r.tile) lo = mid; else hi = mid - 1;
   }
-  const int e = lo;
-  const int mte = (c.offs[e + 1] - c.offs[e] + BM - 1) / BM;
-  const int local = t - c.tstart[e];
-  TileCoord r;
-  r.e = e;
+  r.e = lo;
+  const int mte = (c.offs[r.e + 1] - c.offs[r.e] + BM - 1) / BM;
+  const int local = r.tile - c.tstart[r.e];
   r.nt = local / mte;
   r.mt = local - r.nt * mte;
-  (void)ntw;
   return r;
+}
+
+// Split count: 1 when there are at least two tiles per CTA; otherwise the
+// smallest S whose units fill the grid's waves to >= 90% (else the best one),
+// with >= 4 K-blocks per unit and the units within the workspace.
+__device__ int choose_splits(int tiles, int grid, int kblocks, int max_units) {
+  if (tiles <= 0 || tiles >= 2 * grid) return 1;
+  int smax = min(MAX_SPLITS, kblocks / 4);
+  smax = min(smax, max_units / tiles);
+  if (smax <= 1) return 1;
+  int best = 1;
+  float best_eff = 0.f;
+  for (int s = 1; s <= smax; ++s) {
+    const int units = tiles * s;
+    const int waves = (units + grid - 1) / grid;
+    const float eff = static_cast<float>(units) / static_cast<float>(waves * grid);
+    if (eff >= 0.9f) return s;
+    if (eff > best_eff + 1e-6f) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
 }
 
 __device__ __forceinline__ void set_abort(Ctl& c, int32_t* status) {
@@ -101,19 +141,46 @@ __device__ __forceinline__ bool aborted(const Ctl& c) {
   return *reinterpret_cast<const volatile int*>(&c.abort) != 0;
 }
 
+__device__ __forceinline__ void epi_bar() {   // the 4 epilogue warps only
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
+
+// 16 h values (16 gate and 16 up accumulator columns) -> 16 bf16.
+__device__ __forceinline__ void store_h16(__nv_bfloat16* dst, const float* g, const float* u) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    pk[j] = moe::pack_bf16x2(silu_mul(g[2 * j], u[2 * j]), silu_mul(g[2 * j + 1], u[2 * j + 1]));
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+// 16 accumulator columns scaled by sc -> 16 fp32.
+__device__ __forceinline__ void store_y16(float* dst, const float* v, float sc) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    d4[j] = make_float4(v[4 * j] * sc, v[4 * j + 1] * sc, v[4 * j + 2] * sc, v[4 * j + 3] * sc);
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const int32_t* __restrict__ offsets, int E, int K, int ntw,
                         int rows_per_expert, const float* __restrict__ packed_w,
-                        void* __restrict__ out, int ldo, int32_t* status) {
+                        void* __restrict__ out, int ldo, int* __restrict__ counters,
+                        float* __restrict__ partials, int max_units, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Ctl& c = *reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int kblocks = K / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -166,14 +233,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 31) {
       c.offs[E] = offsets[E];
       c.tstart[E] = incl * ntw;
+      c.splits = (counters != nullptr && partials != nullptr && incl * ntw <= COUNTER_INTS)
+                     ? choose_splits(incl * ntw, gridDim.x, kblocks, max_units)
+                     : 1;
     }
   }
   moe::tc_fence_before();
   __syncthreads();
   moe::tc_fence_after();
 
-  const int total = c.tstart[E];
-  const int kblocks = K / BK;
+  const int S = c.splits;
+  const int total = c.tstart[E] * S;        // units
   const uint32_t tmem = c.tmem_base;
 
   if (warp == 0) {
@@ -182,11 +252,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued[STAGES] = {0, 0, 0, 0};
-      for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x) {
-        const TileCoord tc = decode_tile(c, E, ntw, t);
-        const int arow = c.offs[tc.e] + tc.mt * BM;
+      for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x) {
+        const Unit un = decode_unit(c, E, kblocks, u);
+        const int arow = c.offs[un.e] + un.mt * BM;
         bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
             set_abort(c, status);
             ok = false;
@@ -197,9 +267,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
           moe::tma_load_2d(sa, &tmA, fb, kb * BK, arow);
           if (EPI == EPI_SWIGLU)
-            moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, tc.nt * (BN / 2), 2 * tc.e);
+            moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, un.nt * (BN / 2), 2 * un.e);
           else
-            moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, tc.e * rows_per_expert + tc.nt * BN);
+            moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, un.e * rows_per_expert + un.nt * BN);
           ++issued[stage];
           if (++stage == STAGES) {
             stage = 0;
@@ -218,7 +288,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x, ++i) {
+      for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x, ++i) {
+        const Unit un = decode_unit(c, E, kblocks, u);
         const int buf = i & 1;
         if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
           set_abort(c, status);
@@ -227,7 +298,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         moe::tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
         bool ok = true;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase)) {
             set_abort(c, status);
             ok = false;
@@ -239,7 +310,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = moe::sw128_kmajor_desc(sa + kk * 32);
             const uint64_t bd = moe::sw128_kmajor_desc(sa + A_BYTES + kk * 32);
-            moe::tc_mma_f16(d, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            moe::tc_mma_f16(d, ad, bd, IDESC, (kb > un.kb0 || kk > 0) ? 1u : 0u);
           }
           moe::tc_commit(moe::smem_addr(&c.empty[stage]));
           if (++stage == STAGES) {
@@ -259,45 +330,54 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;          // row of the tile owned by this thread
     int i = 0;
-    for (int t = blockIdx.x; t < total && !aborted(c); t += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x, ++i) {
       const int buf = i & 1;
       if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1)) {
         set_abort(c, status);
         break;
       }
       moe::tc_fence_after();
-      const TileCoord tc = decode_tile(c, E, ntw, t);
-      const int rows_valid = c.offs[tc.e + 1] - c.offs[tc.e] - tc.mt * BM;
+      const Unit un = decode_unit(c, E, kblocks, u);
+      const int rows_valid = c.offs[un.e + 1] - c.offs[un.e] - un.mt * BM;
       const bool live = row < rows_valid;
-      const size_t grow = static_cast<size_t>(c.offs[tc.e] + tc.mt * BM + row);
+      const size_t grow = static_cast<size_t>(c.offs[un.e] + un.mt * BM + row);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN);
-      if (EPI == EPI_SWIGLU) {
-        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + grow * ldo + tc.nt * (BN / 2);
+      if (S == 1) {
+        if (EPI == EPI_SWIGLU) {
+          __nv_bfloat16* dst =
+              static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 2; cc += 16) {
-          uint32_t g[16], u[16];
-          moe::tmem_ld16(taddr + cc, g);
-          moe::tmem_ld16(taddr + BN / 2 + cc, u);
-          moe::tmem_ld_wait();
-          uint32_t pk[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float g0 = __uint_as_float(g[2 * j]), g1 = __uint_as_float(g[2 * j + 1]);
-            const float u0 = __uint_as_float(u[2 * j]), u1 = __uint_as_float(u[2 * j + 1]);
-            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
-            pk[j] = moe::pack_bf16x2(h0, h1);
+          for (int cc = 0; cc < BN / 2; cc += 16) {
+            uint32_t g[16], v[16];
+            moe::tmem_ld16(taddr + cc, g);
+            moe::tmem_ld16(taddr + BN / 2 + cc, v);
+            moe::tmem_ld_wait();
+            if (live)
+              store_h16(dst + cc, reinterpret_cast<const float*>(g),
+                        reinterpret_cast<const float*>(v));
           }
-          if (live) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
-            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          const float sc = live ? (packed_w ? packed_w[grow] : 1.f) : 0.f;
+          float* dst = static_cast<float*>(out) + grow * ldo + un.nt * BN;
+#pragma unroll 1
+          for (int cc = 0; cc < BN; cc += 32) {
+            uint32_t a[16], b[16];
+            moe::tmem_ld16(taddr + cc, a);
+            moe::tmem_ld16(taddr + cc + 16, b);
+            moe::tmem_ld_wait();
+            if (live) {
+              store_y16(dst + cc, reinterpret_cast<const float*>(a), sc);
+              store_y16(dst + cc + 16, reinterpret_cast<const float*>(b), sc);
+            }
           }
         }
+        moe::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
       } else {
-        const float sc = live ? (packed_w ? packed_w[grow] : 1.f) : 0.f;
-        float* dst = static_cast<float*>(out) + grow * ldo + tc.nt * BN;
+        // Partial of one K-slice: valid rows to this unit's workspace slot.
+        float* slot = partials + static_cast<size_t>(u) * (BM * BN) + static_cast<size_t>(row) * BN;
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 32) {
           uint32_t a[16], b[16];
@@ -305,21 +385,72 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           moe::tmem_ld16(taddr + cc + 16, b);
           moe::tmem_ld_wait();
           if (live) {
-            float4* d4 = reinterpret_cast<float4*>(dst + cc);
+            store_y16(slot + cc, reinterpret_cast<const float*>(a), 1.f);
+            store_y16(slot + cc + 16, reinterpret_cast<const float*>(b), 1.f);
+          }
+        }
+        moe::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));   // TMEM free
+        __threadfence();
+        epi_bar();
+        if (warp == 2 && lane == 0) {
+          const int old = atomicAdd(&counters[un.tile], 1);
+          const int last = old == S - 1;
+          if (last) counters[un.tile] = 0;       // ready for the next call
+          c.last_flag = last;
+        }
+        epi_bar();
+        const bool last = c.last_flag != 0;
+        epi_bar();                               // everyone read the flag before it changes
+        if (last) {
+          __threadfence();
+          if (live) {
+            const float* base = partials + static_cast<size_t>(un.tile) * S * (BM * BN) +
+                                static_cast<size_t>(row) * BN;
+            if (EPI == EPI_SWIGLU) {
+              __nv_bfloat16* dst =
+                  static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
+#pragma unroll 1
+              for (int cc = 0; cc < BN / 2; cc += 16) {
+                float g[16], v[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              d4[j] = make_float4(__uint_as_float(a[4 * j]) * sc, __uint_as_float(a[4 * j + 1]) * sc,
-                                  __uint_as_float(a[4 * j + 2]) * sc, __uint_as_float(a[4 * j + 3]) * sc);
+                for (int j = 0; j < 16; ++j) g[j] = v[j] = 0.f;
+                for (int s = 0; s < S; ++s) {           // slice order: deterministic
+                  const float4* pg = reinterpret_cast<const float4*>(base + s * (BM * BN) + cc);
+                  const float4* pu =
+                      reinterpret_cast<const float4*>(base + s * (BM * BN) + BN / 2 + cc);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              d4[4 + j] = make_float4(__uint_as_float(b[4 * j]) * sc, __uint_as_float(b[4 * j + 1]) * sc,
-                                      __uint_as_float(b[4 * j + 2]) * sc, __uint_as_float(b[4 * j + 3]) * sc);
+                  for (int j = 0; j < 4; ++j) {
+                    const float4 x = __ldcg(pg + j), y = __ldcg(pu + j);
+                    g[4 * j] += x.x; g[4 * j + 1] += x.y; g[4 * j + 2] += x.z; g[4 * j + 3] += x.w;
+                    v[4 * j] += y.x; v[4 * j + 1] += y.y; v[4 * j + 2] += y.z; v[4 * j + 3] += y.w;
+                  }
+                }
+                store_h16(dst + cc, g, v);
+              }
+            } else {
+              const float sc = packed_w ? packed_w[grow] : 1.f;
+              float* dst = static_cast<float*>(out) + grow * ldo + un.nt * BN;
+#pragma unroll 1
+              for (int cc = 0; cc < BN; cc += 16) {
+                float v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                for (int s = 0; s < S; ++s) {
+                  const float4* p = reinterpret_cast<const float4*>(base + s * (BM * BN) + cc);
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const float4 x = __ldcg(p + j);
+                    v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
+                  }
+                }
+                store_y16(dst + cc, v, sc);
+              }
+            }
           }
         }
       }
-      moe::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
     }
   }
 
@@ -345,8 +476,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+bool encode_uncached(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                     const cuuint64_t* strides_bytes, const cuuint32_t* box) {
   auto fn = get_encode();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
@@ -355,6 +486,46 @@ bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Small cache of encoded tensor maps: a layer called again on the same
+// buffers reuses its descriptors instead of encoding four per call.  The map
+// depends only on the key (device, base, rank, dims, strides, box).
+struct MapKey {
+  int dev, rank;
+  const void* base;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+};
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  constexpr int kSlots = 64;
+  static std::mutex mu;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static int used = 0, next = 0;
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));
+  cudaGetDevice(&k.dev);
+  k.rank = rank;
+  k.base = base;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+    if (i + 1 < rank) k.strides[i] = strides_bytes[i];
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (std::memcmp(&keys[i], &k, sizeof(k)) == 0) {
+      *m = maps[i];
+      return true;
+    }
+  if (!encode_uncached(m, base, rank, dims, strides_bytes, box)) return false;
+  const int slot = used < kSlots ? used++ : (next++ % kSlots);
+  keys[slot] = k;
+  maps[slot] = *m;
+  return true;
 }
 
 // Activations [rows, K] bf16, box 64 x 128.
@@ -369,17 +540,19 @@ bool map_rows(CUtensorMap* m, const void* p, int rows, int K) {
 
 namespace moe_host {
 
+size_t experts_ws_bytes() {
+  return sizeof(int) * COUNTER_INTS + PARTIAL_BYTES * 4 * static_cast<size_t>(num_sms());
+}
+
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, int32_t* status,
-                              cudaStream_t s, const char** why) {
-  cudaError_t e1 = cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SWIGLU>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(SMEM_BYTES));
+                              int H, int I, int E, void* h, void* y, void* ws, size_t ws_bytes,
+                              int32_t* status, cudaStream_t s, const char** why) {
+  cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU>),
+                                static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
-  e1 = cudaFuncSetAttribute(grouped_gemm_kernel<EPI_SCALE>,
-                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                            static_cast<int>(SMEM_BYTES));
+  e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SCALE>),
+                   static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
   CUtensorMap mA1, mB1, mA2, mB2;
   bool ok = map_rows(&mA1, x_packed, N, H) && map_rows(&mA2, h, N, I);
@@ -403,16 +576,29 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
     return cudaErrorInvalidValue;
   }
-  const int mt_bound = (N + BM - 1) / BM + E;
-  const int ntw1 = I / (BN / 2);
-  const int ntw2 = H / BN;
+  // Split-K needs the workspace: counters, then 128 KiB partial slots.
+  int* counters = nullptr;
+  float* partials = nullptr;
+  int max_units = 0;
+  const size_t cbytes = sizeof(int) * COUNTER_INTS;
+  if (ws != nullptr && ws_bytes >= cbytes + PARTIAL_BYTES) {
+    counters = static_cast<int*>(ws);
+    partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + cbytes);
+    max_units = static_cast<int>(std::min<size_t>((ws_bytes - cbytes) / PARTIAL_BYTES, 1 << 20));
+  }
   const int sms = num_sms();
-  const int g1 = std::max(1, std::min(sms, mt_bound * ntw1));
-  const int g2 = std::max(1, std::min(sms, mt_bound * ntw2));
+  int g1 = sms, g2 = sms;
+  if (counters == nullptr) {   // no split possible: never more CTAs than tiles
+    const int mt_bound = (N + BM - 1) / BM + E;
+    g1 = std::max(1, std::min(sms, mt_bound * (I / (BN / 2))));
+    g2 = std::max(1, std::min(sms, mt_bound * (H / BN)));
+  }
   grouped_gemm_kernel<EPI_SWIGLU><<<g1, NTHREADS, SMEM_BYTES, s>>>(
-      mA1, mB1, offsets, E, H, ntw1, 2 * I, nullptr, h, I, status);
+      mA1, mB1, offsets, E, H, I / (BN / 2), 2 * I, nullptr, h, I, counters, partials,
+      max_units, status);
   grouped_gemm_kernel<EPI_SCALE><<<g2, NTHREADS, SMEM_BYTES, s>>>(
-      mA2, mB2, offsets, E, I, ntw2, H, packed_w, y, H, status);
+      mA2, mB2, offsets, E, I, H / BN, H, packed_w, y, H, counters, partials, max_units,
+      status);
   return cudaGetLastError();
 }
 

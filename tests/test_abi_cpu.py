@@ -56,7 +56,8 @@ def test_abi_version_and_workspace_queries(lib):
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
     assert M.moe_dispatch_workspace_bytes(0, 2, 8) == 0
-    assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_BF16) == 0
+    assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_BF16) >= 4096 * 4 + 128 * 1024
+    assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_F32) == 0
 
 
 NULL = None

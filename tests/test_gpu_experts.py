@@ -29,21 +29,33 @@ def _make(counts, H, I, dtype, seed=0, N=None, with_w=True):
     return x, torch.tensor(offs), pw, w13, w2
 
 
-def _run(x, offs, pw, w13, w2, canary=True):
+def _ws(x, w13):
+    N, H = x.shape
+    I = w13.shape[1] // 2
+    code = M.MOE_BF16 if x.dtype == torch.bfloat16 else M.MOE_F32
+    return torch.zeros(max(16, M.moe_experts_workspace_bytes(N, H, I, w13.shape[0], code)),
+                       dtype=torch.uint8, device=DEV)
+
+
+def _run(x, offs, pw, w13, w2, canary=True, ws="zeros"):
     N, H = x.shape
     I = w13.shape[1] // 2
     fill = 1536.0 if canary else 0.0
     h = torch.full((N, I), fill, dtype=x.dtype, device=DEV)
     y = torch.full((N, H), fill, dtype=torch.float32, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    M.moe_experts(dev(x), dev(offs), dev(pw), dev(w13), dev(w2), h, y, status=status)
+    if isinstance(ws, str):
+        ws = _ws(x, w13)
+    M.moe_experts(dev(x), dev(offs), dev(pw), dev(w13), dev(w2), h, y, ws=ws, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
+    if ws is not None:       # the split-K arrival counters are back at zero
+        assert int(ws[:4096 * 4].view(torch.int32).abs().sum().item()) == 0
     return h.cpu(), y.cpu()
 
 
-def _check(x, offs, pw, w13, w2, tol):
-    h, y = _run(x, offs, pw, w13, w2)
+def _check(x, offs, pw, w13, w2, tol, ws="zeros"):
+    h, y = _run(x, offs, pw, w13, w2, ws=ws)
     hn = int(offs[-1])
     ho, yo = O.experts(x[:hn], offs.numpy(), None if pw is None else pw[:hn], w13, w2)
     eh = err_bf16_out(h[:hn], ho) if h.dtype == torch.bfloat16 else rel(h[:hn], ho)
@@ -102,3 +114,31 @@ def test_experts_deterministic():
     h2, y2 = _run(*args)
     assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
     assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+
+
+# Few tiles: the kernels split K across CTAs and reduce the partials in order.
+@pytest.mark.parametrize("counts,H,I", [
+    ([1, 0, 0, 0, 0, 1, 0, 0], 512, 1024),      # decode: one row for each of two experts
+    ([0, 3, 9, 2], 1024, 512),                  # a few rows, long K for w13
+    ([32], 512, 2048),                          # a shared expert at a decode batch: K = 2048 for w2
+    ([300, 5, 0, 1], 1024, 256),                # full + ragged token tiles under a split
+])
+def test_experts_bf16_split_k(counts, H, I):
+    _check(*_make(counts, H, I, torch.bfloat16, seed=11 + sum(counts)), tol=TOL["bf16"])
+
+
+def test_experts_bf16_split_k_matches_unsplit_and_is_deterministic():
+    args = _make([2, 0, 7, 1], 1024, 512, torch.bfloat16, seed=12)
+    h1, y1 = _run(*args)
+    h2, y2 = _run(*args)
+    assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+    h0, y0 = _run(*args, ws=None)            # no workspace: one unit per tile
+    hn = int(args[1][-1])
+    # different fp32 summation order: h may round to a neighbouring bf16 value
+    assert rel(y1[:hn], y0[:hn]) <= 1e-3
+    assert err_bf16_out(h1[:hn], O.to_f64(h0[:hn])) <= 1e-2
+
+
+def test_experts_bf16_without_workspace():
+    _check(*_make([1, 0, 3], 512, 512, torch.bfloat16, seed=13), tol=TOL["bf16"], ws=None)

@@ -53,8 +53,9 @@ def test_route_configs(name):
                                  (200, 5), (256, 8)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("H", [72, 96])
-def test_route_shapes(E, k, dtype, H):
-    cfg = LayerConfig("r", T=131, H=H, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 2 == 0))
+@pytest.mark.parametrize("T", [7, 131])       # one-CTA-per-token path / cluster path
+def test_route_shapes(E, k, dtype, H, T):
+    cfg = LayerConfig("r", T=T, H=H, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 2 == 0))
     p = make_layer(cfg, seed=E + k)
     _check(p["x"], p["W_gate"], None, k, cfg.renormalize)
 
