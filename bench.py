@@ -318,6 +318,15 @@ def run_gpu(args, cfg):
         raise SystemExit(f"device status {int(buf.status.item())} after warm-up")
     counts = buf.counts.cpu().tolist()
 
+    # Timed region: K steps, each bracketed by two events only.  Steps are
+    # enqueued in groups behind a short GPU spin (outside every bracket), so
+    # the GPU runs each group back to back and no bracket contains time spent
+    # waiting for the host.  A second pass of K steps with an event between
+    # stages gives the per-stage split (events between small kernels cost a
+    # few microseconds each, so the step time comes from the first pass).
+    GROUP = 8
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if dist:
@@ -325,22 +334,25 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.3)
-    # Steps are enqueued in groups behind a short GPU spin (outside every timed
-    # bracket), so the GPU runs each group back to back and no stage bracket
-    # contains time spent waiting for the host to issue the next launch.
-    GROUP = 8
     for g0 in range(0, args.steps, GROUP):
         torch.cuda._sleep(int(20e6))            # ~10 ms of GPU spin while the host enqueues
         for i in range(g0, min(args.steps, g0 + GROUP)):
             flush_l2()
-            step(evs[i])
+            step_ev[i][0].record(stream)
+            step()
+            step_ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
     if dist:
         dist.barrier()
+    ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
+    for g0 in range(0, args.steps, GROUP):
+        torch.cuda._sleep(int(20e6))
+        for i in range(g0, min(args.steps, g0 + GROUP)):
+            flush_l2()
+            step(evs[i])
+    torch.cuda.synchronize(dev)
     stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
-    step_ms = [sum(s) for s in stage_ms]
-    ms = sum(step_ms) / args.steps
     per_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(4)]
     ms_max = max_over_ranks(ms, dev)
 

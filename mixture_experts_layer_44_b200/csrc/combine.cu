@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
   const int nvec = H / 8;                               // 8 outputs per thread step
   __shared__ int rows[moe::kMaxTopK];
   __shared__ float gate;
+  moe::grid_dep_wait();
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < k) {
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
       }
     }
   }
+  moe::grid_dep_launch();
 }
 
 }  // namespace
@@ -89,12 +91,10 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
   const int grid = std::max(1, std::min(T, num_sms() * 8));
   const int N = T * k;
   if (dtype == MOE_BF16)
-    combine_kernel<true><<<grid, CNT, 0, s>>>(y, inv_perm, T, H, k, N, shared, shared_gate, out,
-                                              status);
-  else
-    combine_kernel<false><<<grid, CNT, 0, s>>>(y, inv_perm, T, H, k, N, shared, shared_gate, out,
-                                               status);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(CNT), 0, s, 0, y, inv_perm, T, H, k,
+                      N, shared, shared_gate, out, status);
+  return launch_pdl(combine_kernel<false>, dim3(grid), dim3(CNT), 0, s, 0, y, inv_perm, T, H, k,
+                    N, shared, shared_gate, out, status);
 }
 
 }  // namespace moe_host

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "../../include/moe_b200.h"
 
@@ -33,6 +34,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 __device__ __forceinline__ float bf16_to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Programmatic dependent launch.  Every kernel here is launched so that it may
+// start while the previous kernel on the stream finishes; it does its
+// independent set-up, then grid_dep_wait() before the first read of anything
+// the previous kernel wrote (the wait returns once that kernel has completed
+// and its writes are visible).  grid_dep_launch() lets the next kernel begin
+// launching once every CTA of this one has called it (or exited).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Unpack 8 bf16 (one 16-byte vector) into floats.
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
@@ -80,4 +94,32 @@ int num_sms();
 void set_last_error(const std::string& msg);   // the message moe_last_error() returns
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel, size).
 cudaError_t ensure_smem(const void* kernel, int bytes);
+
+// Launch with programmatic stream serialization (and a cluster of cluster_x
+// CTAs along x when cluster_x > 0).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 }  // namespace moe_host

@@ -45,6 +45,7 @@ __device__ __forceinline__ void warp_counts(const int32_t* __restrict__ ids, int
                                             int base, int* wc, int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < DWARPS * E; i += DNT) wc[i] = 0;
+  moe::grid_dep_wait();
   __syncthreads();
   const int w0 = base + warp * PER_WARP;
   for (int r = 0; r < PER_WARP; r += 32) {
@@ -78,6 +79,7 @@ __global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* __re
     for (int w = 0; w < DWARPS; ++w) s += wc[w * E + e];
     bc[static_cast<size_t>(blockIdx.x) * E + e] = s;
   }
+  moe::grid_dep_launch();
 }
 
 // One CTA of 256 threads (E <= 256).
@@ -86,6 +88,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
                                                             int32_t* __restrict__ offsets) {
   __shared__ int s_scan[256];
   const int e = threadIdx.x;
+  moe::grid_dep_wait();
   int total = 0;
   if (e < E)
     for (int b = 0; b < B; ++b) total += bc[static_cast<size_t>(b) * E + e];
@@ -111,6 +114,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
     }
   }
   if (e == 255) offsets[E] = s_scan[255];
+  moe::grid_dep_launch();
 }
 
 __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
@@ -156,6 +160,7 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
     __syncwarp();
   }
+  moe::grid_dep_launch();
 }
 
 // ------------------------------------------------- single-CTA variant ---
@@ -175,6 +180,7 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   for (int i = threadIdx.x; i < SMALL_WARPS * E; i += blockDim.x) wc[i] = 0;
+  moe::grid_dep_wait();
   __syncthreads();
   const int per = (N + SMALL_WARPS - 1) / SMALL_WARPS;
   const int w0 = warp * per, w1 = min(N, w0 + per);
@@ -242,6 +248,7 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
     if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
     __syncwarp();
   }
+  moe::grid_dep_launch();
   if (x == nullptr) return;
   __syncthreads();
   // 4. gather (small total): one warp per row, 16-byte vectors
@@ -269,6 +276,7 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
   uint8_t* ring = gsm + static_cast<size_t>(warp) * GSLOTS * row_bytes;
   for (int s = 0; s < GSLOTS; ++s) moe::mbar_init(moe::smem_addr(&bars[warp][s]), 1);
   moe::fence_barrier_init();
+  moe::grid_dep_wait();
 
   const int nrows = offsets[E];            // valid rows (assignments with a valid id)
   const int stride = gridDim.x * GW;
@@ -304,12 +312,14 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
     }
   }
   moe::bulk_wait_all();
+  moe::grid_dep_launch();
 }
 
 // Rows too large for the shared-memory ring: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ packed_tok,
     const int32_t* __restrict__ offsets, int E, int row_vecs, uint4* __restrict__ xp) {
+  moe::grid_dep_wait();
   const int nrows = offsets[E];
   const int lane = threadIdx.x & 31;
   for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < nrows;
@@ -318,6 +328,7 @@ __global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
     for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
   }
+  moe::grid_dep_launch();
 }
 
 }  // namespace
@@ -352,40 +363,44 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
   if (N <= SMALL_N) {
     const bool fuse_gather =
         x != nullptr && static_cast<size_t>(N) * row_bytes <= (static_cast<size_t>(1) << 20);
-    dispatch_small_kernel<<<1, SMALL_WARPS * 32, sizeof(int) * SMALL_WARPS * E, s>>>(
-        ids, w, N, E, k, counts, offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,
+    cudaError_t err = launch_pdl(
+        dispatch_small_kernel, dim3(1), dim3(SMALL_WARPS * 32), sizeof(int) * SMALL_WARPS * E, s,
+        0, ids, w, N, E, k, counts, offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,
         fuse_gather ? static_cast<const uint4*>(x) : nullptr, row_bytes / 16,
         static_cast<uint4*>(x_packed), status);
-    cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess || x == nullptr || fuse_gather) return err;
   } else {
     const int B = (N + CHUNK - 1) / CHUNK;
     int32_t* bc = static_cast<int32_t*>(ws);
     const size_t wsm = sizeof(int) * DWARPS * E;
-    dispatch_count_kernel<<<B, DNT, wsm, s>>>(ids, N, E, bc, status);
-    dispatch_scan_kernel<<<1, 256, 0, s>>>(bc, B, E, counts, offsets);
-    dispatch_scatter_kernel<<<B, DNT, wsm, s>>>(ids, w, N, E, k, bc, perm, inv_perm, packed_tok,
-                                                w ? packed_w : nullptr, status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err =
+        launch_pdl(dispatch_count_kernel, dim3(B), dim3(DNT), wsm, s, 0, ids, N, E, bc, status);
+    if (err == cudaSuccess)
+      err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(256), 0, s, 0, bc, B, E, counts,
+                       offsets);
+    if (err == cudaSuccess)
+      err = launch_pdl(dispatch_scatter_kernel, dim3(B), dim3(DNT), wsm, s, 0, ids, w, N, E, k,
+                       static_cast<const int32_t*>(bc), perm, inv_perm, packed_tok,
+                       w ? packed_w : nullptr, status);
     if (err != cudaSuccess || x == nullptr) return err;
   }
   cudaError_t err;
   const size_t gsm = static_cast<size_t>(GW) * GSLOTS * row_bytes;
   if (gsm > 200 * 1024) {
     const int grid = std::max(1, std::min((N + 7) / 8, num_sms() * 8));
-    dispatch_gather_vec_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), packed_tok,
-                                                     offsets, E, row_bytes / 16,
-                                                     static_cast<uint4*>(x_packed));
-    return cudaGetLastError();
+    return launch_pdl(dispatch_gather_vec_kernel, dim3(grid), dim3(256), 0, s, 0,
+                      static_cast<const uint4*>(x), static_cast<const int32_t*>(packed_tok),
+                      static_cast<const int32_t*>(offsets), E, row_bytes / 16,
+                      static_cast<uint4*>(x_packed));
   }
   err = ensure_smem(reinterpret_cast<const void*>(dispatch_gather_kernel), static_cast<int>(gsm));
   if (err != cudaSuccess) return err;
   const int ctas_per_sm = std::max(1, static_cast<int>((200 * 1024) / gsm));
   const int grid = std::max(1, std::min((N + GW - 1) / GW, num_sms() * ctas_per_sm));
-  dispatch_gather_kernel<<<grid, GW * 32, gsm, s>>>(static_cast<const uint8_t*>(x), packed_tok,
-                                                     offsets, E, row_bytes,
-                                                     static_cast<uint8_t*>(x_packed), status);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(GW * 32), gsm, s, 0,
+                    static_cast<const uint8_t*>(x), static_cast<const int32_t*>(packed_tok),
+                    static_cast<const int32_t*>(offsets), E, row_bytes,
+                    static_cast<uint8_t*>(x_packed), status);
 }
 
 }  // namespace moe_host

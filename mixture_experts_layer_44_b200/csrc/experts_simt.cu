@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* __restrict_
   __shared__ __align__(16) float As[SBK][SBM + 4];
   __shared__ __align__(16) float Bs[SBK][NB + 4];
 
+  moe::grid_dep_wait();
   build_tiles(offsets, E, offs, tstart);
   const int t = blockIdx.x;
   if (t >= tstart[E]) return;
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* __restrict_
       out[static_cast<size_t>(gr) * ldo + gc] = v;
     }
   }
+  moe::grid_dep_launch();
 }
 
 }  // namespace
@@ -130,14 +132,16 @@ cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
                                 int H, int I, int E, void* h, void* y, cudaStream_t s) {
   const int mt_bound = (N + SBM - 1) / SBM + E;
   dim3 g1(mt_bound, (I + SBN - 1) / SBN);
-  simt_gemm_kernel<EPI_SWIGLU><<<g1, SNT, 0, s>>>(static_cast<const float*>(x_packed), H,
-                                                  offsets, E, static_cast<const float*>(w13),
-                                                  2 * I, I, nullptr, static_cast<float*>(h), I);
+  const float* no_w = nullptr;
+  cudaError_t err = launch_pdl(simt_gemm_kernel<EPI_SWIGLU>, g1, dim3(SNT), 0, s, 0,
+                               static_cast<const float*>(x_packed), H, offsets, E,
+                               static_cast<const float*>(w13), 2 * I, I, no_w,
+                               static_cast<float*>(h), I);
+  if (err != cudaSuccess) return err;
   dim3 g2(mt_bound, (H + SBN - 1) / SBN);
-  simt_gemm_kernel<EPI_SCALE><<<g2, SNT, 0, s>>>(static_cast<const float*>(h), I, offsets, E,
-                                                 static_cast<const float*>(w2), H, I, packed_w,
-                                                 static_cast<float*>(y), H);
-  return cudaGetLastError();
+  return launch_pdl(simt_gemm_kernel<EPI_SCALE>, g2, dim3(SNT), 0, s, 0,
+                    static_cast<const float*>(h), I, offsets, E, static_cast<const float*>(w2), H,
+                    I, packed_w, static_cast<float*>(y), H);
 }
 
 }  // namespace moe_host

@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
     moe::tmem_relinquish();
   }
+  moe::grid_dep_wait();        // offsets and the A operand come from the previous kernels
   if (warp == 2) {
     // Tile table: per-expert token-tile counts, exclusive scan, x ntw.
     // Lane l owns experts [8l, 8l+8); lane 31 also writes the end entries.
@@ -454,6 +455,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
 
+  moe::grid_dep_launch();
   moe::tc_fence_before();
   __syncthreads();
   moe::tc_fence_after();
@@ -593,13 +595,14 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     g1 = std::max(1, std::min(sms, mt_bound * (I / (BN / 2))));
     g2 = std::max(1, std::min(sms, mt_bound * (H / BN)));
   }
-  grouped_gemm_kernel<EPI_SWIGLU><<<g1, NTHREADS, SMEM_BYTES, s>>>(
-      mA1, mB1, offsets, E, H, I / (BN / 2), 2 * I, nullptr, h, I, counters, partials,
-      max_units, status);
-  grouped_gemm_kernel<EPI_SCALE><<<g2, NTHREADS, SMEM_BYTES, s>>>(
-      mA2, mB2, offsets, E, I, H / BN, H, packed_w, y, H, counters, partials, max_units,
-      status);
-  return cudaGetLastError();
+  const float* no_w = nullptr;
+  cudaError_t err = launch_pdl(grouped_gemm_kernel<EPI_SWIGLU>, dim3(g1), dim3(NTHREADS),
+                               SMEM_BYTES, s, 0, mA1, mB1, offsets, E, H, I / (BN / 2), 2 * I,
+                               no_w, h, I, counters, partials, max_units, status);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(grouped_gemm_kernel<EPI_SCALE>, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
+                    mA2, mB2, offsets, E, I, H / BN, H, packed_w, y, H, counters, partials,
+                    max_units, status);
 }
 
 }  // namespace moe_host

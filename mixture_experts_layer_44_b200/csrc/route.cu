@@ -6,13 +6,15 @@
 // diffulex.moe API reference, "diffulex.moe.topk": NaiveTopKRouter.
 //
 // Batches of more than 64 tokens (or more than 64 experts): a thread-block
-// cluster of S CTAs (S <= 8) owns BT = 64 tokens and all E
-// experts; CTA s of the cluster contracts its own slice of H.  Each CTA
-// stages chunks of KC = 32 columns of x and W_gate (converted to fp32,
-// transposed) in shared memory, prefetching the next chunk into registers
-// while it computes the current one, and accumulates a 4-token x
-// (EPAD/16)-expert register tile per thread (EPAD = 64, 128 or 256: E rounded
-// up).  The S partial logit tiles are then summed through distributed shared
+// cluster of S CTAs (S <= 8) owns BT = 16*TT tokens and all E experts; CTA s
+// of the cluster contracts its own slice of H.  Each CTA stages chunks of
+// KC = 32 columns of x and W_gate (converted to fp32, transposed, without
+// bank conflicts) in double-buffered shared memory, prefetching the next
+// chunk into registers while it computes the current one, and accumulates a
+// TT-token x (EPAD/16)-expert register tile per thread (EPAD = 64, 128 or
+// 256: E rounded up; TT = 8 for EPAD = 64, else 4).  Thread eg owns experts
+// 64*(j/4) + 4*eg + (j%4): each of its float4 reads of W is part of 256
+// contiguous bytes across the warp, free of bank conflicts.  The S partial logit tiles are then summed through distributed shared
 // memory in a fixed rank order (deterministic, no global scratch): CTA s
 // finalises tokens [s*BT/S, (s+1)*BT/S) of the tile, one warp per token, which
 // adds the bias, writes the logits and selects the top k by k rounds of a warp
@@ -28,9 +30,7 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int BT = 64;    // tokens per cluster
 constexpr int KC = 32;    // H chunk
-constexpr int TT = 4;     // tokens per thread
 constexpr int NT = 256;   // threads per CTA
 constexpr int MAX_S = 8;  // CTAs per cluster
 
@@ -123,11 +123,13 @@ __device__ __forceinline__ void select_topk(const float* v, const bool* live, in
 }
 
 // Small batches (T <= 64 tokens, E <= 64 experts: decode): one CTA per token.
-// The 256 threads cover H in one pass of 8-element vectors (thread i takes
-// vectors i, i+256, ...) and keep one partial dot product per expert; the
-// partials are reduced in a fixed order (warp shuffle tree, then warps in
-// order), so the logits do not depend on timing.  Warp 0 then selects.
-template <bool BF16>
+// With EP = E rounded up to a power of two, thread i owns expert i % EP and
+// the 8-element H-vectors v = i / EP + j * (256 / EP); it issues the loads of
+// 16 vectors at a time before any FMA, so a token costs a few memory round
+// trips.  Partials are reduced in a fixed order (lanes of the same expert by
+// a shuffle tree, then warps in order), so the logits do not depend on timing.
+// Warp 0 then selects.
+template <int EP, bool BF16>
 __global__ void __launch_bounds__(NT) route_small_kernel(const void* __restrict__ xv,
                                                          const void* __restrict__ wv,
                                                          const float* __restrict__ bias, int H,
@@ -135,51 +137,76 @@ __global__ void __launch_bounds__(NT) route_small_kernel(const void* __restrict_
                                                          float* __restrict__ logits,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ wout) {
-  constexpr int EMAX = 64;
-  __shared__ float part[NT / 32][EMAX];
+  constexpr int TPE = NT / EP;                 // threads per expert
+  constexpr int BATCH = 16;
+  __shared__ float part[NT / 32][64];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[EMAX];
-#pragma unroll
-  for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+  const int e = threadIdx.x % EP;
+  const int v0 = threadIdx.x / EP;
   const int nvec = H / 8;
-  for (int v = threadIdx.x; v < nvec; v += NT) {
-    float xf[8];
-    load8<BF16>(xv, static_cast<size_t>(t) * H + v * 8, true, xf);
+  moe::grid_dep_wait();
+  float acc = 0.f;
+  if (e < E) {
+    // 8 elements = one uint4 (bf16) or two (fp32); loads are unconditional
+    // (clamped to the last vector) so that all of a batch are in flight.
+    constexpr int Q = BF16 ? 1 : 2;
+    const uint4* xb = reinterpret_cast<const uint4*>(xv) + static_cast<size_t>(t) * (nvec * Q);
+    const uint4* wb = reinterpret_cast<const uint4*>(wv) + static_cast<size_t>(e) * (nvec * Q);
+    for (int vb = v0; vb < nvec; vb += BATCH * TPE) {
+      uint4 xq[BATCH][Q], wq[BATCH][Q];
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < E) {
-        float wf[8];
-        load8<BF16>(wv, static_cast<size_t>(e) * H + v * 8, true, wf);
+      for (int j = 0; j < BATCH; ++j) {
+        const int vc = min(vb + j * TPE, nvec - 1);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[e] = fmaf(xf[j], wf[j], acc[e]);
+        for (int q = 0; q < Q; ++q) {
+          xq[j][q] = __ldg(xb + vc * Q + q);
+          wq[j][q] = __ldg(wb + vc * Q + q);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j) {
+        if (vb + j * TPE >= nvec) break;
+        float xf[8], wf[8];
+        if (BF16) {
+          moe::unpack8(xq[j][0], xf);
+          moe::unpack8(wq[j][0], wf);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            xf[4 * q] = __uint_as_float(xq[j][q].x); xf[4 * q + 1] = __uint_as_float(xq[j][q].y);
+            xf[4 * q + 2] = __uint_as_float(xq[j][q].z); xf[4 * q + 3] = __uint_as_float(xq[j][q].w);
+            wf[4 * q] = __uint_as_float(wq[j][q].x); wf[4 * q + 1] = __uint_as_float(wq[j][q].y);
+            wf[4 * q + 2] = __uint_as_float(wq[j][q].z); wf[4 * q + 3] = __uint_as_float(wq[j][q].w);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc = fmaf(xf[q], wf[q], acc);
       }
     }
   }
+  // lanes holding the same expert: lane, lane + EP, ... inside a warp
 #pragma unroll
-  for (int e = 0; e < EMAX; ++e) {
-    if (e < E) {
-      float a = acc[e];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) part[warp][e] = a;
-    }
-  }
+  for (int o = 16; o >= EP && o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane < (EP < 32 ? EP : 32)) part[warp][e] = acc;
   __syncthreads();
+  moe::grid_dep_launch();
   if (warp != 0) return;
-  constexpr int PER = EMAX / 32;
+  constexpr int PER = 2;                       // experts lane, lane + 32
   float v[PER];
   bool live[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
-    const int e = lane + 32 * j;
-    live[j] = e < E;
+    const int ex = lane + 32 * j;
+    live[j] = ex < E;
     float s = 0.f;
     if (live[j]) {
+      // warps holding expert ex: those whose lanes cover ex % EP
 #pragma unroll
-      for (int w = 0; w < NT / 32; ++w) s += part[w][e];
-      s += bias ? bias[e] : 0.f;
-      logits[static_cast<size_t>(t) * E + e] = s;
+      for (int w = 0; w < NT / 32; ++w)
+        if (EP <= 32 || (w * 32) % EP == (ex / 32) * 32 % EP) s += part[w][ex];
+      s += bias ? bias[ex] : 0.f;
+      logits[static_cast<size_t>(t) * E + ex] = s;
     }
     v[j] = live[j] ? s : -FLT_MAX;
   }
@@ -187,6 +214,15 @@ __global__ void __launch_bounds__(NT) route_small_kernel(const void* __restrict_
   select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
                    wout + static_cast<size_t>(t) * k);
 }
+
+// Token rows per thread: 8 when E <= 64 (more FMAs per shared-memory read),
+// else 4.  A cluster then owns 16 * TT tokens.
+template <int EPAD>
+struct Tile {
+  static constexpr int TT = EPAD == 64 ? 8 : 4;
+  static constexpr int BT = 16 * TT;
+  static constexpr int TE = EPAD / 16;
+};
 
 template <int EPAD, bool BF16>
 __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
@@ -196,13 +232,18 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
                                                    float* __restrict__ logits,
                                                    int32_t* __restrict__ ids,
                                                    float* __restrict__ wout) {
-  constexpr int TE = EPAD / 16;            // experts per thread
-  constexpr int LS = EPAD + 1;             // padded row of the logits tile
-  constexpr int WV = EPAD * (KC / 8) / NT; // W_gate vectors per thread per chunk (1, 2 or 4)
+  constexpr int TT = Tile<EPAD>::TT;
+  constexpr int BTC = Tile<EPAD>::BT;        // tokens per cluster
+  constexpr int TE = Tile<EPAD>::TE;         // experts per thread
+  constexpr int LS = EPAD + 1;               // padded row of the logits tile
+  constexpr int XV = BTC * (KC / 8) / NT;    // x vectors per thread per chunk (1 or 2)
+  constexpr int WV = EPAD * (KC / 8) / NT;   // W_gate vectors per thread per chunk (1, 2 or 4)
+  constexpr int XS = KC * BTC;               // one x buffer  [KC][BTC]
+  constexpr int WS = KC * EPAD;              // one W buffer  [KC][EPAD]
   extern __shared__ __align__(16) float sm[];
-  float* x_s = sm;                         // [KC][BT]
-  float* w_s = sm + KC * BT;               // [KC][EPAD]
-  float* l_s = sm + KC * BT + KC * EPAD;   // [BT][LS] partial logits of this CTA
+  float* x_s = sm;                           // [2][KC][BTC]
+  float* w_s = sm + 2 * XS;                  // [2][KC][EPAD]
+  float* l_s = sm;                           // [BTC][LS] partial logits (after the loop)
 
   cg::cluster_group cluster = cg::this_cluster();
   const int S = static_cast<int>(cluster.num_blocks());
@@ -210,7 +251,7 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
   const int tid = threadIdx.x;
   const int eg = tid & 15;
   const int tg = tid >> 4;
-  const int t0 = blockIdx.y * BT;
+  const int t0 = blockIdx.y * BTC;
   const int h_begin = rank * kc_per_cta * KC;
   const int h_end = min(H, h_begin + kc_per_cta * KC);
 
@@ -220,44 +261,66 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
 #pragma unroll
     for (int j = 0; j < TE; ++j) acc[i][j] = 0.f;
 
-  // Register staging of one chunk: x (one 8-vector per thread), W (WV 8-vectors).
-  const int xt = tid >> 2, xv8 = tid & 3;
-  float xr[8], wr[WV][8];
+  // Register staging of one chunk.  Vector i of the x chunk is token
+  // (i % BTC), columns 8*(i / BTC) .. +8, so a warp stores 32 consecutive
+  // tokens of one column group: no shared-memory bank conflicts.  W likewise.
+  float xr[XV][8], wr[WV][8];
   auto fetch = [&](int h0) {
-    const int hh = h0 + xv8 * 8;
-    load8<BF16>(xv, static_cast<size_t>(t0 + xt) * H + hh, t0 + xt < T && hh < h_end, xr);
+#pragma unroll
+    for (int u = 0; u < XV; ++u) {
+      const int i = tid + u * NT;
+      const int t = i % BTC, hh = h0 + (i / BTC) * 8;
+      load8<BF16>(xv, static_cast<size_t>(t0 + t) * H + hh, t0 + t < T && hh < h_end, xr[u]);
+    }
 #pragma unroll
     for (int u = 0; u < WV; ++u) {
       const int i = tid + u * NT;
-      const int e = i >> 2, hv = h0 + (i & 3) * 8;
+      const int e = i % EPAD, hv = h0 + (i / EPAD) * 8;
       load8<BF16>(wv, static_cast<size_t>(e) * H + hv, e < E && hv < h_end, wr[u]);
     }
   };
-  auto stash = [&]() {
+  auto stash = [&](int b) {
+    float* xs = x_s + b * XS;
+    float* ws = w_s + b * WS;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) x_s[(xv8 * 8 + j) * BT + xt] = xr[j];
+    for (int u = 0; u < XV; ++u) {
+      const int i = tid + u * NT;
+      const int t = i % BTC, v = i / BTC;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[(v * 8 + j) * BTC + t] = xr[u][j];
+    }
 #pragma unroll
     for (int u = 0; u < WV; ++u) {
       const int i = tid + u * NT;
-      const int e = i >> 2, v = i & 3;
+      const int e = i % EPAD, v = i / EPAD;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) w_s[(v * 8 + j) * EPAD + e] = wr[u][j];
+      for (int j = 0; j < 8; ++j) ws[(v * 8 + j) * EPAD + e] = wr[u][j];
     }
   };
 
-  if (h_begin < h_end) fetch(h_begin);
-  for (int h0 = h_begin; h0 < h_end; h0 += KC) {
-    stash();
-    __syncthreads();
-    if (h0 + KC < h_end) fetch(h0 + KC);        // next chunk in flight during the FMAs
+  moe::grid_dep_wait();
+  if (h_begin < h_end) {
+    fetch(h_begin);
+    stash(0);
+  }
+  __syncthreads();
+  int b = 0;
+  for (int h0 = h_begin; h0 < h_end; h0 += KC, b ^= 1) {
+    const bool more = h0 + KC < h_end;
+    if (more) fetch(h0 + KC);                  // next chunk in flight during the FMAs
+    const float* xs = x_s + b * XS;
+    const float* ws = w_s + b * WS;
 #pragma unroll 8
     for (int kk = 0; kk < KC; ++kk) {
-      const float4 xq = *reinterpret_cast<const float4*>(&x_s[kk * BT + tg * TT]);
-      const float xa[TT] = {xq.x, xq.y, xq.z, xq.w};
-      float wa[TE];
+      float xa[TT], wa[TE];
 #pragma unroll
-      for (int j = 0; j < TE; j += 4) {
-        const float4 q = *reinterpret_cast<const float4*>(&w_s[kk * EPAD + eg * TE + j]);
+      for (int i = 0; i < TT; i += 4) {
+        const float4 q = *reinterpret_cast<const float4*>(&xs[kk * BTC + tg * TT + i]);
+        xa[i] = q.x; xa[i + 1] = q.y; xa[i + 2] = q.z; xa[i + 3] = q.w;
+      }
+#pragma unroll
+      for (int j = 0; j < TE; j += 4) {             // experts 64*(j/4) + 4*eg + 0..3
+        const float4 q = *reinterpret_cast<const float4*>(&ws[kk * EPAD + (j / 4) * 64 + eg * 4]);
         wa[j] = q.x; wa[j + 1] = q.y; wa[j + 2] = q.z; wa[j + 3] = q.w;
       }
 #pragma unroll
@@ -265,21 +328,23 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
 #pragma unroll
         for (int j = 0; j < TE; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
     }
+    if (more) stash(b ^ 1);                    // the other buffer was released by the last barrier
     __syncthreads();
   }
 
-  // This CTA's partial logits tile.
+  moe::grid_dep_launch();
+  // This CTA's partial logits tile (aliases the staging buffers, now idle).
 #pragma unroll
   for (int i = 0; i < TT; ++i)
 #pragma unroll
-    for (int j = 0; j < TE; ++j) l_s[(tg * TT + i) * LS + eg * TE + j] = acc[i][j];
+    for (int j = 0; j < TE; ++j) l_s[(tg * TT + i) * LS + (j / 4) * 64 + eg * 4 + (j % 4)] = acc[i][j];
   cluster.sync();
 
-  // Finalise tokens [rank*BT/S, (rank+1)*BT/S): one warp per token.
+  // Finalise tokens [rank*BTC/S, (rank+1)*BTC/S): one warp per token.
   constexpr int PER = EPAD / 32;
   const int warp = tid >> 5, lane = tid & 31;
-  const int per_cta = (BT + S - 1) / S;
-  const int tl_end = min(BT, (rank + 1) * per_cta);
+  const int per_cta = (BTC + S - 1) / S;
+  const int tl_end = min(BTC, (rank + 1) * per_cta);
   for (int tl = rank * per_cta + warp; tl < tl_end; tl += NT / 32) {
     const int t = t0 + tl;
     if (t >= T) break;
@@ -287,8 +352,7 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
     bool live[PER];
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
-      const int e = lane + 32 * j;
-      live[j] = e < E;
+      live[j] = lane + 32 * j < E;
       v[j] = 0.f;
     }
     for (int r = 0; r < S; ++r) {               // fixed order: deterministic sum
@@ -317,31 +381,20 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
 template <int EPAD, bool BF16>
 cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H, int E, int k,
                      int renorm, float* logits, int32_t* ids, float* w, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (KC * BT + KC * EPAD + BT * (EPAD + 1));
+  constexpr int BTC = Tile<EPAD>::BT;
+  const size_t smem =
+      sizeof(float) * std::max(2 * (KC * BTC + KC * EPAD), BTC * (EPAD + 1));
   auto fn = route_kernel<EPAD, BF16>;
   cudaError_t err = moe_host::ensure_smem(reinterpret_cast<const void*>(fn), (int)smem);
   if (err != cudaSuccess) return err;
-  const int tiles = (T + BT - 1) / BT;
+  const int tiles = (T + BTC - 1) / BTC;
   const int chunks = (H + KC - 1) / KC;
   // Enough CTAs for ~4 per SM, never more than one chunk of H each.
   int S = (4 * moe_host::num_sms() + tiles - 1) / tiles;
   S = std::max(1, std::min({S, MAX_S, chunks}));
   const int kc_per_cta = (chunks + S - 1) / S;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, tiles, 1);
-  cfg.blockDim = dim3(NT, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, fn, x, W, b, T, H, E, k, renorm, kc_per_cta, logits, ids, w);
-  if (err != cudaSuccess) return err;
-  return cudaGetLastError();
+  return moe_host::launch_pdl(fn, dim3(S, tiles, 1), dim3(NT, 1, 1), smem, s, S, x, W, b, T, H,
+                              E, k, renorm, kc_per_cta, logits, ids, w);
 }
 
 }  // namespace
@@ -353,13 +406,22 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
                          float* w, cudaStream_t s) {
   const bool bf = dtype == MOE_BF16;
   if (T <= 64 && E <= 64) {
-    if (bf)
-      route_small_kernel<true><<<T, NT, 0, s>>>(x, W_gate, bias, H, E, k, renormalize, logits,
-                                                ids, w);
-    else
-      route_small_kernel<false><<<T, NT, 0, s>>>(x, W_gate, bias, H, E, k, renormalize, logits,
-                                                 ids, w);
-    return cudaGetLastError();
+#define MOE_SMALL_CASE(EPV)                                                                   \
+    if (E <= EPV) {                                                                         \
+      if (bf)                                                                               \
+        return launch_pdl(route_small_kernel<EPV, true>, dim3(T), dim3(NT), 0, s, 0, x,       \
+                          W_gate, bias, H, E, k, renormalize, logits, ids, w);              \
+      return launch_pdl(route_small_kernel<EPV, false>, dim3(T), dim3(NT), 0, s, 0, x, W_gate,  \
+                        bias, H, E, k, renormalize, logits, ids, w);                        \
+    }
+    MOE_SMALL_CASE(1)
+    MOE_SMALL_CASE(2)
+    MOE_SMALL_CASE(4)
+    MOE_SMALL_CASE(8)
+    MOE_SMALL_CASE(16)
+    MOE_SMALL_CASE(32)
+    MOE_SMALL_CASE(64)
+#undef MOE_SMALL_CASE
   }
 #define MOE_ROUTE_CASE(EP)                                                                  \
   if (E <= EP)                                                                              \
