@@ -23,7 +23,7 @@ namespace {
 
 constexpr int CNT = 256;
 
-template <bool OUT_BF16>
+template <bool OUT_BF16, int KT>
 __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ y,
                                                       const int32_t* __restrict__ inv_perm,
                                                       int T, int H, int k, int N,
@@ -50,13 +50,23 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      for (int j = 0; j < k; ++j) {
-        const int p = rows[j];
-        if (p < 0) continue;
-        const float4* src = reinterpret_cast<const float4*>(y + static_cast<size_t>(p) * H) + 2 * v;
-        const float4 a = src[0], b = src[1];
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      // all k rows' loads first (in flight together), then the sums in j order
+      float4 a[KT], b[KT];
+#pragma unroll
+      for (int j = 0; j < KT; ++j) {
+        if (rows[j] >= 0) {
+          const float4* src =
+              reinterpret_cast<const float4*>(y + static_cast<size_t>(rows[j]) * H) + 2 * v;
+          a[j] = src[0];
+          b[j] = src[1];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < KT; ++j) {
+        if (rows[j] >= 0) {
+          acc[0] += a[j].x; acc[1] += a[j].y; acc[2] += a[j].z; acc[3] += a[j].w;
+          acc[4] += b[j].x; acc[5] += b[j].y; acc[6] += b[j].z; acc[7] += b[j].w;
+        }
       }
       if (shared) {
         const float g = gate;
@@ -90,11 +100,27 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
                            int32_t* status, cudaStream_t s) {
   const int grid = std::max(1, std::min(T, num_sms() * 8));
   const int N = T * k;
-  if (dtype == MOE_BF16)
-    return launch_pdl(combine_kernel<true>, dim3(grid), dim3(CNT), 0, s, 0, y, inv_perm, T, H, k,
-                      N, shared, shared_gate, out, status);
-  return launch_pdl(combine_kernel<false>, dim3(grid), dim3(CNT), 0, s, 0, y, inv_perm, T, H, k,
-                    N, shared, shared_gate, out, status);
+  // k is a template parameter so that exactly k rows are loaded, all in flight.
+#define MOE_COMBINE_K(KV)                                                                     \
+  case KV:                                                                                    \
+    return dtype == MOE_BF16                                                                  \
+               ? launch_pdl(combine_kernel<true, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,       \
+                            inv_perm, T, H, k, N, shared, shared_gate, out, status)           \
+               : launch_pdl(combine_kernel<false, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,      \
+                            inv_perm, T, H, k, N, shared, shared_gate, out, status);
+  switch (k) {
+    MOE_COMBINE_K(1)
+    MOE_COMBINE_K(2)
+    MOE_COMBINE_K(3)
+    MOE_COMBINE_K(4)
+    MOE_COMBINE_K(5)
+    MOE_COMBINE_K(6)
+    MOE_COMBINE_K(7)
+    MOE_COMBINE_K(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef MOE_COMBINE_K
 }
 
 }  // namespace moe_host

@@ -8,8 +8,8 @@
 //
 // Small batches (N <= 8192 assignments) take one CTA of 32 warps through
 // count, scan and scatter in a single launch (the same warp-slice algorithm
-// as below), and also gather the rows when they total at most 1 MiB (decode);
-// larger gathers use the bulk-copy kernel.  Larger N takes four launches:
+// as below), and also gather the rows when they total at most 128 KiB
+// (decode); larger gathers use the bulk-copy kernel.  Larger N takes four launches:
 //   count   -- each CTA owns CHUNK consecutive assignments; each warp owns a
 //              contiguous CHUNK/8 slice and counts it per expert with
 //              __match_any_sync (one shared-memory add per distinct expert
@@ -251,12 +251,21 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
   moe::grid_dep_launch();
   if (x == nullptr) return;
   __syncthreads();
-  // 4. gather (small total): one warp per row, 16-byte vectors
+  // 4. gather (small total): one warp per row, 16-byte vectors, 8 loads in
+  //    flight per lane before the stores
   const int nrows = s_scan[moe::kMaxExperts - 1];
   for (int p = warp; p < nrows; p += SMALL_WARPS) {
     const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
-    for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+    for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) q[j] = src[v0 + 32 * j];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];
+    }
   }
 }
 
@@ -326,7 +335,15 @@ __global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
        p += (gridDim.x * blockDim.x) >> 5) {
     const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
-    for (int v = lane; v < row_vecs; v += 32) dst[v] = src[v];
+    for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) q[j] = src[v0 + 32 * j];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];
+    }
   }
   moe::grid_dep_launch();
 }
@@ -361,8 +378,9 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
   const int es = dtype == MOE_BF16 ? 2 : 4;
   const int row_bytes = H * es;
   if (N <= SMALL_N) {
+    // One CTA copies at most 128 KiB of rows; more goes to the multi-CTA gather.
     const bool fuse_gather =
-        x != nullptr && static_cast<size_t>(N) * row_bytes <= (static_cast<size_t>(1) << 20);
+        x != nullptr && static_cast<size_t>(N) * row_bytes <= (static_cast<size_t>(128) << 10);
     cudaError_t err = launch_pdl(
         dispatch_small_kernel, dim3(1), dim3(SMALL_WARPS * 32), sizeof(int) * SMALL_WARPS * E, s,
         0, ids, w, N, E, k, counts, offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,

@@ -32,6 +32,13 @@
 // slice order (deterministic) and applies the epilogue.  The counter returns
 // to zero for the next call.
 //
+// Scheduling.  CTA b starts with unit b.  With a workspace, later units are
+// handed out dynamically: the producer warp takes the next unit from a
+// global ticket counter and passes its id to the MMA and epilogue warps
+// through a small shared-memory ring, so a CTA whose units run fast takes more
+// of them; the last CTA to exit resets the ticket for the next launch.
+// Without one, CTA b takes units b, b+grid, b+2*grid, ...
+//
 // CTA = 6 warps, one CTA per SM, persistent over units:
 //   warp 0    TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
 //   warp 1    MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
@@ -63,7 +70,10 @@ constexpr int NTHREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
 constexpr int MAX_SPLITS = 16;
-constexpr int COUNTER_INTS = 4096;                        // per-tile arrival counters
+constexpr int COUNTER_INTS = 4096;                        // per-tile arrival counters, then
+constexpr int SCHED_TICKET = COUNTER_INTS - 2;            // the unit ticket and the
+constexpr int SCHED_DONE = COUNTER_INTS - 1;              // CTA exit count of dynamic scheduling
+constexpr int UNIT_RING = 8;                              // unit ids handed from producer to consumers
 constexpr size_t PARTIAL_BYTES = sizeof(float) * BM * BN;  // one unit's partial slot
 
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
@@ -74,6 +84,9 @@ struct Ctl {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
+  uint64_t ufull[UNIT_RING];    // producer -> MMA + epilogue: unit id published
+  uint64_t uempty[UNIT_RING];   // MMA + 4 epilogue warps -> producer: slot read
+  int uid[UNIT_RING];
   uint32_t tmem_base;
   int abort;
   int splits;          // S: K-slices per tile (1 = no split)
@@ -192,6 +205,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       moe::mbar_init(moe::smem_addr(&c.tempty[b]), 4);
     }
     moe::mbar_init(moe::smem_addr(&c.drain), 1);
+    for (int r = 0; r < UNIT_RING; ++r) {
+      moe::mbar_init(moe::smem_addr(&c.ufull[r]), 1);
+      moe::mbar_init(moe::smem_addr(&c.uempty[r]), 5);
+    }
     c.abort = 0;
     moe::fence_barrier_init();
     moe::prefetch_tmap(&tmA);
@@ -234,7 +251,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 31) {
       c.offs[E] = offsets[E];
       c.tstart[E] = incl * ntw;
-      c.splits = (counters != nullptr && partials != nullptr && incl * ntw <= COUNTER_INTS)
+      c.splits = (counters != nullptr && partials != nullptr && incl * ntw <= SCHED_TICKET)
                      ? choose_splits(incl * ntw, gridDim.x, kblocks, max_units)
                      : 1;
     }
@@ -252,8 +269,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ------------------------------------------------------ producer ---
       int stage = 0;
       uint32_t phase = 0;
-      int issued[STAGES] = {0, 0, 0, 0};
-      for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x) {
+      int issued[STAGES] = {};
+      int uslot = 0;
+      uint32_t uphase = 0;
+      int next_static = blockIdx.x;
+      for (;;) {
+        // Take the next unit and publish its id (-1: no more work) to the consumers.
+        if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1)) {
+          set_abort(c, status);
+          break;
+        }
+        int u;
+        if (next_static == static_cast<int>(blockIdx.x) || counters == nullptr) {
+          u = next_static;                    // the first unit of every CTA is static
+          next_static += gridDim.x;
+        } else {
+          u = gridDim.x + atomicAdd(&counters[SCHED_TICKET], 1);
+        }
+        if (u >= total || aborted(c)) u = -1;
+        c.uid[uslot] = u;
+        moe::mbar_arrive(moe::smem_addr(&c.ufull[uslot]));
+        if (++uslot == UNIT_RING) {
+          uslot = 0;
+          uphase ^= 1;
+        }
+        if (u < 0) break;
         const Unit un = decode_unit(c, E, kblocks, u);
         const int arow = c.offs[un.e] + un.mt * BM;
         bool ok = true;
@@ -289,7 +329,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
-      for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x, ++i) {
+      int uslot = 0;
+      uint32_t uphase = 0;
+      for (;; ++i) {
+        if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase)) {
+          set_abort(c, status);
+          break;
+        }
+        const int u = c.uid[uslot];
+        moe::mbar_arrive(moe::smem_addr(&c.uempty[uslot]));
+        if (++uslot == UNIT_RING) {
+          uslot = 0;
+          uphase ^= 1;
+        }
+        if (u < 0) break;
         const Unit un = decode_unit(c, E, kblocks, u);
         const int buf = i & 1;
         if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
@@ -331,7 +384,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;          // row of the tile owned by this thread
     int i = 0;
-    for (int u = blockIdx.x; u < total && !aborted(c); u += gridDim.x, ++i) {
+    int uslot = 0;
+    uint32_t uphase = 0;
+    for (;; ++i) {
+      if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase)) {
+        set_abort(c, status);
+        break;
+      }
+      const int u = c.uid[uslot];
+      __syncwarp();
+      if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.uempty[uslot]));
+      if (++uslot == UNIT_RING) {
+        uslot = 0;
+        uphase ^= 1;
+      }
+      if (u < 0) break;
       const int buf = i & 1;
       if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1)) {
         set_abort(c, status);
@@ -405,49 +472,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const bool last = c.last_flag != 0;
         epi_bar();                               // everyone read the flag before it changes
         if (last) {
+          // All 128 epilogue threads reduce the tile: the S partials of every
+          // valid row, summed in slice order (loads of one output batched
+          // across slices so they are in flight together).
           __threadfence();
-          if (live) {
-            const float* base = partials + static_cast<size_t>(un.tile) * S * (BM * BN) +
-                                static_cast<size_t>(row) * BN;
-            if (EPI == EPI_SWIGLU) {
-              __nv_bfloat16* dst =
-                  static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
-#pragma unroll 1
-              for (int cc = 0; cc < BN / 2; cc += 16) {
-                float g[16], v[16];
+          const int et = threadIdx.x - 64;                // 0..127
+          const int nrows = min(rows_valid, BM);
+          const size_t row0 = static_cast<size_t>(c.offs[un.e] + un.mt * BM);
+          const float* base = partials + static_cast<size_t>(un.tile) * S * (BM * BN);
+          if (EPI == EPI_SWIGLU) {
+            const int cg = et & 31;                       // h columns 4cg .. 4cg+3
+            for (int r = et >> 5; r < nrows; r += 4) {
+              float4 g = make_float4(0.f, 0.f, 0.f, 0.f), v = g;
+              const float* pr = base + static_cast<size_t>(r) * BN + cg * 4;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) g[j] = v[j] = 0.f;
-                for (int s = 0; s < S; ++s) {           // slice order: deterministic
-                  const float4* pg = reinterpret_cast<const float4*>(base + s * (BM * BN) + cc);
-                  const float4* pu =
-                      reinterpret_cast<const float4*>(base + s * (BM * BN) + BN / 2 + cc);
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float4 x = __ldcg(pg + j), y = __ldcg(pu + j);
-                    g[4 * j] += x.x; g[4 * j + 1] += x.y; g[4 * j + 2] += x.z; g[4 * j + 3] += x.w;
-                    v[4 * j] += y.x; v[4 * j + 1] += y.y; v[4 * j + 2] += y.z; v[4 * j + 3] += y.w;
-                  }
+              for (int s = 0; s < MAX_SPLITS; ++s) {
+                if (s < S) {
+                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN)));
+                  const float4 b =
+                      __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN) + BN / 2));
+                  g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
+                  v.x += b.x; v.y += b.y; v.z += b.z; v.w += b.w;
                 }
-                store_h16(dst + cc, g, v);
               }
-            } else {
-              const float sc = packed_w ? packed_w[grow] : 1.f;
-              float* dst = static_cast<float*>(out) + grow * ldo + un.nt * BN;
-#pragma unroll 1
-              for (int cc = 0; cc < BN; cc += 16) {
-                float v[16];
+              uint2 pk;
+              pk.x = moe::pack_bf16x2(silu_mul(g.x, v.x), silu_mul(g.y, v.y));
+              pk.y = moe::pack_bf16x2(silu_mul(g.z, v.z), silu_mul(g.w, v.w));
+              *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + (row0 + r) * ldo +
+                                        un.nt * (BN / 2) + cg * 4) = pk;
+            }
+          } else {
+            const int cg = et & 63;                       // y columns 4cg .. 4cg+3
+            for (int r = et >> 6; r < nrows; r += 2) {
+              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+              const float* pr = base + static_cast<size_t>(r) * BN + cg * 4;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = 0.f;
-                for (int s = 0; s < S; ++s) {
-                  const float4* p = reinterpret_cast<const float4*>(base + s * (BM * BN) + cc);
-#pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float4 x = __ldcg(p + j);
-                    v[4 * j] += x.x; v[4 * j + 1] += x.y; v[4 * j + 2] += x.z; v[4 * j + 3] += x.w;
-                  }
+              for (int s = 0; s < MAX_SPLITS; ++s) {
+                if (s < S) {
+                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN)));
+                  v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
                 }
-                store_y16(dst + cc, v, sc);
               }
+              const float sc = packed_w ? packed_w[row0 + r] : 1.f;
+              *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + r) * ldo +
+                                         un.nt * BN + cg * 4) =
+                  make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
             }
           }
         }
@@ -460,6 +529,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   moe::tc_fence_after();
   if (warp == 1) moe::tmem_dealloc(tmem, TMEM_COLS);
+  if (threadIdx.x == 0 && counters != nullptr) {
+    // The last CTA to leave returns the ticket (and the exit count) to zero.
+    __threadfence();
+    if (atomicAdd(&counters[SCHED_DONE], 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(&counters[SCHED_TICKET], 0);
+      atomicExch(&counters[SCHED_DONE], 0);
+    }
+  }
 }
 
 // ------------------------------------------------------ tensor maps ---

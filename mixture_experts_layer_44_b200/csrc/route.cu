@@ -122,66 +122,75 @@ __device__ __forceinline__ void select_topk(const float* v, const bool* live, in
   }
 }
 
-// Small batches (T <= 64 tokens, E <= 64 experts: decode): one CTA per token.
-// With EP = E rounded up to a power of two, thread i owns expert i % EP and
-// the 8-element H-vectors v = i / EP + j * (256 / EP); it issues the loads of
-// 16 vectors at a time before any FMA, so a token costs a few memory round
-// trips.  Partials are reduced in a fixed order (lanes of the same expert by
-// a shuffle tree, then warps in order), so the logits do not depend on timing.
-// Warp 0 then selects.
+// Small batches (T <= 64 tokens, E <= 64 experts: decode): one CTA of 512
+// threads per token.  The token's row of x is staged once in shared memory
+// (fp32).  With EP = E rounded up to a power of two, thread i owns expert
+// i % EP and the 8-element H-vectors v = i / EP + j * (512 / EP) of W_gate,
+// whose loads it issues 16 at a time before any FMA, so a token costs a few
+// memory round trips.  Partials are reduced in a fixed order (lanes of the
+// same expert by a shuffle tree, then warps in order), so the logits do not
+// depend on timing.  Warp 0 then selects.
+constexpr int NS = 512;   // threads per CTA of the small-batch router
+
 template <int EP, bool BF16>
-__global__ void __launch_bounds__(NT) route_small_kernel(const void* __restrict__ xv,
+__global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict__ xv,
                                                          const void* __restrict__ wv,
                                                          const float* __restrict__ bias, int H,
                                                          int E, int k, int renorm,
                                                          float* __restrict__ logits,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ wout) {
-  constexpr int TPE = NT / EP;                 // threads per expert
+  constexpr int TPE = NS / EP;                 // threads per expert
   constexpr int BATCH = 16;
-  __shared__ float part[NT / 32][64];
+  constexpr int Q = BF16 ? 1 : 2;              // 16-byte words per 8 elements
+  extern __shared__ __align__(16) float xs[];  // [H]
+  __shared__ float part[NS / 32][64];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = threadIdx.x % EP;
   const int v0 = threadIdx.x / EP;
   const int nvec = H / 8;
   moe::grid_dep_wait();
+  for (int v = threadIdx.x; v < nvec; v += NS) {
+    float f[8];
+    load8<BF16>(xv, static_cast<size_t>(t) * H + v * 8, true, f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xs[v * 8 + j] = f[j];
+  }
+  __syncthreads();
   float acc = 0.f;
   if (e < E) {
-    // 8 elements = one uint4 (bf16) or two (fp32); loads are unconditional
-    // (clamped to the last vector) so that all of a batch are in flight.
-    constexpr int Q = BF16 ? 1 : 2;
-    const uint4* xb = reinterpret_cast<const uint4*>(xv) + static_cast<size_t>(t) * (nvec * Q);
+    // loads are unconditional (clamped to the last vector) so that all of a
+    // batch are in flight together
     const uint4* wb = reinterpret_cast<const uint4*>(wv) + static_cast<size_t>(e) * (nvec * Q);
     for (int vb = v0; vb < nvec; vb += BATCH * TPE) {
-      uint4 xq[BATCH][Q], wq[BATCH][Q];
+      uint4 wq[BATCH][Q];
 #pragma unroll
       for (int j = 0; j < BATCH; ++j) {
         const int vc = min(vb + j * TPE, nvec - 1);
 #pragma unroll
-        for (int q = 0; q < Q; ++q) {
-          xq[j][q] = __ldg(xb + vc * Q + q);
-          wq[j][q] = __ldg(wb + vc * Q + q);
-        }
+        for (int q = 0; q < Q; ++q) wq[j][q] = moe::ld_nc_v4(wb + vc * Q + q);
       }
 #pragma unroll
       for (int j = 0; j < BATCH; ++j) {
-        if (vb + j * TPE >= nvec) break;
-        float xf[8], wf[8];
+        const int v = vb + j * TPE;
+        if (v >= nvec) break;
+        float wf[8];
         if (BF16) {
-          moe::unpack8(xq[j][0], xf);
           moe::unpack8(wq[j][0], wf);
         } else {
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            xf[4 * q] = __uint_as_float(xq[j][q].x); xf[4 * q + 1] = __uint_as_float(xq[j][q].y);
-            xf[4 * q + 2] = __uint_as_float(xq[j][q].z); xf[4 * q + 3] = __uint_as_float(xq[j][q].w);
             wf[4 * q] = __uint_as_float(wq[j][q].x); wf[4 * q + 1] = __uint_as_float(wq[j][q].y);
             wf[4 * q + 2] = __uint_as_float(wq[j][q].z); wf[4 * q + 3] = __uint_as_float(wq[j][q].w);
           }
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc = fmaf(xf[q], wf[q], acc);
+        const float4 xa = *reinterpret_cast<const float4*>(&xs[v * 8]);
+        const float4 xb = *reinterpret_cast<const float4*>(&xs[v * 8 + 4]);
+        acc = fmaf(xa.x, wf[0], acc); acc = fmaf(xa.y, wf[1], acc);
+        acc = fmaf(xa.z, wf[2], acc); acc = fmaf(xa.w, wf[3], acc);
+        acc = fmaf(xb.x, wf[4], acc); acc = fmaf(xb.y, wf[5], acc);
+        acc = fmaf(xb.z, wf[6], acc); acc = fmaf(xb.w, wf[7], acc);
       }
     }
   }
@@ -203,7 +212,7 @@ __global__ void __launch_bounds__(NT) route_small_kernel(const void* __restrict_
     if (live[j]) {
       // warps holding expert ex: those whose lanes cover ex % EP
 #pragma unroll
-      for (int w = 0; w < NT / 32; ++w)
+      for (int w = 0; w < NS / 32; ++w)
         if (EP <= 32 || (w * 32) % EP == (ex / 32) * 32 % EP) s += part[w][ex];
       s += bias ? bias[ex] : 0.f;
       logits[static_cast<size_t>(t) * E + ex] = s;
@@ -405,14 +414,21 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
                          int E, int k, int renormalize, int dtype, float* logits, int32_t* ids,
                          float* w, cudaStream_t s) {
   const bool bf = dtype == MOE_BF16;
-  if (T <= 64 && E <= 64) {
+  if (T <= 64 && E <= 64 && H <= 32768) {
 #define MOE_SMALL_CASE(EPV)                                                                   \
     if (E <= EPV) {                                                                         \
-      if (bf)                                                                               \
-        return launch_pdl(route_small_kernel<EPV, true>, dim3(T), dim3(NT), 0, s, 0, x,       \
+      if (bf) {                                                                             \
+        cudaError_t e = ensure_smem(                                                        \
+            reinterpret_cast<const void*>(route_small_kernel<EPV, true>), H * 4);           \
+        if (e != cudaSuccess) return e;                                                     \
+        return launch_pdl(route_small_kernel<EPV, true>, dim3(T), dim3(NS), H * 4, s, 0, x,   \
                           W_gate, bias, H, E, k, renormalize, logits, ids, w);              \
-      return launch_pdl(route_small_kernel<EPV, false>, dim3(T), dim3(NT), 0, s, 0, x, W_gate,  \
-                        bias, H, E, k, renormalize, logits, ids, w);                        \
+      }                                                                                     \
+      cudaError_t e = ensure_smem(                                                          \
+          reinterpret_cast<const void*>(route_small_kernel<EPV, false>), H * 4);            \
+      if (e != cudaSuccess) return e;                                                       \
+      return launch_pdl(route_small_kernel<EPV, false>, dim3(T), dim3(NS), H * 4, s, 0, x,    \
+                        W_gate, bias, H, E, k, renormalize, logits, ids, w);                \
     }
     MOE_SMALL_CASE(1)
     MOE_SMALL_CASE(2)
