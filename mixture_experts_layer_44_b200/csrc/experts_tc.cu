@@ -95,7 +95,9 @@ struct Ctl {
   int tstart[moe::kMaxExperts + 1];   // first tile of expert e (tiles = token tiles x NTW)
 };
 
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+constexpr int STAGE_OUT_BYTES = BM * 128;                  // epilogue staging: 128 rows x 128 B
+constexpr size_t CTL_BYTES = (sizeof(Ctl) + 127) / 128 * 128;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTL_BYTES + STAGE_OUT_BYTES;
 
 struct Unit {
   int tile, e, nt, mt, ks, kb0, kb1;
@@ -160,23 +162,65 @@ __device__ __forceinline__ void epi_bar() {   // the 4 epilogue warps only
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
 
-// 16 h values (16 gate and 16 up accumulator columns) -> 16 bf16.
-__device__ __forceinline__ void store_h16(__nv_bfloat16* dst, const float* g, const float* u) {
-  uint32_t pk[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    pk[j] = moe::pack_bf16x2(silu_mul(g[2 * j], u[2 * j]), silu_mul(g[2 * j + 1], u[2 * j + 1]));
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-}
-
-// 16 accumulator columns scaled by sc -> 16 fp32.
-__device__ __forceinline__ void store_y16(float* dst, const float* v, float sc) {
+// Direct per-thread row stores, used when a tile has few valid rows (there
+// the staging barriers cost more than the scattered stores they save).
+__device__ __forceinline__ void store_f32x32(float* dst, const uint32_t* a, const uint32_t* b,
+                                             float sc) {
   float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int j = 0; j < 4; ++j)
-    d4[j] = make_float4(v[4 * j] * sc, v[4 * j + 1] * sc, v[4 * j + 2] * sc, v[4 * j + 3] * sc);
+    d4[j] = make_float4(__uint_as_float(a[4 * j]) * sc, __uint_as_float(a[4 * j + 1]) * sc,
+                        __uint_as_float(a[4 * j + 2]) * sc, __uint_as_float(a[4 * j + 3]) * sc);
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    d4[4 + j] = make_float4(__uint_as_float(b[4 * j]) * sc, __uint_as_float(b[4 * j + 1]) * sc,
+                            __uint_as_float(b[4 * j + 2]) * sc, __uint_as_float(b[4 * j + 3]) * sc);
+}
+
+constexpr int STAGE_MIN_ROWS = 32;   // stage the epilogue only above this many valid rows
+
+// Epilogue staging.  A thread owns one tile row (its TMEM lane); rows are
+// written to global memory through a 128 row x 128 byte shared buffer so that
+// each warp store covers whole 128-byte row segments (4 rows per instruction)
+// instead of 32 scattered 16-byte pieces.  16-byte chunk j of row r sits at
+// position j ^ (r & 7): conflict-free both when 32 lanes each write their own
+// row and when 8 lanes read one row.
+__device__ __forceinline__ void stage_put(uint8_t* stg, int row, int j, uint4 v) {
+  reinterpret_cast<uint4*>(stg + row * 128)[j ^ (row & 7)] = v;
+}
+
+// Write rows [0, nvalid) of the staged 128-byte chunk to gtile + r * ld_bytes;
+// warp quarter wq handles rows 32*wq .. 32*wq + 31.
+__device__ __forceinline__ void stage_flush(const uint8_t* stg, int wq, int lane, int nvalid,
+                                            uint8_t* gtile, size_t ld_bytes) {
+  const int j = lane & 7;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int r = wq * 32 + it * 4 + (lane >> 3);
+    if (r < nvalid) {
+      const uint4 v = reinterpret_cast<const uint4*>(stg + r * 128)[j ^ (r & 7)];
+      *reinterpret_cast<uint4*>(gtile + static_cast<size_t>(r) * ld_bytes + j * 16) = v;
+    }
+  }
+}
+
+// 32 fp32 accumulator columns (two TMEM loads) scaled by sc -> 8 staged chunks.
+__device__ __forceinline__ void stage_f32x32(uint8_t* stg, int row, const uint32_t* a,
+                                             const uint32_t* b, float sc) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    stage_put(stg, row, j,
+              make_uint4(__float_as_uint(__uint_as_float(a[4 * j]) * sc),
+                         __float_as_uint(__uint_as_float(a[4 * j + 1]) * sc),
+                         __float_as_uint(__uint_as_float(a[4 * j + 2]) * sc),
+                         __float_as_uint(__uint_as_float(a[4 * j + 3]) * sc)));
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    stage_put(stg, row, 4 + j,
+              make_uint4(__float_as_uint(__uint_as_float(b[4 * j]) * sc),
+                         __float_as_uint(__uint_as_float(b[4 * j + 1]) * sc),
+                         __float_as_uint(__uint_as_float(b[4 * j + 2]) * sc),
+                         __float_as_uint(__uint_as_float(b[4 * j + 3]) * sc)));
 }
 
 template <int EPI>
@@ -191,6 +235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   Ctl& c = *reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* stg = smem + STAGES * STAGE_BYTES + CTL_BYTES;   // epilogue staging
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int kblocks = K / BK;
@@ -411,32 +456,84 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const size_t grow = static_cast<size_t>(c.offs[un.e] + un.mt * BM + row);
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN);
+      const int nvalid = rows_valid < BM ? rows_valid : BM;
+      const bool staged = nvalid > STAGE_MIN_ROWS;    // same for all four epilogue warps
+      const size_t row0 = static_cast<size_t>(c.offs[un.e] + un.mt * BM);
       if (S == 1) {
-        if (EPI == EPI_SWIGLU) {
-          __nv_bfloat16* dst =
-              static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
+        if (EPI == EPI_SWIGLU && !staged) {
+          // few valid rows: 16 h columns per step, each thread stores its own row
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
 #pragma unroll 1
           for (int cc = 0; cc < BN / 2; cc += 16) {
             uint32_t g[16], v[16];
             moe::tmem_ld16(taddr + cc, g);
             moe::tmem_ld16(taddr + BN / 2 + cc, v);
             moe::tmem_ld_wait();
-            if (live)
-              store_h16(dst + cc, reinterpret_cast<const float*>(g),
-                        reinterpret_cast<const float*>(v));
+            if (live) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                pk[j] = moe::pack_bf16x2(
+                    silu_mul(__uint_as_float(g[2 * j]), __uint_as_float(v[2 * j])),
+                    silu_mul(__uint_as_float(g[2 * j + 1]), __uint_as_float(v[2 * j + 1])));
+              uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
+              d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        } else if (EPI == EPI_SWIGLU) {
+          // 64 h columns per staged chunk: gate cols hc.., up cols 128+hc..
+          uint8_t* gtile = static_cast<uint8_t*>(out) +
+                           (row0 * ldo + un.nt * (BN / 2)) * sizeof(__nv_bfloat16);
+#pragma unroll 1
+          for (int hc = 0; hc < BN / 2; hc += 64) {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              const int cc = hc + half * 32;
+              uint32_t g0[16], g1[16], v0[16], v1[16];
+              moe::tmem_ld16(taddr + cc, g0);
+              moe::tmem_ld16(taddr + cc + 16, g1);
+              moe::tmem_ld16(taddr + BN / 2 + cc, v0);
+              moe::tmem_ld16(taddr + BN / 2 + cc + 16, v1);
+              moe::tmem_ld_wait();
+              uint32_t pk[16];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                pk[j] = moe::pack_bf16x2(
+                    silu_mul(__uint_as_float(g0[2 * j]), __uint_as_float(v0[2 * j])),
+                    silu_mul(__uint_as_float(g0[2 * j + 1]), __uint_as_float(v0[2 * j + 1])));
+                pk[8 + j] = moe::pack_bf16x2(
+                    silu_mul(__uint_as_float(g1[2 * j]), __uint_as_float(v1[2 * j])),
+                    silu_mul(__uint_as_float(g1[2 * j + 1]), __uint_as_float(v1[2 * j + 1])));
+              }
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                stage_put(stg, row, half * 4 + j,
+                          make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]));
+            }
+            epi_bar();
+            stage_flush(stg, q, lane, nvalid, gtile + hc * sizeof(__nv_bfloat16),
+                        static_cast<size_t>(ldo) * sizeof(__nv_bfloat16));
+            epi_bar();
           }
         } else {
           const float sc = live ? (packed_w ? packed_w[grow] : 1.f) : 0.f;
-          float* dst = static_cast<float*>(out) + grow * ldo + un.nt * BN;
+          uint8_t* gtile = static_cast<uint8_t*>(out) + (row0 * ldo + un.nt * BN) * sizeof(float);
 #pragma unroll 1
           for (int cc = 0; cc < BN; cc += 32) {
             uint32_t a[16], b[16];
             moe::tmem_ld16(taddr + cc, a);
             moe::tmem_ld16(taddr + cc + 16, b);
             moe::tmem_ld_wait();
-            if (live) {
-              store_y16(dst + cc, reinterpret_cast<const float*>(a), sc);
-              store_y16(dst + cc + 16, reinterpret_cast<const float*>(b), sc);
+            if (staged) {
+              stage_f32x32(stg, row, a, b, sc);
+              epi_bar();
+              stage_flush(stg, q, lane, nvalid, gtile + cc * sizeof(float),
+                          static_cast<size_t>(ldo) * sizeof(float));
+              epi_bar();
+            } else if (live) {
+              store_f32x32(reinterpret_cast<float*>(gtile) + static_cast<size_t>(row) * ldo + cc,
+                           a, b, sc);
             }
           }
         }
@@ -445,16 +542,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
       } else {
         // Partial of one K-slice: valid rows to this unit's workspace slot.
-        float* slot = partials + static_cast<size_t>(u) * (BM * BN) + static_cast<size_t>(row) * BN;
+        uint8_t* gtile = reinterpret_cast<uint8_t*>(partials + static_cast<size_t>(u) * (BM * BN));
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 32) {
           uint32_t a[16], b[16];
           moe::tmem_ld16(taddr + cc, a);
           moe::tmem_ld16(taddr + cc + 16, b);
           moe::tmem_ld_wait();
-          if (live) {
-            store_y16(slot + cc, reinterpret_cast<const float*>(a), 1.f);
-            store_y16(slot + cc + 16, reinterpret_cast<const float*>(b), 1.f);
+          if (staged) {
+            stage_f32x32(stg, row, a, b, 1.f);
+            epi_bar();
+            stage_flush(stg, q, lane, nvalid, gtile + cc * sizeof(float), BN * sizeof(float));
+            epi_bar();
+          } else if (live) {
+            store_f32x32(reinterpret_cast<float*>(gtile) + static_cast<size_t>(row) * BN + cc, a,
+                         b, 1.f);
           }
         }
         moe::tc_fence_before();
@@ -477,8 +579,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // across slices so they are in flight together).
           __threadfence();
           const int et = threadIdx.x - 64;                // 0..127
-          const int nrows = min(rows_valid, BM);
-          const size_t row0 = static_cast<size_t>(c.offs[un.e] + un.mt * BM);
+          const int nrows = nvalid;
           const float* base = partials + static_cast<size_t>(un.tile) * S * (BM * BN);
           if (EPI == EPI_SWIGLU) {
             const int cg = et & 31;                       // h columns 4cg .. 4cg+3

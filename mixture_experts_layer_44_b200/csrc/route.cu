@@ -364,11 +364,22 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
       live[j] = lane + 32 * j < E;
       v[j] = 0.f;
     }
-    for (int r = 0; r < S; ++r) {               // fixed order: deterministic sum
-      const float* rl = cluster.map_shared_rank(l_s, r);
+    {
+      // all ranks' partials in flight together, then summed in rank order
+      float pv[MAX_S][PER];
 #pragma unroll
-      for (int j = 0; j < PER; ++j)
-        if (live[j]) v[j] += rl[tl * LS + lane + 32 * j];
+      for (int r = 0; r < MAX_S; ++r) {
+        if (r < S) {
+          const float* rl = cluster.map_shared_rank(l_s, r);
+#pragma unroll
+          for (int j = 0; j < PER; ++j) pv[r][j] = live[j] ? rl[tl * LS + lane + 32 * j] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < MAX_S; ++r)
+        if (r < S)
+#pragma unroll
+          for (int j = 0; j < PER; ++j) v[j] += pv[r][j];
     }
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
