@@ -283,7 +283,7 @@ def run_gpu(args, cfg):
         if ev:
             ev[0].record(stream)
         M.moe_route(x, dp["W_gate"], dp["bias"], cfg.k, cfg.renormalize, buf.logits, buf.ids,
-                    buf.w, stream=stream)
+                    buf.w, status=buf.status, stream=stream)
         if ev:
             ev[1].record(stream)
         M.moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
@@ -294,7 +294,8 @@ def run_gpu(args, cfg):
         M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
                       buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
         if shared:
-            M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
+            M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
+                        status=buf.status, stream=stream)
             M.moe_experts(x, buf.sh_offsets, None, dp["w13s"].unsqueeze(0),
                           dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
                           status=buf.status, stream=stream)

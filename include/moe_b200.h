@@ -70,7 +70,7 @@ const char* moe_last_error(void);
  * diffulex.moe API reference, "diffulex.moe.topk" (NaiveTopKRouter, the
  * standard top-k router).
  *
- *   logits[t,e] = sum_h x[t,h] * W_gate[e,h] + bias[e]      (fp32 FMA)
+ *   logits[t,e] = sum_h x[t,h] * W_gate[e,h] + bias[e]      (fp32 sums)
  *   p[t,:]      = softmax(logits[t,:]) over all E             (fp32)
  *   topk_ids[t,j], j < k: the k experts with the largest logits, in
  *               descending order; equal logits -> lower expert id first
@@ -82,12 +82,21 @@ const char* moe_last_error(void);
  *   logits   device [T,E] fp32, written
  *   topk_ids device [T,k] int32, written (may be NULL when k == 0)
  *   topk_w   device [T,k] fp32, written  (may be NULL when k == 0)
+ *   status   device int32, or NULL: the first device-side error
+ *            (MOE_ERR_TIMEOUT) is recorded there with atomicCAS from 0
  *   k == 0 computes the logits only (e.g. a shared expert's scalar gate
  *   logit with E == 1).  Inputs are assumed finite.
+ *
+ *   fp32: the sums are fp32 FMA chains on the CUDA cores.  bf16 with more
+ *   than 64 tokens or more than 64 experts: the contraction runs on the
+ *   tensor cores (bf16 products are exact in fp32; fp32 accumulation in
+ *   TMEM); smaller bf16 batches use fp32 FMA.  Results are deterministic
+ *   for a given device and shape.
  */
 int moe_route(const void* x, const void* W_gate, const float* bias,
               int T, int H, int E, int k, int renormalize, int dtype,
-              float* logits, int32_t* topk_ids, float* topk_w, void* stream);
+              float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+              void* stream);
 
 /* Bytes of device scratch moe_dispatch needs for (T, k, E). */
 size_t moe_dispatch_workspace_bytes(int T, int k, int E);

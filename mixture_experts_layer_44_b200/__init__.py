@@ -53,7 +53,7 @@ _SZ = ctypes.c_size_t
 _SIGS = {
     "moe_abi_version": (_I, []),
     "moe_last_error": (ctypes.c_char_p, []),
-    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_dispatch_workspace_bytes": (_SZ, [_I, _I, _I]),
     "moe_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_dispatch_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -118,12 +118,13 @@ def moe_last_error() -> str:
 
 
 def moe_route(x, W_gate, bias, k: int, renormalize: bool, logits, topk_ids=None, topk_w=None,
-              stream=None):
+              status=None, stream=None):
     T, H = x.shape
     E = W_gate.shape[0]
     _check(load_library().moe_route(_ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k,
                                     int(bool(renormalize)), _dtype_code(x), _ptr(logits),
-                                    _ptr(topk_ids), _ptr(topk_w), _stream(stream)))
+                                    _ptr(topk_ids), _ptr(topk_w), _ptr(status),
+                                    _stream(stream)))
 
 
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
@@ -240,14 +241,15 @@ def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerB
     """
     E = params["W_gate"].shape[0]
     moe_route(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits, buf.ids,
-              buf.w, stream=stream)
+              buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
     moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
                 buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
     shared = sg = None
     if params.get("w13s") is not None:
-        moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit, stream=stream)
+        moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
+                  status=buf.status, stream=stream)
         moe_experts(x, buf.sh_offsets, None, params["w13s"].unsqueeze(0),
                     params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
                     status=buf.status, stream=stream)

@@ -78,13 +78,13 @@ cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream
 
 extern "C" {
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 const char* moe_last_error(void) { return g_err.c_str(); }
 
 int moe_route(const void* x, const void* W_gate, const float* bias, int T, int H, int E, int k,
               int renormalize, int dtype, float* logits, int32_t* topk_ids, float* topk_w,
-              void* stream) {
+              int32_t* status, void* stream) {
   g_err.clear();
   if (int r = check_dtype(dtype)) return r;
   REQ(x && W_gate && logits, MOE_ERR_INVALID_ARG, "moe_route: null x, W_gate or logits");
@@ -96,12 +96,13 @@ int moe_route(const void* x, const void* W_gate, const float* bias, int T, int H
   REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_route: H must be a multiple of 8");
   REQ(aligned16(x) && aligned16(W_gate), MOE_ERR_INVALID_ARG,
       "moe_route: x and W_gate must be 16-byte aligned");
-  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias),
-      MOE_ERR_INVALID_ARG, "moe_route: outputs and bias must be 4-byte aligned");
+  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias) &&
+          aligned4(status),
+      MOE_ERR_INVALID_ARG, "moe_route: outputs, bias and status must be 4-byte aligned");
   REQ(static_cast<long long>(T) * (H > E ? H : E) < (1ll << 31), MOE_ERR_INVALID_ARG,
       "moe_route: T*H too large");
   cudaError_t e = moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
-                                         logits, topk_ids, topk_w,
+                                         logits, topk_ids, topk_w, status,
                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
 }

@@ -81,7 +81,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 namespace moe_host {
 cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, int T, int H,
                          int E, int k, int renormalize, int dtype, float* logits,
-                         int32_t* ids, float* w, cudaStream_t s);
+                         int32_t* ids, float* w, int32_t* status, cudaStream_t s);
+cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
+                            int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
+                            int32_t* status, cudaStream_t s);
 size_t dispatch_ws_bytes(int T, int k, int E);
 cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, int T, int H,
                             int E, int k, int dtype, int32_t* counts, int32_t* offsets,

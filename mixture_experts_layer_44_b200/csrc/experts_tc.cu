@@ -48,14 +48,12 @@
 // a wait that runs out reports MOE_ERR_TIMEOUT, the CTA drains what it issued
 // and frees its TMEM.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <cstring>
-#include <mutex>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
+#include "tmap.cuh"
 
 namespace {
 
@@ -640,80 +638,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// ------------------------------------------------------ tensor maps ---
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-bool encode_uncached(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                     const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-  auto fn = get_encode();
-  if (!fn) return false;
-  cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
-                  strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// Small cache of encoded tensor maps: a layer called again on the same
-// buffers reuses its descriptors instead of encoding four per call.  The map
-// depends only on the key (device, base, rank, dims, strides, box).
-struct MapKey {
-  int dev, rank;
-  const void* base;
-  cuuint64_t dims[3], strides[2];
-  cuuint32_t box[3];
-};
-
-bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
-  constexpr int kSlots = 64;
-  static std::mutex mu;
-  static MapKey keys[kSlots];
-  static CUtensorMap maps[kSlots];
-  static int used = 0, next = 0;
-  MapKey k;
-  std::memset(&k, 0, sizeof(k));
-  cudaGetDevice(&k.dev);
-  k.rank = rank;
-  k.base = base;
-  for (int i = 0; i < rank; ++i) {
-    k.dims[i] = dims[i];
-    k.box[i] = box[i];
-    if (i + 1 < rank) k.strides[i] = strides_bytes[i];
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < used; ++i)
-    if (std::memcmp(&keys[i], &k, sizeof(k)) == 0) {
-      *m = maps[i];
-      return true;
-    }
-  if (!encode_uncached(m, base, rank, dims, strides_bytes, box)) return false;
-  const int slot = used < kSlots ? used++ : (next++ % kSlots);
-  keys[slot] = k;
-  maps[slot] = *m;
-  return true;
-}
-
 // Activations [rows, K] bf16, box 64 x 128.
 bool map_rows(CUtensorMap* m, const void* p, int rows, int K) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
   const cuuint32_t box[2] = {BK, BM};
-  return encode(m, p, 2, dims, str, box);
+  return moe_host::encode_bf16_sw128(m, p, 2, dims, str, box);
 }
 
 }  // namespace
@@ -743,14 +673,14 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     const cuuint64_t str[2] = {static_cast<cuuint64_t>(H) * 2,
                                static_cast<cuuint64_t>(I) * H * 2};
     const cuuint32_t box[3] = {BK, BN / 2, 2};
-    ok = ok && encode(&mB1, w13, 3, dims, str, box);
+    ok = ok && encode_bf16_sw128(&mB1, w13, 3, dims, str, box);
   }
   {
     // w2 as [E*H][I]
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(E) * H};
     const cuuint64_t str[1] = {static_cast<cuuint64_t>(I) * 2};
     const cuuint32_t box[2] = {BK, BN};
-    ok = ok && encode(&mB2, w2, 2, dims, str, box);
+    ok = ok && encode_bf16_sw128(&mB2, w2, 2, dims, str, box);
   }
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";

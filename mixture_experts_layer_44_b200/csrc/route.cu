@@ -1,30 +1,33 @@
-// Router: gating GEMM on the CUDA cores (fp32 FMA), fused with softmax,
-// warp-shuffle top-k and renormalisation.
+// Router on the CUDA cores (fp32 FMA), fused with softmax, warp-shuffle top-k
+// and renormalisation: every fp32 batch, and bf16 batches of at most 64
+// tokens and 64 experts (larger bf16 batches run on the tensor cores).
 //
 // DWDP-Triton-MoE-Inference-Engine README, "Router Module": router logits,
 // routing probabilities, top-k expert indices, normalized routing weights.
 // diffulex.moe API reference, "diffulex.moe.topk": NaiveTopKRouter.
 //
-// Batches of more than 64 tokens (or more than 64 experts): a thread-block
-// cluster of S CTAs (S <= 8) owns BT = 16*TT tokens and all E experts; CTA s
-// of the cluster contracts its own slice of H.  Each CTA stages chunks of
-// KC = 32 columns of x and W_gate (converted to fp32, transposed, without
-// bank conflicts) in double-buffered shared memory, prefetching the next
-// chunk into registers while it computes the current one, and accumulates a
+// fp32 batches of more than 64 tokens (or more than 64 experts): a
+// thread-block cluster of S CTAs (S <= 8) owns BT = 16*TT tokens and all E
+// experts; CTA s of the cluster contracts its own slice of H.  Each CTA
+// stages chunks of KC = 32 columns of x and W_gate (transposed, without bank
+// conflicts) in double-buffered shared memory, prefetching the next chunk
+// into registers while it computes the current one, and accumulates a
 // TT-token x (EPAD/16)-expert register tile per thread (EPAD = 64, 128 or
 // 256: E rounded up; TT = 8 for EPAD = 64, else 4).  Thread eg owns experts
 // 64*(j/4) + 4*eg + (j%4): each of its float4 reads of W is part of 256
-// contiguous bytes across the warp, free of bank conflicts.  The S partial logit tiles are then summed through distributed shared
-// memory in a fixed rank order (deterministic, no global scratch): CTA s
-// finalises tokens [s*BT/S, (s+1)*BT/S) of the tile, one warp per token, which
-// adds the bias, writes the logits and selects the top k by k rounds of a warp
-// arg-max on the key (logit descending, expert id ascending).
+// contiguous bytes across the warp, free of bank conflicts.  The S partial
+// logit tiles are then summed through distributed shared memory in a fixed
+// rank order (deterministic, no global scratch): CTA s finalises tokens
+// [s*BT/S, (s+1)*BT/S) of the tile, one warp per token, which adds the bias,
+// writes the logits and selects the top k by k rounds of a warp arg-max on
+// the key (logit descending, expert id ascending).
 #include <cooperative_groups.h>
 #include <float.h>
 
 #include <algorithm>
 
 #include "common.cuh"
+#include "select.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -33,10 +36,6 @@ namespace {
 constexpr int KC = 32;    // H chunk
 constexpr int NT = 256;   // threads per CTA
 constexpr int MAX_S = 8;  // CTAs per cluster
-
-__device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
-  return v1 > v2 || (v1 == v2 && i1 < i2);
-}
 
 template <bool BF16>
 __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, float* f) {
@@ -56,71 +55,6 @@ __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, flo
   }
 }
 
-
-// Softmax over the E live logits of one token held by a warp (lane l holds
-// experts l, l+32, ...), then k rounds of a warp arg-max on (logit desc, id
-// asc) over the experts not yet taken; lane r < k writes selection r.
-template <int PER>
-__device__ __forceinline__ void select_topk(const float* v, const bool* live, int k, int renorm,
-                                            int32_t* ids_t, float* w_t) {
-  const int lane = threadIdx.x & 31;
-  float m = -FLT_MAX;
-#pragma unroll
-  for (int j = 0; j < PER; ++j)
-    if (live[j]) m = fmaxf(m, v[j]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float s = 0.f;
-#pragma unroll
-  for (int j = 0; j < PER; ++j)
-    if (live[j]) s += expf(v[j] - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-
-  bool taken[PER];
-#pragma unroll
-  for (int j = 0; j < PER; ++j) taken[j] = !live[j];
-  float ssel = 0.f;
-  float my_v = 0.f;                           // lane r < k keeps selection r
-  int my_id = 0;
-#pragma unroll
-  for (int r = 0; r < moe::kMaxTopK; ++r) {
-    if (r >= k) break;
-    float bv = -FLT_MAX;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-      const int e = lane + 32 * j;
-      if (!taken[j] && (bi == 0x7fffffff || better(v[j], e, bv, bi))) {
-        bv = v[j];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < PER; ++j)
-      if (lane + 32 * j == bi) taken[j] = true;
-    const float ex = expf(bv - m);
-    ssel += ex;
-    if (lane == r) {
-      my_v = ex;
-      my_id = bi;
-    }
-  }
-  if (lane < k) {
-    const float denom = renorm ? ssel : s;
-    ids_t[lane] = my_id;
-    w_t[lane] = my_v / denom;
-  }
-}
 
 // Small batches (T <= 64 tokens, E <= 64 experts: decode): one CTA of 512
 // threads per token.  The token's row of x is staged once in shared memory
@@ -220,7 +154,7 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
     v[j] = live[j] ? s : -FLT_MAX;
   }
   if (k == 0) return;
-  select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
+  moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
                    wout + static_cast<size_t>(t) * k);
 }
 
@@ -392,7 +326,7 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
       }
     }
     if (k == 0) continue;
-    select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
+    moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
                      wout + static_cast<size_t>(t) * k);
   }
   cluster.sync();   // no CTA leaves while another still reads its partial tile
@@ -423,7 +357,7 @@ namespace moe_host {
 
 cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, int T, int H,
                          int E, int k, int renormalize, int dtype, float* logits, int32_t* ids,
-                         float* w, cudaStream_t s) {
+                         float* w, int32_t* status, cudaStream_t s) {
   const bool bf = dtype == MOE_BF16;
   if (T <= 64 && E <= 64 && H <= 32768) {
 #define MOE_SMALL_CASE(EPV)                                                                   \
@@ -450,15 +384,10 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
     MOE_SMALL_CASE(64)
 #undef MOE_SMALL_CASE
   }
-#define MOE_ROUTE_CASE(EP)                                                                  \
-  if (E <= EP)                                                                              \
-    return bf ? launch_t<EP, true>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, \
-                                   s)                                                       \
-              : launch_t<EP, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
-  MOE_ROUTE_CASE(64)
-  MOE_ROUTE_CASE(128)
-  MOE_ROUTE_CASE(256)
-#undef MOE_ROUTE_CASE
+  if (bf) return launch_route_tc(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
+  if (E <= 64) return launch_t<64, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
+  if (E <= 128) return launch_t<128, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
+  if (E <= 256) return launch_t<256, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
   return cudaErrorInvalidValue;
 }
 

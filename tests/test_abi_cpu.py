@@ -52,7 +52,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_workspace_queries(lib):
-    assert M.moe_abi_version() == 1
+    assert M.moe_abi_version() == 2
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
     assert M.moe_dispatch_workspace_bytes(0, 2, 8) == 0
@@ -69,19 +69,19 @@ def _err(lib):
 
 
 def test_route_rejects_bad_arguments_on_the_host(lib):
-    r = lib.moe_route(P, P, NULL, 0, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    r = lib.moe_route(P, P, NULL, 0, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "T and H" in _err(lib)
-    r = lib.moe_route(P, P, NULL, 4, 64, 8, 9, 1, M.MOE_BF16, P, P, P, NULL)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 9, 1, M.MOE_BF16, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "k must be" in _err(lib)
-    r = lib.moe_route(P, P, NULL, 4, 64, 300, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    r = lib.moe_route(P, P, NULL, 4, 64, 300, 2, 1, M.MOE_BF16, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "E must be" in _err(lib)
-    r = lib.moe_route(P, P, NULL, 4, 60, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    r = lib.moe_route(P, P, NULL, 4, 60, 8, 2, 1, M.MOE_BF16, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "multiple of 8" in _err(lib)
-    r = lib.moe_route(ctypes.c_void_p(24), P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL)
+    r = lib.moe_route(ctypes.c_void_p(24), P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "aligned" in _err(lib)
-    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, 7, P, P, P, NULL)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, 7, P, P, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG and "dtype" in _err(lib)
-    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, NULL, P, NULL)
+    r = lib.moe_route(P, P, NULL, 4, 64, 8, 2, 1, M.MOE_BF16, P, NULL, P, NULL, NULL)
     assert r == M.MOE_ERR_INVALID_ARG
 
 

@@ -105,3 +105,49 @@ def test_route_k_equals_E_is_the_full_softmax():
     full = torch.zeros(20, 8)
     full.scatter_(1, ids.long(), w)
     np.testing.assert_allclose(full.numpy(), O.softmax_rows(O.to_f64(logits)), rtol=1e-5)
+
+
+@pytest.mark.parametrize("T,H,E,k", [
+    (4096, 4096, 64, 2),     # 32 token tiles x clusters of 4 H-slices
+    (1024, 4096, 64, 2),     # 8 tiles x clusters of 8
+    (300, 256, 128, 8),      # ragged last tile, 4 H-blocks of 64, two accumulator chains
+    (129, 2048, 256, 8),     # 256 experts: one accumulator chain, 2 tiles
+    (65, 64, 1, 1),          # a single H-block and a single expert
+    (200, 8, 33, 3),         # H shorter than one 64-column block
+    (8192, 2048, 60, 4),     # Qwen1.5-MoE-A2.7B prefill routing
+])
+def test_route_tensor_core_shapes(T, H, E, k):
+    # bf16 batches above 64 tokens take the tensor-core router
+    cfg = LayerConfig("r", T=T, H=H, E=E, k=k, I=8, dtype="bf16", renormalize=True)
+    p = make_layer(cfg, seed=T + E)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    logits = torch.empty(T, E, device=DEV)
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, device=DEV)
+    M.moe_route(dev(p["x"]), dev(p["W_gate"]), None, k, True, logits, ids, w, status=status)
+    logits2 = torch.empty_like(logits)
+    M.moe_route(dev(p["x"]), dev(p["W_gate"]), None, k, True, logits2, ids, w, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(logits, logits2)              # deterministic
+    l64 = O.router_logits(p["x"], p["W_gate"], None)
+    assert rel(logits.cpu(), l64) <= 1e-5
+    ids_o, w_o = O.route_from_logits(logits.cpu(), k, True)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ids_o)
+    np.testing.assert_allclose(w.cpu().numpy(), w_o, rtol=1e-5, atol=0)
+
+
+def test_route_ties_on_the_tensor_core_path():
+    g = torch.Generator().manual_seed(8)
+    x = torch.randn(200, 256, generator=g).to(torch.bfloat16)
+    W = (torch.randn(100, 256, generator=g) / 16).to(torch.bfloat16)
+    W[70] = W[3]
+    W[99] = W[3]
+    logits, ids, _ = _run(x, W, None, 5, True)
+    assert torch.equal(logits[:, 70], logits[:, 3]) and torch.equal(logits[:, 99], logits[:, 3])
+    ids_o, _ = O.route_from_logits(logits, 5, True)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    logits, ids, w = _run(torch.zeros(130, 64, dtype=torch.bfloat16),
+                          torch.randn(80, 64, generator=g).to(torch.bfloat16), None, 4, True)
+    assert ids.tolist() == [[0, 1, 2, 3]] * 130
+    np.testing.assert_allclose(w.numpy(), 0.25, rtol=1e-6)
