@@ -57,13 +57,14 @@ __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, flo
 
 
 // Small batches (T <= 64 tokens, E <= 64 experts: decode): one CTA of 512
-// threads per token.  The token's row of x is staged once in shared memory
-// (fp32).  With EP = E rounded up to a power of two, thread i owns expert
-// i % EP and the 8-element H-vectors v = i / EP + j * (512 / EP) of W_gate,
-// whose loads it issues 16 at a time before any FMA, so a token costs a few
-// memory round trips.  Partials are reduced in a fixed order (lanes of the
-// same expert by a shuffle tree, then warps in order), so the logits do not
-// depend on timing.  Warp 0 then selects.
+// threads (16 warps) per token.  The token's row of x is staged once in
+// shared memory (fp32).  With EP = E rounded up to a power of two, each warp
+// owns EPW = max(1, EP/16) experts and one of WPE = 16/min(EP,16) slices of
+// H; lane l reads the 8-element vectors l, l+32, ... of the slice, so a
+// warp's loads of a W_gate row are contiguous (512 bytes per instruction for
+// bf16), with up to 16 loads in flight per lane.  Per (expert, slice) the
+// lanes' partials are summed by a shuffle tree and warp 0 adds the slices in
+// order, so the logits do not depend on timing.  Warp 0 then selects.
 constexpr int NS = 512;   // threads per CTA of the small-batch router
 
 template <int EP, bool BF16>
@@ -74,15 +75,16 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
                                                          float* __restrict__ logits,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ wout) {
-  constexpr int TPE = NS / EP;                 // threads per expert
-  constexpr int BATCH = 16;
-  constexpr int Q = BF16 ? 1 : 2;              // 16-byte words per 8 elements
-  extern __shared__ __align__(16) float xs[];  // [H]
-  __shared__ float part[NS / 32][64];
+  constexpr int NWARP = NS / 32;
+  constexpr int EPW = EP > NWARP ? EP / NWARP : 1;       // experts per warp
+  constexpr int WPE = EP >= NWARP ? 1 : NWARP / EP;      // warps (H slices) per expert
+  constexpr int GROUPS = NWARP / WPE;                     // expert e = group + GROUPS * i
+  constexpr int Q = BF16 ? 1 : 2;                         // 16-byte words per 8 elements
+  constexpr int BATCH = 16 / (EPW * Q);                   // vectors per expert in flight
+  extern __shared__ __align__(16) float xs[];             // [H]
+  __shared__ float part[EP][WPE];
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = threadIdx.x % EP;
-  const int v0 = threadIdx.x / EP;
   const int nvec = H / 8;
   moe::grid_dep_wait();
   for (int v = threadIdx.x; v < nvec; v += NS) {
@@ -92,46 +94,65 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
     for (int j = 0; j < 8; ++j) xs[v * 8 + j] = f[j];
   }
   __syncthreads();
-  float acc = 0.f;
-  if (e < E) {
-    // loads are unconditional (clamped to the last vector) so that all of a
-    // batch are in flight together
-    const uint4* wb = reinterpret_cast<const uint4*>(wv) + static_cast<size_t>(e) * (nvec * Q);
-    for (int vb = v0; vb < nvec; vb += BATCH * TPE) {
-      uint4 wq[BATCH][Q];
+  const int slice = warp % WPE;
+  const int group = warp / WPE;
+  const int vs = slice * nvec / WPE, ve = (slice + 1) * nvec / WPE;
+  const uint4* wb = reinterpret_cast<const uint4*>(wv);
+  float acc[EPW];
+#pragma unroll
+  for (int i = 0; i < EPW; ++i) acc[i] = 0.f;
+  for (int vb = vs + lane; vb < ve; vb += 32 * BATCH) {
+    // loads are unconditional (clamped to the slice's last vector) so that a
+    // whole batch is in flight before the first FMA
+    uint4 wq[EPW][BATCH][Q];
+#pragma unroll
+    for (int i = 0; i < EPW; ++i) {
+      const int e = min(group + GROUPS * i, E - 1);
 #pragma unroll
       for (int j = 0; j < BATCH; ++j) {
-        const int vc = min(vb + j * TPE, nvec - 1);
+        const int vc = min(vb + 32 * j, ve - 1);
 #pragma unroll
-        for (int q = 0; q < Q; ++q) wq[j][q] = moe::ld_nc_v4(wb + vc * Q + q);
+        for (int q = 0; q < Q; ++q)
+          wq[i][j][q] = moe::ld_nc_v4(wb + (static_cast<size_t>(e) * nvec + vc) * Q + q);
       }
+    }
 #pragma unroll
-      for (int j = 0; j < BATCH; ++j) {
-        const int v = vb + j * TPE;
-        if (v >= nvec) break;
+    for (int j = 0; j < BATCH; ++j) {
+      const int v = vb + 32 * j;
+      if (v >= ve) break;
+      const float4 xa = *reinterpret_cast<const float4*>(&xs[v * 8]);
+      const float4 xb = *reinterpret_cast<const float4*>(&xs[v * 8 + 4]);
+#pragma unroll
+      for (int i = 0; i < EPW; ++i) {
         float wf[8];
         if (BF16) {
-          moe::unpack8(wq[j][0], wf);
+          moe::unpack8(wq[i][j][0], wf);
         } else {
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            wf[4 * q] = __uint_as_float(wq[j][q].x); wf[4 * q + 1] = __uint_as_float(wq[j][q].y);
-            wf[4 * q + 2] = __uint_as_float(wq[j][q].z); wf[4 * q + 3] = __uint_as_float(wq[j][q].w);
+            wf[4 * q] = __uint_as_float(wq[i][j][q].x);
+            wf[4 * q + 1] = __uint_as_float(wq[i][j][q].y);
+            wf[4 * q + 2] = __uint_as_float(wq[i][j][q].z);
+            wf[4 * q + 3] = __uint_as_float(wq[i][j][q].w);
           }
         }
-        const float4 xa = *reinterpret_cast<const float4*>(&xs[v * 8]);
-        const float4 xb = *reinterpret_cast<const float4*>(&xs[v * 8 + 4]);
-        acc = fmaf(xa.x, wf[0], acc); acc = fmaf(xa.y, wf[1], acc);
-        acc = fmaf(xa.z, wf[2], acc); acc = fmaf(xa.w, wf[3], acc);
-        acc = fmaf(xb.x, wf[4], acc); acc = fmaf(xb.y, wf[5], acc);
-        acc = fmaf(xb.z, wf[6], acc); acc = fmaf(xb.w, wf[7], acc);
+        float a = acc[i];
+        a = fmaf(xa.x, wf[0], a); a = fmaf(xa.y, wf[1], a);
+        a = fmaf(xa.z, wf[2], a); a = fmaf(xa.w, wf[3], a);
+        a = fmaf(xb.x, wf[4], a); a = fmaf(xb.y, wf[5], a);
+        a = fmaf(xb.z, wf[6], a); a = fmaf(xb.w, wf[7], a);
+        acc[i] = a;
       }
     }
   }
-  // lanes holding the same expert: lane, lane + EP, ... inside a warp
 #pragma unroll
-  for (int o = 16; o >= EP && o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane < (EP < 32 ? EP : 32)) part[warp][e] = acc;
+  for (int i = 0; i < EPW; ++i) {
+    float a = acc[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    const int e = group + GROUPS * i;
+    if (lane == 0 && e < EP) part[e][slice] = a;
+  }
   __syncthreads();
   moe::grid_dep_launch();
   if (warp != 0) return;
@@ -144,10 +165,8 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
     live[j] = ex < E;
     float s = 0.f;
     if (live[j]) {
-      // warps holding expert ex: those whose lanes cover ex % EP
 #pragma unroll
-      for (int w = 0; w < NS / 32; ++w)
-        if (EP <= 32 || (w * 32) % EP == (ex / 32) * 32 % EP) s += part[w][ex];
+      for (int sl = 0; sl < WPE; ++sl) s += part[ex][sl];
       s += bias ? bias[ex] : 0.f;
       logits[static_cast<size_t>(t) * E + ex] = s;
     }
@@ -155,7 +174,7 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
   }
   if (k == 0) return;
   moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
-                   wout + static_cast<size_t>(t) * k);
+                        wout + static_cast<size_t>(t) * k);
 }
 
 // Token rows per thread: 8 when E <= 64 (more FMAs per shared-memory read),
