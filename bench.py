@@ -59,17 +59,19 @@ def load_peaks():
 def expert_stage_work(cfg, counts):
     """Algorithmic bytes and flops of the grouped-GEMM stage (both passes) for
     the realised per-expert counts: weights of every expert with >= 1 row,
-    x_packed read, h written and read back, y_packed written, routing weights."""
+    x_packed read, h written and read back, y_packed written (fp32), routing
+    weights; with a shared expert also its weights, x read, its h written and
+    read back and its fp32 output written."""
     es = 2 if cfg.dtype == "bf16" else 4
     active = sum(1 for c in counts if c > 0)
     N = int(sum(counts))
     H, I = cfg.H, cfg.I
     wbytes = active * 3 * H * I * es
-    abytes = N * H * es + 2 * N * I * es + N * H * es + N * 4
+    abytes = N * H * es + 2 * N * I * es + N * H * 4 + N * 4
     flops = 2 * N * 3 * H * I
     if cfg.shared_I:
         wbytes += 3 * H * cfg.shared_I * es
-        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * es
+        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * 4
         flops += 2 * cfg.T * 3 * H * cfg.shared_I
     return wbytes + abytes, flops
 
@@ -276,8 +278,6 @@ def run_gpu(args, cfg):
     x = dp["x"]
     E = cfg.E
     shared = cfg.shared_I is not None
-    launches_per_step = M.KERNELS_PER_LAYER + (3 if shared else 0)
-
     def step(ev=None):
         # Each stage's events are recorded on the stream its kernels run on.
         if ev:
@@ -335,6 +335,7 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.3)
+    launches0 = M.moe_launch_count()
     for g0 in range(0, args.steps, GROUP):
         torch.cuda._sleep(int(20e6))            # ~10 ms of GPU spin while the host enqueues
         for i in range(g0, min(args.steps, g0 + GROUP)):
@@ -342,6 +343,7 @@ def run_gpu(args, cfg):
             step_ev[i][0].record(stream)
             step()
             step_ev[i][1].record(stream)
+    gpu_launches = M.moe_launch_count() - launches0     # this library's kernels in the timed steps
     torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
     if dist:
@@ -423,7 +425,7 @@ def run_gpu(args, cfg):
             "e2e": {"value": cfg.T * world / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * es,
                     "d2h_bytes_per_step": cfg.T * cfg.H * es},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": gpu_launches,
             "clocks": clock_info,
             "gpu": torch.cuda.get_device_name(dev),
         }

@@ -60,6 +60,11 @@ typedef enum {
 /* Version of this ABI (bumped on any signature change). */
 int moe_abi_version(void);
 
+/* Number of kernels this library has enqueued in this process so far (all
+ * threads, all devices).  The difference across a region of calls is the
+ * number of GPU kernels those calls launched. */
+unsigned long long moe_launch_count(void);
+
 /* Message for the last non-OK return on the calling thread ("" if none).
  * The string stays valid until the next call on this thread. */
 const char* moe_last_error(void);

@@ -20,13 +20,14 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "MoEError", "lib_path", "load_library", "moe_abi_version", "moe_last_error",
+    "MoEError", "lib_path", "load_library", "moe_abi_version", "moe_launch_count",
+    "moe_last_error",
     "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_experts_workspace_bytes",
     "moe_experts", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
-    "KERNELS_PER_LAYER", "moe_layer_forward_host",
+    "moe_layer_forward_host",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
@@ -52,6 +53,7 @@ _SZ = ctypes.c_size_t
 
 _SIGS = {
     "moe_abi_version": (_I, []),
+    "moe_launch_count": (ctypes.c_ulonglong, []),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_route": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_dispatch_workspace_bytes": (_SZ, [_I, _I, _I]),
@@ -63,10 +65,6 @@ _SIGS = {
     "moe_read_status": (_I, [_P, _P, _P]),
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
 }
-
-# Kernels one moe_layer_forward launches: route 1, dispatch 4 (count, scan,
-# scatter, gather), experts 2 (w13 pass, w2 pass), combine 1.
-KERNELS_PER_LAYER = 8
 
 
 def load_library():
@@ -111,6 +109,11 @@ def _check(code: int):
 
 def moe_abi_version() -> int:
     return load_library().moe_abi_version()
+
+
+def moe_launch_count() -> int:
+    """Kernels this library has enqueued in this process so far."""
+    return int(load_library().moe_launch_count())
 
 
 def moe_last_error() -> str:

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <string>
@@ -15,6 +16,7 @@
 namespace {
 
 thread_local std::string g_err;
+std::atomic<unsigned long long> g_launches{0};
 
 int fail(int code, const std::string& msg) {
   g_err = msg;
@@ -54,6 +56,7 @@ __global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
 
 namespace moe_host {
 void set_last_error(const std::string& msg) { g_err = msg; }
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 cudaError_t ensure_smem(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -72,6 +75,7 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
 
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s) {
   probe_wait_kernel<<<1, 32, 0, s>>>(status, static_cast<uint64_t>(budget_us) * 1000ull);
+  if (cudaPeekAtLastError() == cudaSuccess) moe_host::note_launch();
   return cudaGetLastError();
 }
 }  // namespace moe_host
@@ -79,6 +83,8 @@ cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream
 extern "C" {
 
 int moe_abi_version(void) { return 2; }
+
+unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* moe_last_error(void) { return g_err.c_str(); }
 

@@ -108,6 +108,9 @@ void set_last_error(const std::string& msg);   // the message moe_last_error() r
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel, size).
 cudaError_t ensure_smem(const void* kernel, int bytes);
 
+// Count one kernel enqueued by this library (moe_launch_count).
+void note_launch();
+
 // Launch with programmatic stream serialization (and a cluster of cluster_x
 // CTAs along x when cluster_x > 0).
 template <typename... KArgs, typename... Args>
@@ -133,6 +136,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = n;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 }  // namespace moe_host

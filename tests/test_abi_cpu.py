@@ -31,7 +31,7 @@ def test_header_declares_the_stage_calls():
     names = _declared()
     for n in ("moe_route", "moe_dispatch", "moe_experts", "moe_combine",
               "moe_dispatch_workspace_bytes", "moe_experts_workspace_bytes", "moe_read_status",
-              "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version"):
+              "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version", "moe_launch_count"):
         assert n in names
 
 
@@ -53,6 +53,7 @@ def test_library_is_built_for_sm100a_only():
 
 def test_abi_version_and_workspace_queries(lib):
     assert M.moe_abi_version() == 2
+    assert M.moe_launch_count() == 0     # nothing launched on a CPU-only host
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
     assert M.moe_dispatch_workspace_bytes(0, 2, 8) == 0
