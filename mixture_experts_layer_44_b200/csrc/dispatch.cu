@@ -184,18 +184,27 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
   __syncthreads();
   const int per = (N + SMALL_WARPS - 1) / SMALL_WARPS;
   const int w0 = warp * per, w1 = min(N, w0 + per);
+  // The warp's slice of ids, read once (all loads in flight together) and
+  // kept in registers for both passes; -1 marks no assignment / a bad id.
+  constexpr int ROUNDS = SMALL_PER_WARP / 32;
+  const int nr = w1 > w0 ? (w1 - w0 + 31) / 32 : 0;   // rounds this warp needs
+  int eid[ROUNDS];
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    const int f = w0 + 32 * i + lane;
+    eid[i] = f < w1 ? ids[f] : -1;
+  }
   // 1. per-warp counts over this warp's contiguous slice
-  for (int r = w0; r < w1; r += 32) {
-    const int f = r + lane;
-    int e = -1;
-    if (f < w1) {
-      e = ids[f];
-      if (e < 0 || e >= E) {
-        moe::report(status, MOE_ERR_BAD_INDEX);
-        inv_perm[f] = -1;
-        e = -1;
-      }
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    if (i >= nr) break;
+    const int f = w0 + 32 * i + lane;
+    if (f < w1 && (eid[i] < 0 || eid[i] >= E)) {
+      moe::report(status, MOE_ERR_BAD_INDEX);
+      inv_perm[f] = -1;
+      eid[i] = -1;
     }
+    const int e = eid[i];
     const int key = e >= 0 ? e : -1 - lane;
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
@@ -228,13 +237,11 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
   if (e == 0) offsets[E] = s_scan[moe::kMaxExperts - 1];
   __syncthreads();
   // 3. stable scatter: slices in warp order, rounds in order, lanes in order
-  for (int r = w0; r < w1; r += 32) {
-    const int f = r + lane;
-    int ex = -1;
-    if (f < w1) {
-      ex = ids[f];
-      if (ex < 0 || ex >= E) ex = -1;
-    }
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    if (i >= nr) break;
+    const int f = w0 + 32 * i + lane;
+    const int ex = eid[i];
     const int key = ex >= 0 ? ex : -1 - lane;
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (ex >= 0) {
