@@ -124,11 +124,14 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
 
 // Split count: 1 when there are at least two tiles per CTA; otherwise the
 // smallest S whose units fill the grid's waves to >= 90% (else the best one),
-// with >= 4 K-blocks per unit and the units within the workspace.
-__device__ int choose_splits(int tiles, int grid, int kblocks, int max_units) {
+// with >= 4 K-blocks per unit, the units within the workspace, and at most
+// 128 partial rows per tile (S x the fullest tile's valid rows), since one
+// CTA reads them all back.
+__device__ int choose_splits(int tiles, int grid, int kblocks, int max_units, int rows_max) {
   if (tiles <= 0 || tiles >= 2 * grid) return 1;
   int smax = min(MAX_SPLITS, kblocks / 4);
   smax = min(smax, max_units / tiles);
+  smax = min(smax, max(2, BM / max(1, rows_max)));
   if (smax <= 1) return 1;
   int best = 1;
   float best_eff = 0.f;
@@ -267,17 +270,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Lane l owns experts [8l, 8l+8); lane 31 also writes the end entries.
     int cnt[8];
     int local = 0;
+    int rmax = 0;                     // valid rows of the fullest tile
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane * 8 + j;
       int m = 0;
       if (e < E) {
         c.offs[e] = offsets[e];
-        m = (offsets[e + 1] - offsets[e] + BM - 1) / BM;
+        const int rows = offsets[e + 1] - offsets[e];
+        m = (rows + BM - 1) / BM;
+        rmax = max(rmax, min(rows, BM));
       }
       cnt[j] = m;
       local += m;
     }
+    rmax = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(rmax)));
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       c.offs[E] = offsets[E];
       c.tstart[E] = incl * ntw;
       c.splits = (counters != nullptr && partials != nullptr && incl * ntw <= SCHED_TICKET)
-                     ? choose_splits(incl * ntw, gridDim.x, kblocks, max_units)
+                     ? choose_splits(incl * ntw, gridDim.x, kblocks, max_units, rmax)
                      : 1;
     }
   }
