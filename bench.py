@@ -291,14 +291,24 @@ def run_gpu(args, cfg):
                        stream=stream)
         if ev:
             ev[2].record(stream)
-        M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
-                      buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
-        if shared:
+        if not shared:
+            M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
+                          buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
+        else:
             M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
                         status=buf.status, stream=stream)
-            M.moe_experts(x, buf.sh_offsets, None, dp["w13s"].unsqueeze(0),
-                          dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
-                          status=buf.status, stream=stream)
+            if buf.fuse_shared:
+                M.moe_experts_shared(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"],
+                                     dp["w2"], buf.h, buf.y_packed, x, dp["w13s"], dp["w2s"],
+                                     buf.sh_h, buf.sh_y, ws=buf.ws_experts, status=buf.status,
+                                     stream=stream)
+            else:
+                M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"],
+                              buf.h, buf.y_packed, ws=buf.ws_experts, status=buf.status,
+                              stream=stream)
+                M.moe_experts(x, buf.sh_offsets, None, dp["w13s"].unsqueeze(0),
+                              dp["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
+                              status=buf.status, stream=stream)
         if ev:
             ev[3].record(stream)
         M.moe_combine(buf.y_packed, buf.inv_perm, cfg.T, cfg.k, buf.out,

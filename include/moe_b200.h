@@ -212,6 +212,27 @@ int moe_experts(const void* x_packed, const int32_t* offsets, const float* packe
                 int32_t* status, void* stream);
 
 /*
+ * moe_experts_shared -- the Executor of moe_experts plus one shared expert
+ * in the same pair of launches (diffulex.moe.layer, "SharedExpertMLP": an
+ * expert every token goes through).  The routed part is exactly moe_experts.
+ * The shared part computes, for every t < T,
+ *   h_s[t,i] = silu(x[t,:] . w13s[i,:]) * (x[t,:] . w13s[I_s+i,:])
+ *   y_s[t,c] = h_s[t,:] . w2s[c,:]                 (no routing weight)
+ * Its tiles are scheduled first, beside the routed ones, so the weight
+ * streams of both share every SM instead of running one after the other.
+ * bf16 only (fp32 returns MOE_ERR_UNSUPPORTED: call moe_experts twice).
+ *
+ *   x    device [T,H] bf16          w13s device [2*I_s,H]   w2s device [H,I_s]
+ *   h_s  device [T,I_s] bf16, written   y_s device [T,H] fp32, written
+ *   I_s % 128 == 0; all other arguments, results and rules as moe_experts.
+ */
+int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float* packed_w,
+                       const void* w13, const void* w2, int N, int H, int I, int E,
+                       const void* x, int T, const void* w13s, const void* w2s, int I_s,
+                       int dtype, void* h, void* y_packed, void* h_s, float* y_s, void* ws,
+                       size_t ws_bytes, int32_t* status, void* stream);
+
+/*
  * moe_combine -- Merger.  DWDP README, "Merger Module": restore token-major
  * assignment order, accumulate the top-k expert outputs and reshape back to
  * the token layout.  Routing weights were already applied by moe_experts.

@@ -24,7 +24,7 @@ __all__ = [
     "moe_last_error",
     "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_experts_workspace_bytes",
-    "moe_experts", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
+    "moe_experts", "moe_experts_shared", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
     "moe_layer_forward_host",
@@ -61,6 +61,8 @@ _SIGS = {
     "moe_dispatch_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_experts_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "moe_experts": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
+    "moe_experts_shared": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _I, _P, _P,
+                                _P, _P, _P, _SZ, _P, _P]),
     "moe_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_read_status": (_I, [_P, _P, _P]),
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
@@ -175,6 +177,22 @@ def moe_experts(x_packed, offsets, packed_w, w13, w2, h, y_packed, ws=None, stat
         ws.numel() * ws.element_size() if ws is not None else 0, _ptr(status), _stream(stream)))
 
 
+def moe_experts_shared(x_packed, offsets, packed_w, w13, w2, h, y_packed, x, w13s, w2s, h_s,
+                       y_s, ws=None, status=None, stream=None):
+    """moe_experts plus a shared expert (every row of x through w13s [2I_s,H],
+    w2s [H,I_s] into h_s, y_s) in the same two launches (bf16 only)."""
+    N, H = x_packed.shape
+    E = w13.shape[0]
+    I = w13.shape[1] // 2
+    T = x.shape[0]
+    I_s = w13s.shape[0] // 2
+    _check(load_library().moe_experts_shared(
+        _ptr(x_packed), _ptr(offsets), _ptr(packed_w), _ptr(w13), _ptr(w2), N, H, I, E,
+        _ptr(x), T, _ptr(w13s), _ptr(w2s), I_s, _dtype_code(x_packed), _ptr(h), _ptr(y_packed),
+        _ptr(h_s), _ptr(y_s), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
+        _ptr(status), _stream(stream)))
+
+
 def moe_combine(y_packed, inv_perm, T: int, k: int, out, shared=None, shared_gate_logit=None,
                 status=None, stream=None):
     H = out.shape[1]
@@ -228,6 +246,9 @@ class MoELayerBuffers:
                                                 else MOE_F32)), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
         self.shared_I = shared_I
+        # bf16 tensor-core layers run the shared expert inside the routed launches
+        self.fuse_shared = bool(shared_I) and dtype == torch.bfloat16 and H % 256 == 0 and \
+            I % 128 == 0 and shared_I % 128 == 0
         if shared_I:
             self.sg_logit = torch.empty(T, 1, **f32)
             self.sh_offsets = torch.tensor([0, T], **i32)
@@ -247,15 +268,25 @@ def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerB
               buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
-    moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
-                buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
     shared = sg = None
-    if params.get("w13s") is not None:
+    if params.get("w13s") is None:
+        moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
+                    buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
+    else:
         moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
                   status=buf.status, stream=stream)
-        moe_experts(x, buf.sh_offsets, None, params["w13s"].unsqueeze(0),
-                    params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
-                    status=buf.status, stream=stream)
+        if buf.fuse_shared:
+            moe_experts_shared(buf.x_packed, buf.offsets, buf.packed_w, params["w13"],
+                               params["w2"], buf.h, buf.y_packed, x, params["w13s"],
+                               params["w2s"], buf.sh_h, buf.sh_y, ws=buf.ws_experts,
+                               status=buf.status, stream=stream)
+        else:
+            moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"],
+                        buf.h, buf.y_packed, ws=buf.ws_experts, status=buf.status,
+                        stream=stream)
+            moe_experts(x, buf.sh_offsets, None, params["w13s"].unsqueeze(0),
+                        params["w2s"].unsqueeze(0), buf.sh_h, buf.sh_y, ws=buf.ws_experts,
+                        status=buf.status, stream=stream)
         shared, sg = buf.sh_y, buf.sg_logit
     moe_combine(buf.y_packed, buf.inv_perm, buf.T, k, buf.out, shared, sg, status=buf.status,
                 stream=stream)

@@ -158,39 +158,75 @@ size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype) {
   return dtype == MOE_BF16 ? moe_host::experts_ws_bytes() : 0;
 }
 
-int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
-                const void* w13, const void* w2, int N, int H, int I, int E, int dtype, void* h,
-                void* y_packed, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
-  g_err.clear();
+namespace {
+
+// Shared body of moe_experts and moe_experts_shared (sh == NULL: no shared
+// expert).
+int experts_impl(const char* fn, const void* x_packed, const int32_t* offsets,
+                 const float* packed_w, const void* w13, const void* w2, int N, int H, int I,
+                 int E, int dtype, void* h, void* y_packed, const moe_host::SharedGroup* sh,
+                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  const std::string f = std::string(fn) + ": ";
   if (int r = check_dtype(dtype)) return r;
-  REQ(N >= 0, MOE_ERR_INVALID_ARG, "moe_experts: N must be >= 0");
-  if (N == 0) return MOE_OK;
+  REQ(N >= 0, MOE_ERR_INVALID_ARG, f + "N must be >= 0");
+  if (N == 0 && sh == nullptr) return MOE_OK;
   REQ(x_packed && offsets && w13 && w2 && h && y_packed, MOE_ERR_INVALID_ARG,
-      "moe_experts: null input or output");
-  REQ(H >= 1 && I >= 1, MOE_ERR_INVALID_ARG, "moe_experts: H and I must be >= 1");
-  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_experts: E must be in [1, 256]");
-  REQ(H % 8 == 0 && I % 8 == 0, MOE_ERR_INVALID_ARG, "moe_experts: H and I must be multiples of 8");
+      f + "null input or output");
+  REQ(H >= 1 && I >= 1, MOE_ERR_INVALID_ARG, f + "H and I must be >= 1");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, f + "E must be in [1, 256]");
+  REQ(H % 8 == 0 && I % 8 == 0, MOE_ERR_INVALID_ARG, f + "H and I must be multiples of 8");
   REQ(aligned16(x_packed) && aligned16(w13) && aligned16(w2) && aligned16(h) && aligned16(y_packed),
-      MOE_ERR_INVALID_ARG, "moe_experts: tensors must be 16-byte aligned");
+      MOE_ERR_INVALID_ARG, f + "tensors must be 16-byte aligned");
   REQ(aligned4(offsets) && aligned4(packed_w) && aligned4(status), MOE_ERR_INVALID_ARG,
-      "moe_experts: offsets / packed_w / status must be 4-byte aligned");
-  REQ(aligned16(ws), MOE_ERR_INVALID_ARG, "moe_experts: ws must be 16-byte aligned");
+      f + "offsets / packed_w / status must be 4-byte aligned");
+  REQ(aligned16(ws), MOE_ERR_INVALID_ARG, f + "ws must be 16-byte aligned");
   REQ(static_cast<long long>(N) * (H > I ? H : I) < (1ll << 40) && N < (1 << 30),
-      MOE_ERR_INVALID_ARG, "moe_experts: N too large");
+      MOE_ERR_INVALID_ARG, f + "N too large");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == MOE_BF16) {
     REQ(H % 256 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
-        "moe_experts: the bf16 tensor-core path needs H % 256 == 0 and I % 128 == 0");
+        f + "the bf16 tensor-core path needs H % 256 == 0 and I % 128 == 0");
     const char* why = "";
     e = moe_host::launch_experts_tc(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h, y_packed,
-                                    ws, ws_bytes, status, s, &why);
-    if (e != cudaSuccess && why[0]) return fail(MOE_ERR_CUDA, std::string("moe_experts: ") + why);
+                                    sh, ws, ws_bytes, status, s, &why);
+    if (e != cudaSuccess && why[0]) return fail(MOE_ERR_CUDA, f + why);
   } else {
+    REQ(sh == nullptr, MOE_ERR_UNSUPPORTED,
+        f + "fp32: call moe_experts for the routed and for the shared expert");
     e = moe_host::launch_experts_simt(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h,
                                       y_packed, s);
   }
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_experts launch");
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, (f + "launch").c_str());
+}
+
+}  // namespace
+
+int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
+                const void* w13, const void* w2, int N, int H, int I, int E, int dtype, void* h,
+                void* y_packed, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  g_err.clear();
+  return experts_impl("moe_experts", x_packed, offsets, packed_w, w13, w2, N, H, I, E, dtype, h,
+                      y_packed, nullptr, ws, ws_bytes, status, stream);
+}
+
+int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float* packed_w,
+                       const void* w13, const void* w2, int N, int H, int I, int E,
+                       const void* x, int T, const void* w13s, const void* w2s, int I_s,
+                       int dtype, void* h, void* y_packed, void* h_s, float* y_s, void* ws,
+                       size_t ws_bytes, int32_t* status, void* stream) {
+  g_err.clear();
+  REQ(x && w13s && w2s && h_s && y_s, MOE_ERR_INVALID_ARG,
+      "moe_experts_shared: null shared-expert input or output");
+  REQ(T >= 1 && I_s >= 1, MOE_ERR_INVALID_ARG, "moe_experts_shared: T and I_s must be >= 1");
+  REQ(aligned16(x) && aligned16(w13s) && aligned16(w2s) && aligned16(h_s) && aligned16(y_s),
+      MOE_ERR_INVALID_ARG, "moe_experts_shared: shared-expert tensors must be 16-byte aligned");
+  REQ(I_s % 128 == 0, MOE_ERR_UNSUPPORTED, "moe_experts_shared: I_s must be a multiple of 128");
+  REQ(static_cast<long long>(T) * (H > I_s ? H : I_s) < (1ll << 40) && T < (1 << 30),
+      MOE_ERR_INVALID_ARG, "moe_experts_shared: T too large");
+  const moe_host::SharedGroup sh{x, T, w13s, w2s, I_s, h_s, y_s};
+  return experts_impl("moe_experts_shared", x_packed, offsets, packed_w, w13, w2, N, H, I, E,
+                      dtype, h, y_packed, &sh, ws, ws_bytes, status, stream);
 }
 
 int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,

@@ -92,10 +92,22 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
                             float* packed_w, void* x_packed, void* ws, int32_t* status,
                             cudaStream_t s);
 size_t experts_ws_bytes();
+// The optional shared expert of moe_experts_shared: every row of x [T,H]
+// through w13 [2I,H] / w2 [H,I] into h [T,I] (bf16) and y [T,H] (fp32).
+struct SharedGroup {
+  const void* x;
+  int T;
+  const void* w13;
+  const void* w2;
+  int I;
+  void* h;
+  void* y;
+};
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, void* ws, size_t ws_bytes,
-                              int32_t* status, cudaStream_t s, const char** why);
+                              int H, int I, int E, void* h, void* y, const SharedGroup* sh,
+                              void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s,
+                              const char** why);
 cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
                                 const float* packed_w, const void* w13, const void* w2, int N,
                                 int H, int I, int E, void* h, void* y, cudaStream_t s);

@@ -87,38 +87,71 @@ struct Ctl {
   int uid[UNIT_RING];
   uint32_t tmem_base;
   int abort;
-  int splits;          // S: K-slices per tile (1 = no split)
+  int splits;          // S: K-slices per routed tile (1 = no split)
+  int splits2;         // K-slices per shared-expert tile
   int last_flag;       // epilogue: this unit is the last of its tile
+  int n2;              // tiles of the second group (a shared expert), numbered first
+  int mte2;            // its token tiles
+  int rows2;           // its rows
   int offs[moe::kMaxExperts + 1];
-  int tstart[moe::kMaxExperts + 1];   // first tile of expert e (tiles = token tiles x NTW)
+  int tstart[moe::kMaxExperts + 1];   // first tile of routed expert e (after the n2 shared tiles)
 };
 
 constexpr int STAGE_OUT_BYTES = BM * 128;                  // epilogue staging: 128 rows x 128 B
 constexpr size_t CTL_BYTES = (sizeof(Ctl) + 127) / 128 * 128;
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTL_BYTES + STAGE_OUT_BYTES;
 
+// A work unit: tile (group g, expert e, weight tile nt, token tile mt) and
+// its K-slice [kb0, kb1).  Group 1 is the optional shared expert (all rows of
+// its own input), group 0 the routed experts.  Its rows are [row0, rend).
 struct Unit {
-  int tile, e, nt, mt, ks, kb0, kb1;
+  int tile, g, e, nt, mt, ks, S, kb0, kb1, row0, rend;
 };
 
-__device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, int u) {
+__device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, int kblocks2,
+                                            int u) {
+  // Units: the shared tiles' slices first (splits2 each), then the routed
+  // tiles' (splits each).  The unit id is also the partial slot of a slice.
   Unit r;
-  const int S = c.splits;
-  r.tile = u / S;
-  r.ks = u - r.tile * S;
-  r.kb0 = (r.ks * kblocks) / S;
-  r.kb1 = ((r.ks + 1) * kblocks) / S;
-  // largest e with tstart[e] <= tile (experts without tiles share their successor's start)
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (c.tstart[mid] <= r.tile) lo = mid; else hi = mid - 1;
+  const int u2 = c.n2 * c.splits2;
+  if (u < u2) {
+    r.S = c.splits2;
+    r.tile = u / r.S;
+    r.ks = u - r.tile * r.S;
+  } else {
+    r.S = c.splits;
+    const int v = u - u2;
+    r.tile = c.n2 + v / r.S;
+    r.ks = v - (r.tile - c.n2) * r.S;
   }
-  r.e = lo;
-  const int mte = (c.offs[r.e + 1] - c.offs[r.e] + BM - 1) / BM;
-  const int local = r.tile - c.tstart[r.e];
-  r.nt = local / mte;
-  r.mt = local - r.nt * mte;
+  int kb;
+  if (r.tile < c.n2) {
+    r.g = 1;
+    r.e = 0;
+    r.nt = r.tile / c.mte2;
+    r.mt = r.tile - r.nt * c.mte2;
+    r.row0 = r.mt * BM;
+    r.rend = c.rows2;
+    kb = kblocks2;
+  } else {
+    // largest e with tstart[e] <= tile (experts without tiles share their successor's start)
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (c.tstart[mid] <= r.tile) lo = mid; else hi = mid - 1;
+    }
+    r.g = 0;
+    r.e = lo;
+    const int mte = (c.offs[r.e + 1] - c.offs[r.e] + BM - 1) / BM;
+    const int local = r.tile - c.tstart[r.e];
+    r.nt = local / mte;
+    r.mt = local - r.nt * mte;
+    r.row0 = c.offs[r.e] + r.mt * BM;
+    r.rend = c.offs[r.e + 1];
+    kb = kblocks;
+  }
+  r.kb0 = (r.ks * kb) / r.S;
+  r.kb1 = ((r.ks + 1) * kb) / r.S;
   return r;
 }
 
@@ -228,9 +261,12 @@ template <int EPI>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmA2,
+                        const __grid_constant__ CUtensorMap tmB2,
                         const int32_t* __restrict__ offsets, int E, int K, int ntw,
                         int rows_per_expert, const float* __restrict__ packed_w,
-                        void* __restrict__ out, int ldo, int* __restrict__ counters,
+                        void* __restrict__ out, int ldo, int rows2, int K2, int ntw2,
+                        void* __restrict__ out2, int ldo2, int* __restrict__ counters,
                         float* __restrict__ partials, int max_units, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -240,6 +276,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int kblocks = K / BK;
+  const int kblocks2 = K2 / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -259,6 +296,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     moe::fence_barrier_init();
     moe::prefetch_tmap(&tmA);
     moe::prefetch_tmap(&tmB);
+    if (rows2 > 0) {
+      moe::prefetch_tmap(&tmA2);
+      moe::prefetch_tmap(&tmB2);
+    }
   }
   if (warp == 1) {
     moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
@@ -285,6 +326,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       local += m;
     }
     rmax = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(rmax)));
+    const int mte2 = (rows2 + BM - 1) / BM;      // the shared group's tiles come first
+    const int n2 = mte2 * ntw2;
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -295,23 +338,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane * 8 + j;
-      if (e < E) c.tstart[e] = run * ntw;
+      if (e < E) c.tstart[e] = n2 + run * ntw;
       run += cnt[j];
     }
     if (lane == 31) {
       c.offs[E] = offsets[E];
-      c.tstart[E] = incl * ntw;
-      c.splits = (counters != nullptr && partials != nullptr && incl * ntw <= SCHED_TICKET)
-                     ? choose_splits(incl * ntw, gridDim.x, kblocks, max_units, rmax)
-                     : 1;
+      const int tiles = n2 + incl * ntw;
+      c.tstart[E] = tiles;
+      c.n2 = n2;
+      c.mte2 = mte2;
+      c.rows2 = rows2;
+      const int rt = incl * ntw;                  // routed tiles
+      int sp = 1, sp2 = 1;
+      if (counters != nullptr && partials != nullptr && tiles <= SCHED_TICKET) {
+        if (rt == 0) {
+          sp2 = choose_splits(n2, gridDim.x, kblocks2, max_units, min(rows2, BM));
+        } else {
+          sp = choose_splits(tiles, gridDim.x, kblocks, max_units, max(rmax, min(rows2, BM)));
+          if (n2 > 0 && kblocks2 > kblocks) {
+            // a longer shared K is cut into slices about as long as the routed units
+            sp2 = min(sp * ((kblocks2 + kblocks - 1) / kblocks), MAX_SPLITS);
+            sp2 = min(sp2, max(1, kblocks2 / 4));
+            sp2 = min(sp2, max(2, BM / max(1, min(rows2, BM))));
+            if (n2 * sp2 + rt * sp > max_units) sp2 = sp;
+          } else {
+            sp2 = sp;
+          }
+        }
+      }
+      c.splits = sp;
+      c.splits2 = sp2;
     }
   }
   moe::tc_fence_before();
   __syncthreads();
   moe::tc_fence_after();
 
-  const int S = c.splits;
-  const int total = c.tstart[E] * S;        // units
+  const int total = c.n2 * c.splits2 + (c.tstart[E] - c.n2) * c.splits;   // units
   const uint32_t tmem = c.tmem_base;
 
   if (warp == 0) {
@@ -344,8 +407,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit(c, E, kblocks, u);
-        const int arow = c.offs[un.e] + un.mt * BM;
+        const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
+        const int arow = un.row0;
+        const CUtensorMap* ma = un.g ? &tmA2 : &tmA;
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
@@ -356,11 +420,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t fb = moe::smem_addr(&c.full[stage]);
           const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
           moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          moe::tma_load_2d(sa, &tmA, fb, kb * BK, arow);
-          if (EPI == EPI_SWIGLU)
+          moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
+          if (un.g) {
+            if (EPI == EPI_SWIGLU)
+              moe::tma_load_3d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), 0);
+            else
+              moe::tma_load_2d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * BN);
+          } else if (EPI == EPI_SWIGLU) {
             moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, un.nt * (BN / 2), 2 * un.e);
-          else
+          } else {
             moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, un.e * rows_per_expert + un.nt * BN);
+          }
           ++issued[stage];
           if (++stage == STAGES) {
             stage = 0;
@@ -393,7 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit(c, E, kblocks, u);
+        const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
         const int buf = i & 1;
         if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
           set_abort(c, status);
@@ -455,19 +525,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       moe::tc_fence_after();
-      const Unit un = decode_unit(c, E, kblocks, u);
-      const int rows_valid = c.offs[un.e + 1] - c.offs[un.e] - un.mt * BM;
+      const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
+      const int rows_valid = un.rend - un.row0;
       const bool live = row < rows_valid;
-      const size_t grow = static_cast<size_t>(c.offs[un.e] + un.mt * BM + row);
+      const size_t grow = static_cast<size_t>(un.row0 + row);
+      void* const uout = un.g ? out2 : out;          // the unit's group's output
+      const int uldo = un.g ? ldo2 : ldo;
+      const float* const upw = un.g ? nullptr : packed_w;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN);
       const int nvalid = rows_valid < BM ? rows_valid : BM;
       const bool staged = nvalid > STAGE_MIN_ROWS;    // same for all four epilogue warps
-      const size_t row0 = static_cast<size_t>(c.offs[un.e] + un.mt * BM);
+      const size_t row0 = static_cast<size_t>(un.row0);
+      const int S = un.S;
       if (S == 1) {
         if (EPI == EPI_SWIGLU && !staged) {
           // few valid rows: 16 h columns per step, each thread stores its own row
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + grow * ldo + un.nt * (BN / 2);
+          __nv_bfloat16* dst =
+              static_cast<__nv_bfloat16*>(uout) + grow * uldo + un.nt * (BN / 2);
 #pragma unroll 1
           for (int cc = 0; cc < BN / 2; cc += 16) {
             uint32_t g[16], v[16];
@@ -488,8 +563,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         } else if (EPI == EPI_SWIGLU) {
           // 64 h columns per staged chunk: gate cols hc.., up cols 128+hc..
-          uint8_t* gtile = static_cast<uint8_t*>(out) +
-                           (row0 * ldo + un.nt * (BN / 2)) * sizeof(__nv_bfloat16);
+          uint8_t* gtile = static_cast<uint8_t*>(uout) +
+                           (row0 * uldo + un.nt * (BN / 2)) * sizeof(__nv_bfloat16);
 #pragma unroll 1
           for (int hc = 0; hc < BN / 2; hc += 64) {
 #pragma unroll 1
@@ -518,12 +593,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             epi_bar();
             stage_flush(stg, q, lane, nvalid, gtile + hc * sizeof(__nv_bfloat16),
-                        static_cast<size_t>(ldo) * sizeof(__nv_bfloat16));
+                        static_cast<size_t>(uldo) * sizeof(__nv_bfloat16));
             epi_bar();
           }
         } else {
-          const float sc = live ? (packed_w ? packed_w[grow] : 1.f) : 0.f;
-          uint8_t* gtile = static_cast<uint8_t*>(out) + (row0 * ldo + un.nt * BN) * sizeof(float);
+          const float sc = live ? (upw ? upw[grow] : 1.f) : 0.f;
+          uint8_t* gtile =
+              static_cast<uint8_t*>(uout) + (row0 * uldo + un.nt * BN) * sizeof(float);
 #pragma unroll 1
           for (int cc = 0; cc < BN; cc += 32) {
             uint32_t a[16], b[16];
@@ -534,10 +610,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               stage_f32x32(stg, row, a, b, sc);
               epi_bar();
               stage_flush(stg, q, lane, nvalid, gtile + cc * sizeof(float),
-                          static_cast<size_t>(ldo) * sizeof(float));
+                          static_cast<size_t>(uldo) * sizeof(float));
               epi_bar();
             } else if (live) {
-              store_f32x32(reinterpret_cast<float*>(gtile) + static_cast<size_t>(row) * ldo + cc,
+              store_f32x32(reinterpret_cast<float*>(gtile) + static_cast<size_t>(row) * uldo + cc,
                            a, b, sc);
             }
           }
@@ -585,7 +661,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __threadfence();
           const int et = threadIdx.x - 64;                // 0..127
           const int nrows = nvalid;
-          const float* base = partials + static_cast<size_t>(un.tile) * S * (BM * BN);
+          const float* base = partials + static_cast<size_t>(u - un.ks) * (BM * BN);
           if (EPI == EPI_SWIGLU) {
             const int cg = et & 31;                       // h columns 4cg .. 4cg+3
             for (int r = et >> 5; r < nrows; r += 4) {
@@ -604,7 +680,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               uint2 pk;
               pk.x = moe::pack_bf16x2(silu_mul(g.x, v.x), silu_mul(g.y, v.y));
               pk.y = moe::pack_bf16x2(silu_mul(g.z, v.z), silu_mul(g.w, v.w));
-              *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + (row0 + r) * ldo +
+              *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(uout) + (row0 + r) * uldo +
                                         un.nt * (BN / 2) + cg * 4) = pk;
             }
           } else {
@@ -619,8 +695,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
                 }
               }
-              const float sc = packed_w ? packed_w[row0 + r] : 1.f;
-              *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + r) * ldo +
+              const float sc = upw ? upw[row0 + r] : 1.f;
+              *reinterpret_cast<float4*>(static_cast<float*>(uout) + (row0 + r) * uldo +
                                          un.nt * BN + cg * 4) =
                   make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
             }
@@ -663,16 +739,18 @@ size_t experts_ws_bytes() {
 
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, void* ws, size_t ws_bytes,
-                              int32_t* status, cudaStream_t s, const char** why) {
+                              int H, int I, int E, void* h, void* y, const SharedGroup* sh,
+                              void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s,
+                              const char** why) {
   cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU>),
                                 static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
   e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SCALE>),
                    static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
+  const int nmap = N > 0 ? N : 1;           // a map needs one row; no tile reads it when N == 0
   CUtensorMap mA1, mB1, mA2, mB2;
-  bool ok = map_rows(&mA1, x_packed, N, H) && map_rows(&mA2, h, N, I);
+  bool ok = map_rows(&mA1, x_packed, nmap, H) && map_rows(&mA2, h, nmap, I);
   {
     // w13 as [2E][I][H]: one box = 128 gate rows + the matching 128 up rows.
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
@@ -688,6 +766,22 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     const cuuint64_t str[1] = {static_cast<cuuint64_t>(I) * 2};
     const cuuint32_t box[2] = {BK, BN};
     ok = ok && encode_bf16_sw128(&mB2, w2, 2, dims, str, box);
+  }
+  // The shared expert's maps (x [T][H], w13s as [2][Is][H], h_s [T][Is], w2s [H][Is]);
+  // without one the routed maps stand in, unread.
+  CUtensorMap sA1 = mA1, sB1 = mB1, sA2 = mA2, sB2 = mB2;
+  const int T2 = sh ? sh->T : 0, Is = sh ? sh->I : 0;
+  if (sh) {
+    ok = ok && map_rows(&sA1, sh->x, T2, H) && map_rows(&sA2, sh->h, T2, Is);
+    const cuuint64_t d1[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(Is), 2};
+    const cuuint64_t s1[2] = {static_cast<cuuint64_t>(H) * 2,
+                              static_cast<cuuint64_t>(Is) * H * 2};
+    const cuuint32_t b1[3] = {BK, BN / 2, 2};
+    ok = ok && encode_bf16_sw128(&sB1, sh->w13, 3, d1, s1, b1);
+    const cuuint64_t d2[2] = {static_cast<cuuint64_t>(Is), static_cast<cuuint64_t>(H)};
+    const cuuint64_t s2[1] = {static_cast<cuuint64_t>(Is) * 2};
+    const cuuint32_t b2[2] = {BK, BN};
+    ok = ok && encode_bf16_sw128(&sB2, sh->w2, 2, d2, s2, b2);
   }
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
@@ -707,17 +801,19 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   int g1 = sms, g2 = sms;
   if (counters == nullptr) {   // no split possible: never more CTAs than tiles
     const int mt_bound = (N + BM - 1) / BM + E;
-    g1 = std::max(1, std::min(sms, mt_bound * (I / (BN / 2))));
-    g2 = std::max(1, std::min(sms, mt_bound * (H / BN)));
+    const int mt2 = (T2 + BM - 1) / BM;
+    g1 = std::max(1, std::min(sms, mt_bound * (I / (BN / 2)) + mt2 * (Is / (BN / 2))));
+    g2 = std::max(1, std::min(sms, (mt_bound + mt2) * (H / BN)));
   }
   const float* no_w = nullptr;
   cudaError_t err = launch_pdl(grouped_gemm_kernel<EPI_SWIGLU>, dim3(g1), dim3(NTHREADS),
-                               SMEM_BYTES, s, 0, mA1, mB1, offsets, E, H, I / (BN / 2), 2 * I,
-                               no_w, h, I, counters, partials, max_units, status);
+                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, offsets, E, H, I / (BN / 2),
+                               2 * I, no_w, h, I, T2, H, Is / (BN / 2), sh ? sh->h : nullptr, Is,
+                               counters, partials, max_units, status);
   if (err != cudaSuccess) return err;
   return launch_pdl(grouped_gemm_kernel<EPI_SCALE>, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
-                    mA2, mB2, offsets, E, I, H / BN, H, packed_w, y, H, counters, partials,
-                    max_units, status);
+                    mA2, mB2, sA2, sB2, offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
+                    sh ? sh->y : nullptr, H, counters, partials, max_units, status);
 }
 
 }  // namespace moe_host

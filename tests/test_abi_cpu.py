@@ -29,7 +29,7 @@ def lib():
 
 def test_header_declares_the_stage_calls():
     names = _declared()
-    for n in ("moe_route", "moe_dispatch", "moe_experts", "moe_combine",
+    for n in ("moe_route", "moe_dispatch", "moe_experts", "moe_experts_shared", "moe_combine",
               "moe_dispatch_workspace_bytes", "moe_experts_workspace_bytes", "moe_read_status",
               "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version", "moe_launch_count"):
         assert n in names
@@ -112,6 +112,22 @@ def test_experts_rejects_bad_arguments_on_the_host(lib):
     assert lib.moe_experts(*a) == M.MOE_OK
     a = list(base); a[3] = NULL
     assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+
+
+def test_experts_shared_rejects_bad_arguments_on_the_host(lib):
+    # routed part as above, then x, T, w13s, w2s, I_s, dtype, h, y, h_s, y_s, ws, bytes, status, stream
+    base = [P, P, P, P, P, 100, 256, 128, 4, P, 32, P, P, 512, M.MOE_BF16, P, P, P, P, NULL, 0,
+            NULL, NULL]
+    a = list(base); a[13] = 100           # I_s not a multiple of 128
+    assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED and "I_s" in _err(lib)
+    a = list(base); a[10] = 0             # T < 1
+    assert lib.moe_experts_shared(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[18] = NULL          # no y_s
+    assert lib.moe_experts_shared(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[14] = M.MOE_F32     # fp32 runs the two experts separately
+    assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED
+    a = list(base); a[6] = 200            # the routed rules still apply
+    assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED and "H % 256" in _err(lib)
 
 
 def test_combine_and_status_reject_bad_arguments_on_the_host(lib):

@@ -142,3 +142,42 @@ def test_experts_bf16_split_k_matches_unsplit_and_is_deterministic():
 
 def test_experts_bf16_without_workspace():
     _check(*_make([1, 0, 3], 512, 512, torch.bfloat16, seed=13), tol=TOL["bf16"], ws=None)
+
+
+@pytest.mark.parametrize("counts,H,I,T,Is", [
+    ([2, 0, 3, 2, 5, 4, 0, 1], 512, 256, 8, 512),     # decode: split-K over both groups
+    ([300, 0, 129, 40], 256, 128, 200, 384),          # prefill-like: no split
+    ([0, 0, 0, 1], 256, 128, 130, 256),               # shared rows span two token tiles
+])
+def test_experts_shared_matches_separate_calls(counts, H, I, T, Is):
+    x_packed, offs, pw, w13, w2 = _make(counts, H, I, torch.bfloat16, seed=T + Is)
+    g = torch.Generator().manual_seed(T)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    w13s = (torch.randn(2 * Is, H, generator=g) / H ** 0.5).to(torch.bfloat16)
+    w2s = (torch.randn(H, Is, generator=g) / Is ** 0.5).to(torch.bfloat16)
+    N = x_packed.shape[0]
+    h = torch.full((N, I), 1536.0, dtype=torch.bfloat16, device=DEV)
+    y = torch.full((N, H), 1536.0, dtype=torch.float32, device=DEV)
+    hs = torch.full((T, Is), 1536.0, dtype=torch.bfloat16, device=DEV)
+    ys = torch.full((T, H), 1536.0, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ws = _ws(x_packed, w13)
+    M.moe_experts_shared(dev(x_packed), dev(offs), dev(pw), dev(w13), dev(w2), h, y, dev(x),
+                         dev(w13s), dev(w2s), hs, ys, ws=ws, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert int(ws[:4096 * 4].view(torch.int32).abs().sum().item()) == 0
+    # routed part against the oracle, as moe_experts
+    ho, yo = O.experts(x_packed, offs.numpy(), pw, w13, w2)
+    assert err_bf16_out(h.cpu(), ho) <= TOL["bf16"] and rel(y.cpu(), yo) <= TOL["bf16"]
+    # shared part: every row of x through the dense SwiGLU MLP
+    hso, yso = O.experts(x, np.array([0, T]), None, w13s.unsqueeze(0), w2s.unsqueeze(0))
+    assert err_bf16_out(hs.cpu(), hso) <= TOL["bf16"] and rel(ys.cpu(), yso) <= TOL["bf16"]
+    np.testing.assert_allclose(ys.cpu().numpy(), O.shared_expert(x, w13s, w2s), rtol=0,
+                               atol=TOL["bf16"] * float(np.sqrt(np.mean(yso ** 2))))
+    # the same launch twice gives the same bits
+    y2 = torch.empty_like(y); ys2 = torch.empty_like(ys)
+    M.moe_experts_shared(dev(x_packed), dev(offs), dev(pw), dev(w13), dev(w2), h, y2, dev(x),
+                         dev(w13s), dev(w2s), hs, ys2, ws=ws, status=status)
+    torch.cuda.synchronize()
+    assert torch.equal(y2, y) and torch.equal(ys2, ys)
