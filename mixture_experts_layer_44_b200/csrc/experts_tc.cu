@@ -108,24 +108,26 @@ struct Unit {
   int tile, g, e, nt, mt, ks, S, kb0, kb1, row0, rend;
 };
 
+template <bool SHARED>
 __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, int kblocks2,
                                             int u) {
   // Units: the shared tiles' slices first (splits2 each), then the routed
   // tiles' (splits each).  The unit id is also the partial slot of a slice.
   Unit r;
-  const int u2 = c.n2 * c.splits2;
-  if (u < u2) {
+  const int u2 = SHARED ? c.n2 * c.splits2 : 0;
+  if (SHARED && u < u2) {
     r.S = c.splits2;
     r.tile = u / r.S;
     r.ks = u - r.tile * r.S;
   } else {
     r.S = c.splits;
+    const int n2 = SHARED ? c.n2 : 0;
     const int v = u - u2;
-    r.tile = c.n2 + v / r.S;
-    r.ks = v - (r.tile - c.n2) * r.S;
+    r.tile = n2 + v / r.S;
+    r.ks = v - (r.tile - n2) * r.S;
   }
   int kb;
-  if (r.tile < c.n2) {
+  if (SHARED && r.tile < c.n2) {
     r.g = 1;
     r.e = 0;
     r.nt = r.tile / c.mte2;
@@ -257,7 +259,7 @@ __device__ __forceinline__ void stage_f32x32(uint8_t* stg, int row, const uint32
                          __float_as_uint(__uint_as_float(b[4 * j + 3]) * sc)));
 }
 
-template <int EPI>
+template <int EPI, bool SHARED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -277,6 +279,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int lane = threadIdx.x & 31;
   const int kblocks = K / BK;
   const int kblocks2 = K2 / BK;
+  rows2 = SHARED ? rows2 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -407,9 +410,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
+        const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int arow = un.row0;
-        const CUtensorMap* ma = un.g ? &tmA2 : &tmA;
+        const bool g1 = SHARED && un.g;
+        const CUtensorMap* ma = g1 ? &tmA2 : &tmA;
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
@@ -421,7 +425,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
           moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
           moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
-          if (un.g) {
+          if (g1) {
             if (EPI == EPI_SWIGLU)
               moe::tma_load_3d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), 0);
             else
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
+        const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int buf = i & 1;
         if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
           set_abort(c, status);
@@ -525,13 +529,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       moe::tc_fence_after();
-      const Unit un = decode_unit(c, E, kblocks, kblocks2, u);
+      const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
       const int rows_valid = un.rend - un.row0;
       const bool live = row < rows_valid;
       const size_t grow = static_cast<size_t>(un.row0 + row);
-      void* const uout = un.g ? out2 : out;          // the unit's group's output
-      const int uldo = un.g ? ldo2 : ldo;
-      const float* const upw = un.g ? nullptr : packed_w;
+      const bool g1 = SHARED && un.g;
+      void* const uout = g1 ? out2 : out;            // the unit's group's output
+      const int uldo = g1 ? ldo2 : ldo;
+      const float* const upw = g1 ? nullptr : packed_w;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN);
       const int nvalid = rows_valid < BM ? rows_valid : BM;
@@ -742,11 +747,12 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               int H, int I, int E, void* h, void* y, const SharedGroup* sh,
                               void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s,
                               const char** why) {
-  cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SWIGLU>),
-                                static_cast<int>(SMEM_BYTES));
+  // The shared-expert group is compiled in only where it is used.
+  auto k1 = sh ? grouped_gemm_kernel<EPI_SWIGLU, true> : grouped_gemm_kernel<EPI_SWIGLU, false>;
+  auto k2 = sh ? grouped_gemm_kernel<EPI_SCALE, true> : grouped_gemm_kernel<EPI_SCALE, false>;
+  cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(k1), static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
-  e1 = ensure_smem(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI_SCALE>),
-                   static_cast<int>(SMEM_BYTES));
+  e1 = ensure_smem(reinterpret_cast<const void*>(k2), static_cast<int>(SMEM_BYTES));
   if (e1 != cudaSuccess) return e1;
   const int nmap = N > 0 ? N : 1;           // a map needs one row; no tile reads it when N == 0
   CUtensorMap mA1, mB1, mA2, mB2;
@@ -806,12 +812,12 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     g2 = std::max(1, std::min(sms, (mt_bound + mt2) * (H / BN)));
   }
   const float* no_w = nullptr;
-  cudaError_t err = launch_pdl(grouped_gemm_kernel<EPI_SWIGLU>, dim3(g1), dim3(NTHREADS),
+  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS),
                                SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, offsets, E, H, I / (BN / 2),
                                2 * I, no_w, h, I, T2, H, Is / (BN / 2), sh ? sh->h : nullptr, Is,
                                counters, partials, max_units, status);
   if (err != cudaSuccess) return err;
-  return launch_pdl(grouped_gemm_kernel<EPI_SCALE>, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
+  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
                     mA2, mB2, sA2, sB2, offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
                     sh ? sh->y : nullptr, H, counters, partials, max_units, status);
 }
