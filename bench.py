@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -93,12 +94,22 @@ def layer_work(cfg, counts):
     return b, f
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without comments and without whitespace runs (string
+    literals in these files hold no comment markers)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_source_hash():
+    """Hash of the grouped GEMM's code (comments and layout ignored, so that
+    a comment edit does not discard counters taken on the same code)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixture_experts_layer_44_b200", "csrc")
     for name in ("experts_tc.cu", "sm100_ptx.cuh", "common.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -24,13 +24,22 @@
 // weight tiles, token tiles fastest, so CTAs running at the same time share a
 // weight tile through L2.  Experts with no rows own no tiles.
 //
+// Shared expert (diffulex.moe.layer, "SharedExpertMLP").  With SHARED the
+// same launches also run a second group: every row of its own input x [T,H]
+// through its own w13s [2Is,H] (pass 1, into h_s) and w2s [H,Is] (pass 2,
+// into y_s, no routing weight).  Its tiles are numbered before the routed
+// ones, so the two weight streams share the SMs instead of following each
+// other.  The routed-only build (SHARED = false) carries none of it.
+//
 // Split-K.  When a pass has fewer tiles than two per CTA (decode batches, a
 // shared expert, a long K), every CTA derives the same split count S from the
 // tile count, the grid and K, and the work unit becomes (tile, K-slice).  A
-// unit stores the valid rows of its fp32 partial in the workspace; the last
-// unit of a tile to finish (a per-tile arrival counter) adds the S partials in
-// slice order (deterministic) and applies the epilogue.  The counter returns
-// to zero for the next call.
+// shared group whose K is longer than the routed one is cut into more slices,
+// about as long as the routed units.  A unit stores the valid rows of its fp32
+// partial in the workspace slot numbered like the unit; the last unit of a
+// tile to finish (a per-tile arrival counter) adds the S partials in slice
+// order (deterministic) and applies the epilogue.  The counter returns to zero
+// for the next call.
 //
 // Scheduling.  CTA b starts with unit b.  With a workspace, later units are
 // handed out dynamically: the producer warp takes the next unit from a

@@ -57,6 +57,14 @@ def test_ncu_traffic_is_dropped_when_the_kernel_changed(tmp_path, monkeypatch):
     assert bench.ncu_traffic("builder_bf16") == 123
 
 
+def test_kernel_hash_ignores_comments_but_not_code():
+    a = "int f(int x) {  // doubles\n  return 2 * x; /* fast */ }"
+    b = "int f(int x) {\n  return 2 * x;\n}"
+    c = "int f(int x) { return 3 * x; }"
+    assert bench.strip_comments(a) == bench.strip_comments(b)
+    assert bench.strip_comments(a) != bench.strip_comments(c)
+
+
 def test_reference_arm_prints_one_json_line_and_other_ranks_exit_quietly():
     cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
            "--workload", "tiny_f32", "--steps", "2", "--warmup", "3"]
