@@ -16,8 +16,20 @@ steps.  N > 1 (torchrun, one rank per GPU) runs independent replicas of the
 layer, each on its own token batch (weak scaling; the layer has no exchange
 step on one GPU's worth of experts), timed as the max over ranks.
 
-Prints ONE JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
-oracle instead (a bounded token sample per step; rank 0 only).
+Prints ONE JSON line on rank 0.  At N = 1 the line also carries a
+``workloads`` object: every full-size workload (the builder layer, the
+Qwen1.5-MoE-A2.7B shape at T = 32 and 8192, the Qwen3-30B-A3B shape at
+T = 16384, the large-expert decode layer at T = 1, 8, 64) timed the same way,
+each with its stage split, its layer roofline and its grouped-GEMM roofline
+against the measured and the nominal peaks (``--headline-only`` skips them).
+``--impl reference`` times the fp64 CPU oracle instead (a bounded token
+sample per step; rank 0 only).
+
+Roofline of the grouped GEMM (``roofline``): its algorithmic bytes are the
+weights of the experts that received tokens (plus a shared expert's); its
+flops 2*N*3*H*I (+ the shared expert's).  The packed intermediates it also
+moves (x_packed, h, fp32 y_packed) are reported beside it
+(``bytes_incl_packed``, ``frac_incl_packed``), not in ``frac``.
 """
 from __future__ import annotations
 
@@ -59,23 +71,38 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback (6.65 TB/s, 1.59 PFLOP/s earlier pool measurement)"
 
 
-def expert_stage_work(cfg, counts):
-    """Algorithmic bytes and flops of the grouped-GEMM stage (both passes) for
-    the realised per-expert counts: weights of every expert with >= 1 row,
-    x_packed read, h written and read back, y_packed written (fp32), routing
-    weights; with a shared expert also its weights, x read, its h written and
-    read back and its fp32 output written."""
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}   # B200 nominal HBM3e and dense bf16
+
+
+def expert_weight_work(cfg, counts):
+    """Algorithmic bytes and flops of the grouped-GEMM stage (both passes):
+    the weights of every expert with >= 1 row (w13 and w2), plus the shared
+    expert's; flops 2*N*3*H*I (+ 2*T*3*H*I_s).  The packed intermediates
+    (x_packed, h, y_packed) are not algorithmic and are not counted."""
     es = 2 if cfg.dtype == "bf16" else 4
     active = sum(1 for c in counts if c > 0)
     N = int(sum(counts))
     H, I = cfg.H, cfg.I
     wbytes = active * 3 * H * I * es
-    abytes = N * H * es + 2 * N * I * es + N * H * 4 + N * 4
     flops = 2 * N * 3 * H * I
     if cfg.shared_I:
         wbytes += 3 * H * cfg.shared_I * es
-        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * 4
         flops += 2 * cfg.T * 3 * H * cfg.shared_I
+    return wbytes, flops
+
+
+def expert_stage_work(cfg, counts):
+    """The same stage's bytes INCLUDING the materialised intermediates (x_packed
+    read, h written and read back, fp32 y_packed written, routing weights;
+    with a shared expert also its x read, h_s written and read, fp32 output
+    written), and its flops."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    N = int(sum(counts))
+    H, I = cfg.H, cfg.I
+    wbytes, flops = expert_weight_work(cfg, counts)
+    abytes = N * H * es + 2 * N * I * es + N * H * 4 + N * 4
+    if cfg.shared_I:
+        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * 4
     return wbytes + abytes, flops
 
 
@@ -92,6 +119,58 @@ def layer_work(cfg, counts):
         b += 3 * H * cfg.shared_I * es + H * es
         f += 2 * T * 3 * H * cfg.shared_I + 2 * T * H
     return b, f
+
+
+def gemm_roofline(cfg, counts, t_ms, peaks):
+    """Roofline of the grouped-GEMM stage over the live stage time t_ms:
+    bound "tensor" when its flops per algorithmic byte reach the measured
+    ridge, else "hbm"; fractions of the measured peaks and of the nominal
+    ones; the intermediates-inclusive byte rate beside it."""
+    wb, fl = expert_weight_work(cfg, counts)
+    ib, _ = expert_stage_work(cfg, counts)
+    t = t_ms / 1e3
+    hbm, tf = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    if fl / wb >= tf * 1e12 / (hbm * 1e9):
+        r = {"bound": "tensor", "achieved": fl / t / 1e12, "peak": tf, "unit": "TFLOP/s"}
+        r["frac_nominal"] = r["achieved"] / NOMINAL["bf16_tflops"]
+    else:
+        r = {"bound": "hbm", "achieved": wb / t / 1e9, "peak": hbm, "unit": "GB/s"}
+        r["frac_nominal"] = r["achieved"] / NOMINAL["hbm_gbs"]
+    r["frac"] = r["achieved"] / r["peak"]
+    r["bytes_alg"] = wb
+    r["flops"] = fl
+    r["bytes_incl_packed"] = ib
+    r["gbs_incl_packed"] = ib / t / 1e9
+    r["frac_incl_packed"] = r["gbs_incl_packed"] / hbm
+    return r
+
+
+def layer_roofline(cfg, counts, ms, peaks):
+    """t_roof = max(layer bytes / HBM, layer flops / bf16 peak) against the
+    measured step time, for the measured and for the nominal peaks."""
+    lb, lf = layer_work(cfg, counts)
+    out = {"bytes": lb, "flops": lf}
+    for tag, pk in (("", peaks), ("_nominal", NOMINAL)):
+        tb = lb / (pk["hbm_gbs"] * 1e9)
+        tfl = lf / (pk["bf16_tflops"] * 1e12)
+        out["bound" + tag] = "hbm" if tb >= tfl else "tensor"
+        out["t_roof_ms" + tag] = max(tb, tfl) * 1e3
+        out["frac" + tag] = max(tb, tfl) / (ms / 1e3)
+    return out
+
+
+def zipf_slope(counts):
+    """Least-squares slope of log(count) against log(rank) over the experts
+    that received tokens (rank 1 = the most loaded): the realised skew."""
+    import math
+    c = sorted((x for x in counts if x > 0), reverse=True)
+    if len(c) < 2:
+        return None
+    xs = [math.log(r) for r in range(1, len(c) + 1)]
+    ys = [math.log(v) for v in c]
+    mx, my = sum(xs) / len(xs), sum(ys) / len(ys)
+    sxx = sum((a - mx) ** 2 for a in xs)
+    return sum((a - mx) * (b - my) for a, b in zip(xs, ys)) / sxx
 
 
 def strip_comments(src: str) -> str:
@@ -193,16 +272,23 @@ class ClockSampler:
         except (FileNotFoundError, OSError):
             self.proc = None
 
-    def stop(self):
+    def stop_raw(self) -> str:
+        """Stop sampling; the CSV rows seen ("" without nvidia-smi)."""
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return ""
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        return parse_clock_samples(out)
+        self.proc = None
+        return out
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        return parse_clock_samples(self.stop_raw())
 
 
 # ---------------------------------------------------------- CPU oracle ---
@@ -264,42 +350,32 @@ def workload_config(cfg, counts):
 
 # ------------------------------------------------------------ GPU path ---
 
-def run_gpu(args, cfg):
-    import mixture_experts_layer_44_b200 as M
+FULL_WORKLOADS = ["builder_bf16", "qwen15_t32", "qwen15_t8192", "qwen3_t16384", "decode_t1",
+                  "decode_t8", "decode_t64"]
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    M.load_library()
-    dev = torch.device("cuda", local)
 
-    p = rank_inputs(cfg, rank)
-    dp = {k: (v.to(dev) if v is not None else None) for k, v in p.items()}
-    buf = M.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.torch_dtype, device=dev,
-                            shared_I=cfg.shared_I)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    x = dp["x"]
-    E = cfg.E
-    shared = cfg.shared_I is not None
-    def step(ev=None):
+class Layer:
+    """One layer instance on the device with its buffers, and its step."""
+
+    def __init__(self, M, cfg, rank, dev, stream):
+        self.M, self.cfg, self.stream = M, cfg, stream
+        self.p = rank_inputs(cfg, rank)
+        self.dp = {k: (v.to(dev) if v is not None else None) for k, v in self.p.items()}
+        self.buf = M.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.torch_dtype,
+                                     device=dev, shared_I=cfg.shared_I)
+
+    def step(self, ev=None):
         # Each stage's events are recorded on the stream its kernels run on.
+        M, cfg, buf, dp, stream = self.M, self.cfg, self.buf, self.dp, self.stream
+        x = dp["x"]
+        shared = cfg.shared_I is not None
         if ev:
             ev[0].record(stream)
         M.moe_route(x, dp["W_gate"], dp["bias"], cfg.k, cfg.renormalize, buf.logits, buf.ids,
                     buf.w, status=buf.status, stream=stream)
         if ev:
             ev[1].record(stream)
-        M.moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
+        M.moe_dispatch(buf.ids, buf.w, x, cfg.E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                        buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status,
                        stream=stream)
         if ev:
@@ -330,57 +406,111 @@ def run_gpu(args, cfg):
         if ev:
             ev[4].record(stream)
 
+
+def time_layer(layer, steps, warmup, flush, dev, dist=None, clocks=None):
+    """Warm up, then time ``steps`` steps (one event pair each, L2 flushed
+    before every step, outside the events), then a second pass with an event
+    between stages.  Returns (mean ms per step, mean ms per stage, library
+    kernels launched in the timed steps, raw clock samples or None)."""
+    M, stream = layer.M, layer.stream
+
     def flush_l2():
         flush.zero_()                 # write > L2 ...
         flush.sum()                   # ... then read it, leaving clean lines only
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush_l2()
-        step()
+        layer.step()
     torch.cuda.synchronize(dev)
-    if int(buf.status.item()) != 0:
-        raise SystemExit(f"device status {int(buf.status.item())} after warm-up")
-    counts = buf.counts.cpu().tolist()
-
-    # Timed region: K steps, each bracketed by two events only.  Steps are
-    # enqueued in groups behind a short GPU spin (outside every bracket), so
-    # the GPU runs each group back to back and no bracket contains time spent
-    # waiting for the host.  A second pass of K steps with an event between
-    # stages gives the per-stage split (events between small kernels cost a
-    # few microseconds each, so the step time comes from the first pass).
+    if int(layer.buf.status.item()) != 0:
+        raise SystemExit(f"device status {int(layer.buf.status.item())} after warm-up "
+                         f"({layer.cfg.name})")
+    # Steps are enqueued in groups behind a short GPU spin (outside every
+    # bracket), so the GPU runs each group back to back and no bracket
+    # contains time spent waiting for the host.  Events between small kernels
+    # cost a few microseconds each, so the step time comes from the first pass.
     GROUP = 8
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+               for _ in range(steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.3)
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
     launches0 = M.moe_launch_count()
-    for g0 in range(0, args.steps, GROUP):
+    for g0 in range(0, steps, GROUP):
         torch.cuda._sleep(int(20e6))            # ~10 ms of GPU spin while the host enqueues
-        for i in range(g0, min(args.steps, g0 + GROUP)):
+        for i in range(g0, min(steps, g0 + GROUP)):
             flush_l2()
             step_ev[i][0].record(stream)
-            step()
+            layer.step()
             step_ev[i][1].record(stream)
-    gpu_launches = M.moe_launch_count() - launches0     # this library's kernels in the timed steps
+    launches = M.moe_launch_count() - launches0     # this library's kernels in the timed steps
     torch.cuda.synchronize(dev)
-    clock_info = clocks.stop()
+    raw = clocks.stop_raw() if clocks else None
     if dist:
         dist.barrier()
-    ms = sum(a.elapsed_time(b) for a, b in step_ev) / args.steps
-    for g0 in range(0, args.steps, GROUP):
+    ms = sum(a.elapsed_time(b) for a, b in step_ev) / steps
+    for g0 in range(0, steps, GROUP):
         torch.cuda._sleep(int(20e6))
-        for i in range(g0, min(args.steps, g0 + GROUP)):
+        for i in range(g0, min(steps, g0 + GROUP)):
             flush_l2()
-            step(evs[i])
+            layer.step(evs[i])
     torch.cuda.synchronize(dev)
-    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
-    per_stage = [sum(s[j] for s in stage_ms) / args.steps for j in range(4)]
+    stage_ms = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(steps)]
+    per_stage = [sum(s[j] for s in stage_ms) / steps for j in range(4)]
+    if int(layer.buf.status.item()) != 0:
+        raise SystemExit(f"device status {int(layer.buf.status.item())} after timing "
+                         f"({layer.cfg.name})")
+    return ms, per_stage, launches, raw
+
+
+def stage_dict(per_stage):
+    return {"route": per_stage[0], "dispatch": per_stage[1], "experts": per_stage[2],
+            "combine": per_stage[3]}
+
+
+def workload_summary(cfg, counts, ms, per_stage, launches, steps, peaks):
+    """One entry of the line's ``workloads`` object."""
+    return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3), "T": cfg.T,
+            "stage_ms": stage_dict(per_stage),
+            "layer_roofline": layer_roofline(cfg, counts, ms, peaks),
+            "gemm_roofline": gemm_roofline(cfg, counts, per_stage[2], peaks),
+            "active_experts": sum(1 for c in counts if c > 0), "max_expert_rows": max(counts),
+            "zipf_slope_realised": zipf_slope(counts) if cfg.zipf_s is not None else None,
+            "gpu_launches_per_step": launches / steps}
+
+
+def run_gpu(args, cfg):
+    import mixture_experts_layer_44_b200 as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    M.load_library()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_src = load_peaks()
+
+    layer = Layer(M, cfg, rank, dev, stream)
+    clocks = ClockSampler(local)
+    ms, per_stage, gpu_launches, raw_clocks = time_layer(layer, args.steps, args.warmup, flush,
+                                                         dev, dist, clocks)
+    counts = layer.buf.counts.cpu().tolist()
     ms_max = max_over_ranks(ms, dev)
+    p, dp, buf = layer.p, layer.dp, layer.buf
 
     # End to end through the public API with host buffers: pinned x in, out back.
     x_host = p["x"].pin_memory()
@@ -393,7 +523,8 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize(dev)
     e2e_ms_list = []
     for _ in range(e2e_steps):
-        flush_l2()
+        flush.zero_()
+        flush.sum()
         e_start.record(stream)
         M.moe_layer_forward_host(x_host, dp, cfg.k, cfg.renormalize, buf, out_host, stream=stream)
         e_end.record(stream)
@@ -403,28 +534,36 @@ def run_gpu(args, cfg):
     e2e_ms = max_over_ranks(e2e_ms, dev)
     if int(buf.status.item()) != 0:
         raise SystemExit(f"device status {int(buf.status.item())} after timing")
+    del layer, dp, buf
+
+    # Every other full-size workload, one at a time, at N = 1 (the same timing).
+    workloads = {}
+    if cfg.name in FULL_WORKLOADS:
+        workloads[cfg.name] = workload_summary(cfg, counts, ms, per_stage, gpu_launches,
+                                               args.steps, peaks)
+    clock_raw = [raw_clocks] if raw_clocks else []
+    if world == 1 and args.all_workloads:
+        for name in FULL_WORKLOADS:
+            if name == cfg.name:
+                continue
+            wcfg = CONFIGS[name]
+            wl = Layer(M, wcfg, rank, dev, stream)
+            wms, wst, wla, wraw = time_layer(wl, args.steps, max(3, min(args.warmup, 5)), flush,
+                                             dev, None, clocks)
+            if wraw:
+                clock_raw.append(wraw)
+            workloads[name] = workload_summary(wcfg, wl.buf.counts.cpu().tolist(), wms, wst,
+                                               wla, args.steps, peaks)
+            del wl
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        peaks, peak_src = load_peaks()
-        hbm = peaks["hbm_gbs"]
-        tf = peaks["bf16_tflops"]
-        bytes_x, flops_x = expert_stage_work(cfg, counts)
-        t_x = per_stage[2] / 1e3
-        ai = flops_x / bytes_x
-        ridge = tf * 1e12 / (hbm * 1e9)
-        if ai >= ridge:
-            roof = {"bound": "tensor", "achieved": flops_x / t_x / 1e12, "peak": tf,
-                    "unit": "TFLOP/s"}
-        else:
-            roof = {"bound": "hbm", "achieved": bytes_x / t_x / 1e9, "peak": hbm, "unit": "GB/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        tr = ncu_traffic(cfg.name)
-        roof["traffic"] = tr
+        roof = gemm_roofline(cfg, counts, per_stage[2], peaks)
+        roof["traffic"] = ncu_traffic(cfg.name)
         roof["kernel"] = ("grouped_gemm_kernel (tcgen05), both passes of moe_experts: "
-                          f"{bytes_x/1e9:.3f} GB and {flops_x/1e9:.1f} GFLOP per step")
-        roof["peak_source"] = peak_src
-        lb, lf = layer_work(cfg, counts)
-        t_roof = max(lb / (hbm * 1e9), lf / (tf * 1e12))
+                          f"{roof['bytes_alg']/1e9:.3f} GB of activated expert weights and "
+                          f"{roof['flops']/1e9:.1f} GFLOP per step")
+        roof["peak_source"] = peak_src + ", burst figures (each step lasts under 2 ms)"
         cpu = None
         if not args.no_cpu_baseline:
             ntok = min(CPU_SAMPLE_TOKENS, cfg.T)
@@ -437,17 +576,19 @@ def run_gpu(args, cfg):
                    "sample": f"first {ntok} of {cfg.T} tokens, fp64 numpy oracle (router, "
                              f"dispatch, experts, merge), {runs} run(s), {secs:.1f} s"}
         es = 2 if cfg.dtype == "bf16" else 4
+        wcfg = workload_config(cfg, counts)
+        wcfg["zipf_slope_realised"] = zipf_slope(counts) if cfg.zipf_s is not None else None
+        clock_info = parse_clock_samples("\n".join(clock_raw)) if clock_raw else \
+            {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         line = {
             "metric": METRIC, "value": cfg.T * world / (ms_max / 1e3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights)",
-            "config": workload_config(cfg, counts),
+            "config": wcfg,
             "roofline": roof,
-            "layer_roofline": {"bytes": lb, "flops": lf, "t_roof_ms": t_roof * 1e3,
-                               "frac": t_roof / (ms / 1e3)},
-            "stage_ms": {"route": per_stage[0], "dispatch": per_stage[1],
-                         "experts": per_stage[2], "combine": per_stage[3]},
+            "layer_roofline": layer_roofline(cfg, counts, ms, peaks),
+            "stage_ms": stage_dict(per_stage),
             "cpu_baseline": cpu,
             "e2e": {"value": cfg.T * world / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.H * es,
@@ -455,6 +596,7 @@ def run_gpu(args, cfg):
             "gpu_launches": gpu_launches,
             "clocks": clock_info,
             "gpu": torch.cuda.get_device_name(dev),
+            "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
     if dist:
@@ -471,6 +613,9 @@ def main():
     ap.add_argument("--workload", default="builder_bf16", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", dest="all_workloads", action="store_false",
+                    help="skip the other full-size workloads (the line's `workloads` object); "
+                         "they are measured by default at N = 1")
     ap.add_argument("--profile-small", action="store_true",
                     help="the workload with E=16 experts and T=1024 tokens (weights 0.55 GB, "
                          "still above L2): the case detailed ncu captures run on")

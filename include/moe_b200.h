@@ -156,8 +156,10 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x,
  *     larger problems return MOE_ERR_INVALID_ARG with a message naming the
  *     limit.  Use moe_dispatch with a workspace for them.
  *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress, then cached), so make that first call
- *     before any stream capture.
+ *     device (cudaGetSymbolAddress), so make that first call before any
+ *     stream capture.  The address is cached per device and CUDA context and
+ *     looked up again when the context changes (after cudaDeviceReset, the
+ *     next call does the look-up again: make it outside a capture too).
  *   - All calls share the one array and it keeps the last call's contents
  *     (nothing in it needs to start at zero).  Two calls whose work overlaps
  *     on the GPU (different streams, or different host threads) race on it:

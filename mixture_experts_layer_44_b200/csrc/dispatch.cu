@@ -25,6 +25,8 @@
 //   gather  -- x_packed[p] = x[packed_tok[p]] with bulk asynchronous copies
 //              (global -> shared -> global on the TMA engine), one issuing
 //              lane per warp, a 4-row ring per warp.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <mutex>
 #include <string>
@@ -450,23 +452,57 @@ static __device__ __align__(256) int32_t g_dispatch_scratch[kNoAllocScratchInts]
 
 namespace {
 
+// Id of the calling thread's current CUDA context (0 if it cannot be read).
+// Context ids are never reused within a process, so a cached address keyed
+// on one cannot outlive the context it was taken in (cudaDeviceReset
+// destroys the primary context; the next one gets a new id).
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_cur == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // Device address of g_dispatch_scratch on the current device.  In host code
 // the array's name only stands in for the symbol; the address a kernel may
-// use comes from cudaGetSymbolAddress, called once per device (with that
-// device current) and cached.
+// use comes from cudaGetSymbolAddress, called with the device current.  It is
+// cached per device together with the id of the context it was taken in,
+// and looked up again whenever that context has changed (after a
+// cudaDeviceReset, say), so a stale address is never handed to a kernel.
 cudaError_t noalloc_scratch(void** out) {
   static std::mutex mu;
   static void* cached[kMaxDevices] = {};
+  static unsigned long long cached_ctx[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();   // 0 before the first runtime call
+  if (cached[dev] == nullptr || ctx == 0 || cached_ctx[dev] != ctx) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+    e = cudaGetSymbolAddress(&p, g_dispatch_scratch);    // makes the primary context current
     if (e != cudaSuccess) return e;
     cached[dev] = p;
+    cached_ctx[dev] = current_context_id();
   }
   *out = cached[dev];
   return cudaSuccess;

@@ -27,6 +27,45 @@ def test_expert_stage_work_counts_only_active_experts():
     assert b == 2 * 3 * H * I * 2 + N * H * 2 + 2 * N * I * 2 + N * H * 4 + N * 4
 
 
+def test_gemm_roofline_counts_only_activated_weights():
+    cfg = CONFIGS["builder_bf16"]
+    counts = [0] * 64
+    counts[3] = 8000
+    counts[9] = 192
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}
+    H, I, N = 4096, 1408, 8192
+    wb, fl = bench.expert_weight_work(cfg, counts)
+    assert wb == 2 * 3 * H * I * 2 and fl == 2 * N * 3 * H * I
+    r = bench.gemm_roofline(cfg, counts, 0.5, peaks)
+    # flops / weight bytes = 2*8192/2 = 8192 > ridge 250: tensor bound
+    assert r["bound"] == "tensor"
+    assert abs(r["achieved"] - fl / 0.5e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 1500.0) < 1e-12
+    assert abs(r["frac_nominal"] - r["achieved"] / 2250.0) < 1e-12
+    assert r["bytes_incl_packed"] == bench.expert_stage_work(cfg, counts)[0]
+    # every expert active at uniform load: weight-bound
+    r = bench.gemm_roofline(cfg, [128] * 64, 0.4, peaks)
+    assert r["bound"] == "hbm"
+    assert abs(r["achieved"] - 64 * 3 * H * I * 2 / 0.4e-3 / 1e9) < 1e-6
+    assert r["frac_incl_packed"] > r["frac"]
+
+
+def test_layer_roofline_against_measured_and_nominal_peaks():
+    cfg = CONFIGS["decode_t1"]
+    counts = [0, 1, 0, 0, 0, 0, 1, 0]
+    lb, lf = bench.layer_work(cfg, counts)
+    r = bench.layer_roofline(cfg, counts, 0.2, {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0})
+    assert r["bound"] == r["bound_nominal"] == "hbm"
+    assert abs(r["frac"] - lb / 6000e9 / 0.2e-3) < 1e-12
+    assert abs(r["frac_nominal"] - lb / 8000e9 / 0.2e-3) < 1e-12
+
+
+def test_zipf_slope_of_an_exact_power_law():
+    counts = [int(round(1e6 * r ** -1.1)) for r in range(1, 121)] + [0] * 8
+    assert abs(bench.zipf_slope(counts) + 1.1) < 1e-3
+    assert bench.zipf_slope([5, 0, 0]) is None
+
+
 def test_layer_work_includes_router_and_shared_expert():
     cfg = CONFIGS["qwen15_t32"]
     counts = [1] * 60

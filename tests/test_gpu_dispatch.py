@@ -99,3 +99,41 @@ def test_dispatch_bad_ids_are_reported_and_skipped():
     flat = valid.reshape(-1).tolist()
     order = sorted([f for f in range(8) if 0 <= flat[f] < 4], key=lambda f: (flat[f], f))
     assert g["perm"][:6].tolist() == order
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dispatch_bad_ids_on_the_multi_block_path(dtype):
+    # 5000 tokens x top-2 = 10000 assignments: the count / scan / scatter kernels
+    # (2048 assignments per block) and the bulk-copy gather; out-of-range ids in
+    # several blocks, including the last, partial one.
+    rng = np.random.default_rng(21)
+    T, k, E, H = 5000, 2, 64, 96
+    ids = rand_ids(rng, T, k, E)
+    flat = ids.view(-1)
+    bad = {5: 64, 2047: -1, 2048: 1000, 4100: -7, 9000: 64, 9999: 2 ** 31 - 1}
+    for f, e in bad.items():
+        flat[f] = e
+    w = torch.tensor(rng.random((T, k)), dtype=torch.float32)
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(21)).to(dtype)
+    g = _run(ids, w, x, E)
+    assert int(g["status"][0]) == M.MOE_ERR_BAD_INDEX
+    # expected: the stable order (expert, then flat index) of the valid assignments only
+    fl = flat.numpy().astype(np.int64)
+    valid = np.nonzero((fl >= 0) & (fl < E))[0]
+    nv = len(valid)
+    order = valid[np.lexsort((valid, fl[valid]))]
+    counts = np.bincount(fl[valid], minlength=E)
+    np.testing.assert_array_equal(g["counts"].numpy(), counts)
+    np.testing.assert_array_equal(g["offsets"].numpy(), np.concatenate([[0], np.cumsum(counts)]))
+    assert g["offsets"][E].item() == nv == T * k - len(bad)
+    np.testing.assert_array_equal(g["perm"][:nv].numpy(), order)
+    inv = np.full(T * k, -1)
+    inv[order] = np.arange(nv)
+    np.testing.assert_array_equal(g["inv_perm"].numpy(), inv)
+    np.testing.assert_array_equal(g["packed_tok"][:nv].numpy(), order // k)
+    np.testing.assert_array_equal(g["packed_w"][:nv].numpy(), w.numpy().reshape(-1)[order])
+    want = x[torch.as_tensor(order // k)]
+    assert torch.equal(g["x_packed"][:nv].contiguous().view(torch.uint8),
+                       want.contiguous().view(torch.uint8))
+    # rows past the valid ones are left as they were
+    assert (g["perm"][nv:] == -7).all() and (g["packed_tok"][nv:] == -7).all()

@@ -5,15 +5,25 @@ benchmark times (moe_layer_forward over MoELayerBuffers), for every workload.
   ids identical to the oracle's selection on the GPU's own logits; against
   the oracle's own fp64 selection, a differing id is allowed only where the
   two experts' fp64 logits differ by less than 1e-5;
-* dispatch: identical to the oracle's stable sort of the GPU's ids;
-* output: every token (tiny workload) or a sample of tokens (full-size
-  workloads) against the oracle's per-token form with the GPU's ids and the
-  oracle's fp64 weights: 1e-5 (fp32) / 2e-2 (bf16) of the rms.  A bf16
-  output is allowed its own final rounding (half an ulp) on top of the 2e-2:
-  the exactly rounded oracle would already score ~2e-2 on the plain
-  max |err| / rms at these sizes.  The same workloads with an fp32 output
-  meet 2e-2 with no allowance at all.
+* dispatch: identical to the oracle's stable sort of the GPU's ids, and
+  x_packed byte-identical to x gathered by packed_tok;
+* experts, at full size: EVERY row of h and of y_packed (and of the shared
+  expert's h_s / y_s) against the oracle's experts() fed the GPU's own
+  x_packed, offsets and packed_w: y_packed (fp32) within 2e-2 of the rms,
+  h (bf16) within 2e-2 beyond its own final rounding;
+* output, at full size: every token of the merged output, against the
+  oracle's merge of its own expert outputs: the fp32 merge within 2e-2 of the
+  rms, the bf16 output within 2e-2 beyond its final rounding (the plain
+  max |err| / rms of the bf16 output is recorded beside it); and a sample
+  of tokens against the oracle's direct per-token form with its own fp64
+  routing weights.
+
+Set MOE_PARITY_REPORT to a file name to append one JSON line of error
+figures per workload to it.
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -76,22 +86,69 @@ FULL = ["builder_bf16", "qwen15_t32", "qwen15_t8192", "qwen3_t16384", "decode_t1
         "decode_t64"]
 
 
+def _report(rec):
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_sampled(name):
+def test_full_size_workload(name):
     cfg = CONFIGS[name]
     p = make_layer(cfg, seed=0)
     buf, out = _forward(cfg, p)
     l64, ids = _check_route_and_dispatch(cfg, p, buf)
+    rec = {"workload": name}
+    # x_packed: byte-identical rows of x in the dispatch order
+    packed_tok = buf.packed_tok.cpu()
+    x_packed = buf.x_packed.cpu()
+    assert torch.equal(x_packed.view(torch.int16), p["x"][packed_tok.long()].view(torch.int16))
+    # every row of both expert passes, fed the GPU's own packed inputs
+    offsets = buf.offsets.cpu().numpy()
+    h_o, y_o = O.experts(x_packed, offsets, buf.packed_w.cpu(), p["w13"], p["w2"])
+    del x_packed
+    rec["h_err"] = err_bf16_out(buf.h.cpu(), h_o)
+    rec["h_err_plain"] = rel(buf.h.cpu(), h_o)
+    del h_o
+    rec["y_packed_err"] = rel(buf.y_packed.cpu(), y_o)
+    assert rec["h_err"] <= TOL["bf16"], rec
+    assert rec["y_packed_err"] <= TOL["bf16"], rec
+    shared = sg = None
+    if cfg.shared_I:
+        hs_o, shared = O.experts(p["x"], np.array([0, cfg.T]), None, p["w13s"].unsqueeze(0),
+                                 p["w2s"].unsqueeze(0))
+        sg = O.shared_gate_logit(p["x"], p["w_sg"])
+        rec["shared_h_err"] = err_bf16_out(buf.sh_h.cpu(), hs_o)
+        rec["shared_y_err"] = rel(buf.sh_y.cpu(), shared)
+        rec["shared_gate_logit_err"] = rel(buf.sg_logit.cpu().reshape(-1), sg)
+        assert rec["shared_h_err"] <= TOL["bf16"], rec
+        assert rec["shared_y_err"] <= TOL["bf16"], rec
+        assert rec["shared_gate_logit_err"] <= 1e-5, rec
+        del hs_o
+    # every token of the merged output
+    want = O.combine(y_o, buf.inv_perm.cpu().numpy(), cfg.T, cfg.k, shared, sg)
+    del y_o
+    rec["out32_err"] = rel(buf.out32, want)
+    rec["out_bf16_err"] = err_bf16_out(out, want)
+    rec["out_bf16_err_plain"] = rel(out, want)
+    # the exactly rounded oracle output, for scale: what the bf16 store alone costs
+    rec["oracle_rounded_err_plain"] = rel(torch.tensor(want).float().to(torch.bfloat16), want)
+    assert rec["out32_err"] <= TOL["bf16"], rec
+    assert rec["out_bf16_err"] <= TOL["bf16"], rec
+    # a sample of tokens against the direct per-token form with fp64 weights
     rng = np.random.default_rng(0)
     n = min(cfg.T, 24)
     toks = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, size=n, replace=False)]))
     w64 = O.routing_weights(l64[toks], ids[toks], cfg.renormalize)
-    want = O.moe_forward_tokens(p, toks, ids[toks], w64)
+    direct = O.moe_forward_tokens(p, toks, ids[toks], w64)
     sel = torch.as_tensor(toks)
-    assert err_bf16_out(out[sel], want) <= TOL["bf16"]
-    assert rel(buf.out32[sel], want) <= TOL["bf16"]
+    rec["direct_sample_err"] = rel(buf.out32[sel], direct)
+    assert err_bf16_out(out[sel], direct) <= TOL["bf16"]
+    assert rec["direct_sample_err"] <= TOL["bf16"], rec
     if cfg.zipf_s is not None:
         counts = buf.counts.cpu().numpy()
         assert counts.max() > 4 * max(1, np.median(counts))       # skewed load
         if cfg.empty_tail:
             assert (counts == 0).sum() >= cfg.empty_tail
+    _report(rec)

@@ -6,9 +6,11 @@ framework's allocator, a serving loop that allocates nothing once running).
 For them the library offers moe_dispatch_noalloc, which keeps its count table
 in a fixed array inside the library instead of a caller workspace.  These
 tests call it through the C ABI and require its outputs to equal, bit for
-bit, those of moe_dispatch on the same inputs, on two calls in a row (the
-second call sees the first call's leftovers in the shared array).  This file
-is collected last on purpose.
+bit, those of moe_dispatch on the same inputs, on two calls in a row.  Both
+calls are large enough (more than 8192 assignments) to take the multi-block
+path whose per-block counts live in the shared array, so the second call
+runs on the first call's leftovers there.  This file is collected last on
+purpose.
 """
 import ctypes
 
@@ -66,10 +68,12 @@ def test_noalloc_dispatch_equals_the_workspace_dispatch_on_two_calls_in_a_row():
     w = torch.rand(16384, 8, device="cuda")
     x = torch.randn(16384, 256, device="cuda").to(torch.bfloat16)
     _both(ids, w, x, 128)
-    # call 2: a smaller, different problem right after, on the same shared array
-    ids = _ids(rng, 777, 3, 60)
-    w = torch.rand(777, 3, device="cuda")
-    x = torch.randn(777, 64, device="cuda")
+    # call 2: a smaller, different problem right after, on the same shared array:
+    # 5000 tokens x top-3 = 15000 assignments -> 8 count blocks x 60 experts of
+    # the array, all of which still hold call 1's block bases
+    ids = _ids(rng, 5000, 3, 60)
+    w = torch.rand(5000, 3, device="cuda")
+    x = torch.randn(5000, 64, device="cuda")
     _both(ids, w, x, 60)
 
 
