@@ -27,9 +27,10 @@
  *    never trap: a bad entry is skipped and reported.  moe_read_status()
  *    copies the word to the host.
  *  - Sizes: 1 <= T; 1 <= E <= 256; 0 <= k <= min(E, 8) (k = 0 only in
- *    moe_route, "logits only"); H, I >= 1 with H % 8 == 0 and I % 8 == 0
+ *    moe_route, "logits only"; moe_dispatch takes 1 <= k <= 8 and ids that
+ *    may repeat within a token); H, I >= 1 with H % 8 == 0 and I % 8 == 0
  *    (whole 16-byte vectors); the bf16 tensor-core expert path also needs
- *    H % 256 == 0 and I % 128 == 0, else moe_experts returns
+ *    H % 256 == 0 and I % 64 == 0, else moe_experts returns
  *    MOE_ERR_UNSUPPORTED.  Activation and weight tensors must be 16-byte
  *    aligned; index, weight and status arrays 4-byte aligned.
  */
@@ -57,7 +58,7 @@ typedef enum {
   MOE_BF16 = 1   /* activations, weights and outputs in bf16, fp32 inside  */
 } moe_dtype_t;
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped on any added entry point or signature change). */
 int moe_abi_version(void);
 
 /* Number of kernels this library has enqueued in this process so far (all
@@ -226,7 +227,7 @@ int moe_experts(const void* x_packed, const int32_t* offsets, const float* packe
  *
  *   x    device [T,H] bf16          w13s device [2*I_s,H]   w2s device [H,I_s]
  *   h_s  device [T,I_s] bf16, written   y_s device [T,H] fp32, written
- *   I_s % 128 == 0; all other arguments, results and rules as moe_experts.
+ *   I_s % 64 == 0; all other arguments, results and rules as moe_experts.
  */
 int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float* packed_w,
                        const void* w13, const void* w2, int N, int H, int I, int E,
@@ -256,6 +257,129 @@ int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float
 int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,
                 const float* shared, const float* shared_gate_logit, int dtype,
                 void* out, int32_t* status, void* stream);
+
+/*
+ * ---- Expert and tensor parallelism: the pieces a rank runs --------------
+ *
+ * metrale ep_dispatch.rs (module doc): the served expert-parallel MoE is
+ * "masked-local plus all-reduce".  A rank that owns experts [s, e) of E runs
+ * the full router and dispatcher on its tokens, then
+ *   moe_gather(..., s, e, ...)          rows of its experts only,
+ *   moe_experts(x_packed, offsets + s, packed_w, w13_local, w2_local, N, H,
+ *               I, e - s, ...)          its experts (offsets hold absolute
+ *                                       packed rows, so the rank's slice of
+ *                                       offsets is a valid table for them),
+ *   moe_combine_range(..., s, e, ..., MOE_F32, partial)
+ *                                       its share of every token's sum,
+ * the caller adds the ranks' fp32 partials (an all-reduce), and
+ * moe_finalize rounds the sum once.  Tensor parallelism (diffulex.moe.layer,
+ * TPFusedMoE; the modelexpress refit test's INTER_PER_TP slices, "w1 low, w3
+ * high") is the same with every expert present on every rank but its I
+ * split: rank r holds rows [r*I/tp, (r+1)*I/tp) of each half of w13 as one
+ * [E, 2*I/tp, H] buffer and the same columns of w2 as [E, H, I/tp]; its
+ * moe_experts (with I/tp) and moe_combine (fp32 out) give a partial that the
+ * all-reduce and moe_finalize complete.
+ */
+
+/*
+ * moe_gather -- the Executor's "gather token activations for scheduled
+ * expert ranges" (DWDP README, "Executor Module") for the experts
+ * [expert_start, expert_end) alone:
+ *   x_packed[p,:] = x[packed_tok[p],:]  for p in [offsets[expert_start],
+ *                                              offsets[expert_end])
+ * Other rows of x_packed are left untouched.  moe_dispatch with x == NULL
+ * followed by moe_gather over [0, E) is moe_dispatch with x.
+ *
+ *   x          device [T,H] (dtype)        packed_tok device [N] int32 and
+ *   offsets    device [E+1] int32, as moe_dispatch writes them (trusted:
+ *              rows and tokens in range)
+ *   0 <= expert_start <= expert_end <= E;  N = rows of x_packed (T*k)
+ *   x_packed   device [N,H] (dtype), written in the range only
+ */
+int moe_gather(const void* x, const int32_t* packed_tok, const int32_t* offsets, int E,
+               int expert_start, int expert_end, int N, int H, int dtype, void* x_packed,
+               int32_t* status, void* stream);
+
+/*
+ * moe_combine_range -- masked-local Merger: moe_combine restricted to the
+ * rows of experts [expert_start, expert_end) (packed rows [offsets[s],
+ * offsets[e])); a token's other assignments contribute nothing:
+ *   out[t,:] = sum_{j<k, s <= id(t,j) < e} y_packed[inv_perm[t*k+j],:]
+ *              (j in order, fp32)  + sigmoid(gate[t]) * shared[t,:] if given
+ * Written as `dtype` (MOE_F32 for a partial that an all-reduce will add).
+ * Arguments and errors as moe_combine, plus offsets (device [E+1] int32)
+ * and 0 <= expert_start <= expert_end <= E.
+ */
+int moe_combine_range(const float* y_packed, const int32_t* inv_perm, const int32_t* offsets,
+                      int E, int expert_start, int expert_end, int T, int H, int k,
+                      const float* shared, const float* shared_gate_logit, int dtype, void* out,
+                      int32_t* status, void* stream);
+
+/*
+ * moe_finalize -- the one rounding after the ranks' partial outputs were
+ * added: out[t,h] = acc[t,h] rounded to `dtype` (bf16: round to nearest
+ * even; fp32: a copy).  acc device [T,H] fp32, out device [T,H] (dtype);
+ * both 16-byte aligned, H % 8 == 0.
+ */
+int moe_finalize(const float* acc, int T, int H, int dtype, void* out, void* stream);
+
+/* Bytes of device scratch moe_ep_partition needs (0 for num_tokens * top_k
+ * <= 2048, when one block does all the work). */
+size_t moe_ep_partition_workspace_bytes(int num_tokens, int top_k);
+
+/*
+ * moe_ep_partition -- metrale ep_dispatch.rs, "EpRoutingTable" /
+ * "build_ep_routing_table", on the device: the row-major [num_tokens, top_k]
+ * assignments split into a local bucket (expert id in [local_expert_start,
+ * local_expert_end)) and a remote bucket (every other id).  Entry i of a
+ * bucket is the triple (*_token_indices[i], *_expert_ids[i], *_weights[i])
+ * of one assignment; both buckets keep the order the assignments were given
+ * (flat index token * top_k + j ascending).  Expert ids are global (not
+ * rank-relative) and compared as unsigned 32-bit values, like the page's
+ * u32 ids.
+ *
+ *   gate_indices device [n_indices] int32, gate_weights device [n_weights] f32
+ *   n_indices / n_weights must both equal num_tokens * top_k: otherwise
+ *       MOE_ERR_INVALID_ARG with the message "gate_indices length mismatch" /
+ *       "gate_weights length mismatch" (where the page's function panics)
+ *   local_* and remote_* device arrays of num_tokens * top_k entries each
+ *       (the caller cannot know the split in advance); bucket i is written
+ *       in entries [0, bucket_counts[i])
+ *   bucket_counts device int32[2]: local count, remote count (they add up
+ *       to num_tokens * top_k, the table's total_count)
+ *   ws / ws_bytes: device scratch of moe_ep_partition_workspace_bytes()
+ *   num_tokens >= 0, top_k >= 1, 0 <= local_expert_start <= local_expert_end
+ */
+int moe_ep_partition(const int32_t* gate_indices, size_t n_indices, const float* gate_weights,
+                     size_t n_weights, int num_tokens, int top_k, int local_expert_start,
+                     int local_expert_end, int32_t* local_token_indices,
+                     int32_t* local_expert_ids, float* local_weights,
+                     int32_t* remote_token_indices, int32_t* remote_expert_ids,
+                     float* remote_weights, int32_t* bucket_counts, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * All-to-all dispatcher (diffulex.moe API reference, "diffulex.moe.dispatcher":
+ * NaiveA2ADispatcher / TokenDispatcher move tokens between ranks for expert
+ * execution).  With the E experts split over `world` ranks in contiguous
+ * ranges (rank q owns [floor(E*q/world), floor(E*(q+1)/world))):
+ *
+ * moe_ep_owner -- owner[f] = the rank owning expert ids[f], f < n.  An id
+ * outside [0, E) gives owner -1 and sets MOE_ERR_BAD_INDEX in `status`
+ * (device int32 or NULL).  ids, owner: device int32 [n].
+ * Dispatching the [T,k] owner table with moe_dispatch (E = world) groups a
+ * rank's assignments by destination, in assignment order inside each group.
+ *
+ * moe_ep_pack_ids -- for the rows p < offsets[world] of that dispatch:
+ *   local_ids[p] = ids[perm[p]] - (first expert of its owner),
+ * the expert id the receiving rank uses for its own [0, E_local) experts.
+ * ids device [n] int32 (the routed expert ids), perm / offsets the owner
+ * dispatch's outputs (device [n] / [world+1] int32), local_ids device [n].
+ */
+int moe_ep_owner(const int32_t* ids, int n, int E, int world, int32_t* owner, int32_t* status,
+                 void* stream);
+int moe_ep_pack_ids(const int32_t* ids, const int32_t* perm, const int32_t* offsets, int n,
+                    int E, int world, int32_t* local_ids, void* stream);
 
 /* Copy the device status word to *host_status after the stream's prior work
  * (synchronises `stream`).  Returns MOE_OK or MOE_ERR_CUDA. */

@@ -27,7 +27,8 @@ __all__ = [
     "moe_experts", "moe_experts_shared", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
-    "moe_layer_forward_host",
+    "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
+    "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
@@ -66,6 +67,14 @@ _SIGS = {
     "moe_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_read_status": (_I, [_P, _P, _P]),
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
+    "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_combine_range": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
+    "moe_finalize": (_I, [_P, _I, _I, _I, _P, _P]),
+    "moe_ep_partition_workspace_bytes": (_SZ, [_I, _I]),
+    "moe_ep_owner": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "moe_ep_pack_ids": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
+    "moe_ep_partition": (_I, [_P, _SZ, _P, _SZ, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                              _SZ, _P]),
 }
 
 
@@ -201,6 +210,64 @@ def moe_combine(y_packed, inv_perm, T: int, k: int, out, shared=None, shared_gat
         _dtype_code(out), _ptr(out), _ptr(status), _stream(stream)))
 
 
+def moe_gather(x, packed_tok, offsets, expert_start: int, expert_end: int, x_packed,
+               status=None, stream=None):
+    """x_packed rows of the experts [expert_start, expert_end) only."""
+    N, H = x_packed.shape
+    E = offsets.shape[0] - 1
+    _check(load_library().moe_gather(
+        _ptr(x), _ptr(packed_tok), _ptr(offsets), E, expert_start, expert_end, N, H,
+        _dtype_code(x), _ptr(x_packed), _ptr(status), _stream(stream)))
+
+
+def moe_combine_range(y_packed, inv_perm, offsets, expert_start: int, expert_end: int, T: int,
+                      k: int, out, shared=None, shared_gate_logit=None, status=None,
+                      stream=None):
+    """Masked-local merge: only the rows of experts [expert_start, expert_end)."""
+    H = out.shape[1]
+    E = offsets.shape[0] - 1
+    _check(load_library().moe_combine_range(
+        _ptr(y_packed), _ptr(inv_perm), _ptr(offsets), E, expert_start, expert_end, T, H, k,
+        _ptr(shared), _ptr(shared_gate_logit), _dtype_code(out), _ptr(out), _ptr(status),
+        _stream(stream)))
+
+
+def moe_finalize(acc, out, stream=None):
+    """out = acc (fp32 [T,H]) rounded once to out's dtype."""
+    T, H = out.shape
+    _check(load_library().moe_finalize(_ptr(acc), T, H, _dtype_code(out), _ptr(out),
+                                       _stream(stream)))
+
+
+def moe_ep_partition_workspace_bytes(num_tokens: int, top_k: int) -> int:
+    return load_library().moe_ep_partition_workspace_bytes(num_tokens, top_k)
+
+
+def moe_ep_partition(gate_indices, gate_weights, num_tokens: int, top_k: int,
+                     local_expert_start: int, local_expert_end: int, local_token_indices,
+                     local_expert_ids, local_weights, remote_token_indices, remote_expert_ids,
+                     remote_weights, bucket_counts, ws=None, stream=None):
+    """metrale's build_ep_routing_table on the device (see moe_b200.h)."""
+    _check(load_library().moe_ep_partition(
+        _ptr(gate_indices), gate_indices.numel(), _ptr(gate_weights), gate_weights.numel(),
+        num_tokens, top_k, local_expert_start, local_expert_end, _ptr(local_token_indices),
+        _ptr(local_expert_ids), _ptr(local_weights), _ptr(remote_token_indices),
+        _ptr(remote_expert_ids), _ptr(remote_weights), _ptr(bucket_counts), _ptr(ws),
+        ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def moe_ep_owner(ids, E: int, world: int, owner, status=None, stream=None):
+    """owner[f] = rank owning expert ids[f] (contiguous split of E over world)."""
+    _check(load_library().moe_ep_owner(_ptr(ids), ids.numel(), E, world, _ptr(owner),
+                                       _ptr(status), _stream(stream)))
+
+
+def moe_ep_pack_ids(ids, perm, offsets, E: int, world: int, local_ids, stream=None):
+    """local_ids[p] = ids[perm[p]] minus its owner's first expert (rows p < offsets[world])."""
+    _check(load_library().moe_ep_pack_ids(_ptr(ids), _ptr(perm), _ptr(offsets), ids.numel(), E,
+                                          world, _ptr(local_ids), _stream(stream)))
+
+
 def moe_read_status(status, stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(load_library().moe_read_status(_ptr(status), _stream(stream), ctypes.byref(v)))
@@ -248,7 +315,7 @@ class MoELayerBuffers:
         self.shared_I = shared_I
         # bf16 tensor-core layers run the shared expert inside the routed launches
         self.fuse_shared = bool(shared_I) and dtype == torch.bfloat16 and H % 256 == 0 and \
-            I % 128 == 0 and shared_I % 128 == 0
+            I % 64 == 0 and shared_I % 64 == 0
         if shared_I:
             self.sg_logit = torch.empty(T, 1, **f32)
             self.sh_offsets = torch.tensor([0, T], **i32)

@@ -82,7 +82,7 @@ cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream
 
 extern "C" {
 
-int moe_abi_version(void) { return 2; }
+int moe_abi_version(void) { return 3; }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -129,8 +129,7 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x, in
   REQ(!topk_w || packed_w, MOE_ERR_INVALID_ARG, "moe_dispatch: topk_w given but packed_w is null");
   REQ(T >= 1, MOE_ERR_INVALID_ARG, "moe_dispatch: T must be >= 1");
   REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_dispatch: E must be in [1, 256]");
-  REQ(k >= 1 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
-      "moe_dispatch: k must be in [1, min(E, 8)]");
+  REQ(k >= 1 && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG, "moe_dispatch: k must be in [1, 8]");
   REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG, "moe_dispatch: T*k too large");
   REQ(aligned4(topk_ids) && aligned4(topk_w) && aligned4(counts) && aligned4(offsets) &&
           aligned4(perm) && aligned4(inv_perm) && aligned4(packed_tok) && aligned4(packed_w),
@@ -185,8 +184,8 @@ int experts_impl(const char* fn, const void* x_packed, const int32_t* offsets,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == MOE_BF16) {
-    REQ(H % 256 == 0 && I % 128 == 0, MOE_ERR_UNSUPPORTED,
-        f + "the bf16 tensor-core path needs H % 256 == 0 and I % 128 == 0");
+    REQ(H % 256 == 0 && I % 64 == 0, MOE_ERR_UNSUPPORTED,
+        f + "the bf16 tensor-core path needs H % 256 == 0 and I % 64 == 0");
     const char* why = "";
     e = moe_host::launch_experts_tc(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h, y_packed,
                                     sh, ws, ws_bytes, status, s, &why);
@@ -221,7 +220,7 @@ int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float
   REQ(T >= 1 && I_s >= 1, MOE_ERR_INVALID_ARG, "moe_experts_shared: T and I_s must be >= 1");
   REQ(aligned16(x) && aligned16(w13s) && aligned16(w2s) && aligned16(h_s) && aligned16(y_s),
       MOE_ERR_INVALID_ARG, "moe_experts_shared: shared-expert tensors must be 16-byte aligned");
-  REQ(I_s % 128 == 0, MOE_ERR_UNSUPPORTED, "moe_experts_shared: I_s must be a multiple of 128");
+  REQ(I_s % 64 == 0, MOE_ERR_UNSUPPORTED, "moe_experts_shared: I_s must be a multiple of 64");
   REQ(static_cast<long long>(T) * (H > I_s ? H : I_s) < (1ll << 40) && T < (1 << 30),
       MOE_ERR_INVALID_ARG, "moe_experts_shared: T too large");
   const moe_host::SharedGroup sh{x, T, w13s, w2s, I_s, h_s, y_s};
@@ -246,6 +245,138 @@ int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, in
   cudaError_t e = moe_host::launch_combine(y_packed, inv_perm, T, H, k, shared, shared_gate_logit,
                                            dtype, out, status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
+}
+
+int moe_combine_range(const float* y_packed, const int32_t* inv_perm, const int32_t* offsets,
+                      int E, int expert_start, int expert_end, int T, int H, int k,
+                      const float* shared, const float* shared_gate_logit, int dtype, void* out,
+                      int32_t* status, void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(y_packed && inv_perm && offsets && out, MOE_ERR_INVALID_ARG,
+      "moe_combine_range: null y_packed, inv_perm, offsets or out");
+  REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_combine_range: T and H must be >= 1");
+  REQ(k >= 1 && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG, "moe_combine_range: k must be in [1, 8]");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_combine_range: E must be in [1, 256]");
+  REQ(expert_start >= 0 && expert_start <= expert_end && expert_end <= E, MOE_ERR_INVALID_ARG,
+      "moe_combine_range: need 0 <= expert_start <= expert_end <= E");
+  REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_combine_range: H must be a multiple of 8");
+  REQ(aligned16(y_packed) && aligned16(out) && aligned16(shared), MOE_ERR_INVALID_ARG,
+      "moe_combine_range: y_packed, shared and out must be 16-byte aligned");
+  REQ(aligned4(inv_perm) && aligned4(offsets) && aligned4(shared_gate_logit) && aligned4(status),
+      MOE_ERR_INVALID_ARG, "moe_combine_range: index / gate / status arrays must be 4-byte aligned");
+  REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG,
+      "moe_combine_range: T*k too large");
+  cudaError_t e = moe_host::launch_combine(y_packed, inv_perm, T, H, k, shared, shared_gate_logit,
+                                           dtype, out, status, static_cast<cudaStream_t>(stream),
+                                           offsets, expert_start, expert_end);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine_range launch");
+}
+
+int moe_finalize(const float* acc, int T, int H, int dtype, void* out, void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(acc && out, MOE_ERR_INVALID_ARG, "moe_finalize: null acc or out");
+  REQ(T >= 1 && H >= 1 && H % 8 == 0, MOE_ERR_INVALID_ARG,
+      "moe_finalize: need T >= 1 and H a positive multiple of 8");
+  REQ(aligned16(acc) && aligned16(out), MOE_ERR_INVALID_ARG,
+      "moe_finalize: acc and out must be 16-byte aligned");
+  cudaError_t e = moe_host::launch_finalize(acc, T, H, dtype, out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_finalize launch");
+}
+
+int moe_gather(const void* x, const int32_t* packed_tok, const int32_t* offsets, int E,
+               int expert_start, int expert_end, int N, int H, int dtype, void* x_packed,
+               int32_t* status, void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  REQ(x && packed_tok && offsets && x_packed, MOE_ERR_INVALID_ARG,
+      "moe_gather: null x, packed_tok, offsets or x_packed");
+  REQ(N >= 1 && H >= 1 && H % 8 == 0, MOE_ERR_INVALID_ARG,
+      "moe_gather: need N >= 1 and H a positive multiple of 8");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_gather: E must be in [1, 256]");
+  REQ(expert_start >= 0 && expert_start <= expert_end && expert_end <= E, MOE_ERR_INVALID_ARG,
+      "moe_gather: need 0 <= expert_start <= expert_end <= E");
+  REQ(aligned16(x) && aligned16(x_packed), MOE_ERR_INVALID_ARG,
+      "moe_gather: x and x_packed must be 16-byte aligned");
+  REQ(aligned4(packed_tok) && aligned4(offsets) && aligned4(status), MOE_ERR_INVALID_ARG,
+      "moe_gather: index and status arrays must be 4-byte aligned");
+  REQ(N < (1 << 30) && static_cast<long long>(N) * H < (1ll << 40), MOE_ERR_INVALID_ARG,
+      "moe_gather: N too large");
+  cudaError_t e = moe_host::launch_gather(x, packed_tok, offsets, expert_start, expert_end, N, H,
+                                          dtype, x_packed, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_gather launch");
+}
+
+size_t moe_ep_partition_workspace_bytes(int num_tokens, int top_k) {
+  if (num_tokens < 0 || top_k < 1) return 0;
+  return moe_host::ep_partition_ws_bytes(static_cast<long long>(num_tokens) * top_k);
+}
+
+int moe_ep_partition(const int32_t* gate_indices, size_t n_indices, const float* gate_weights,
+                     size_t n_weights, int num_tokens, int top_k, int local_expert_start,
+                     int local_expert_end, int32_t* local_token_indices,
+                     int32_t* local_expert_ids, float* local_weights,
+                     int32_t* remote_token_indices, int32_t* remote_expert_ids,
+                     float* remote_weights, int32_t* bucket_counts, void* ws, size_t ws_bytes,
+                     void* stream) {
+  g_err.clear();
+  REQ(num_tokens >= 0 && top_k >= 1, MOE_ERR_INVALID_ARG,
+      "moe_ep_partition: need num_tokens >= 0 and top_k >= 1");
+  const long long total = static_cast<long long>(num_tokens) * top_k;
+  REQ(total < (1ll << 31), MOE_ERR_INVALID_ARG, "moe_ep_partition: num_tokens*top_k too large");
+  // The page's build_ep_routing_table panics on these two; here they are errors.
+  REQ(static_cast<long long>(n_indices) == total, MOE_ERR_INVALID_ARG,
+      "gate_indices length mismatch");
+  REQ(static_cast<long long>(n_weights) == total, MOE_ERR_INVALID_ARG,
+      "gate_weights length mismatch");
+  REQ(local_expert_start >= 0 && local_expert_start <= local_expert_end, MOE_ERR_INVALID_ARG,
+      "moe_ep_partition: need 0 <= local_expert_start <= local_expert_end");
+  REQ(bucket_counts != nullptr, MOE_ERR_INVALID_ARG, "moe_ep_partition: null bucket_counts");
+  REQ(total == 0 || (gate_indices && gate_weights && local_token_indices && local_expert_ids &&
+                     local_weights && remote_token_indices && remote_expert_ids && remote_weights),
+      MOE_ERR_INVALID_ARG, "moe_ep_partition: null input or bucket array");
+  REQ(aligned4(gate_indices) && aligned4(gate_weights) && aligned4(local_token_indices) &&
+          aligned4(local_expert_ids) && aligned4(local_weights) &&
+          aligned4(remote_token_indices) && aligned4(remote_expert_ids) &&
+          aligned4(remote_weights) && aligned4(bucket_counts),
+      MOE_ERR_INVALID_ARG, "moe_ep_partition: arrays must be 4-byte aligned");
+  const size_t need = moe_host::ep_partition_ws_bytes(total);
+  REQ(total <= 2048 || (ws && ws_bytes >= need && aligned4(ws)), MOE_ERR_INVALID_ARG,
+      "moe_ep_partition: workspace missing or smaller than moe_ep_partition_workspace_bytes()");
+  cudaError_t e = moe_host::launch_ep_partition(
+      gate_indices, gate_weights, static_cast<int>(total), top_k,
+      static_cast<unsigned>(local_expert_start), static_cast<unsigned>(local_expert_end),
+      local_token_indices, local_expert_ids, local_weights, remote_token_indices,
+      remote_expert_ids, remote_weights, bucket_counts, ws, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_partition launch");
+}
+
+int moe_ep_owner(const int32_t* ids, int n, int E, int world, int32_t* owner, int32_t* status,
+                 void* stream) {
+  g_err.clear();
+  REQ(ids && owner, MOE_ERR_INVALID_ARG, "moe_ep_owner: null ids or owner");
+  REQ(n >= 1 && E >= 1 && world >= 1 && world <= E, MOE_ERR_INVALID_ARG,
+      "moe_ep_owner: need n >= 1 and 1 <= world <= E");
+  REQ(aligned4(ids) && aligned4(owner) && aligned4(status), MOE_ERR_INVALID_ARG,
+      "moe_ep_owner: arrays must be 4-byte aligned");
+  cudaError_t e = moe_host::launch_ep_owner(ids, n, E, world, owner, status,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_owner launch");
+}
+
+int moe_ep_pack_ids(const int32_t* ids, const int32_t* perm, const int32_t* offsets, int n,
+                    int E, int world, int32_t* local_ids, void* stream) {
+  g_err.clear();
+  REQ(ids && perm && offsets && local_ids, MOE_ERR_INVALID_ARG,
+      "moe_ep_pack_ids: null ids, perm, offsets or local_ids");
+  REQ(n >= 1 && E >= 1 && world >= 1 && world <= E, MOE_ERR_INVALID_ARG,
+      "moe_ep_pack_ids: need n >= 1 and 1 <= world <= E");
+  REQ(aligned4(ids) && aligned4(perm) && aligned4(offsets) && aligned4(local_ids),
+      MOE_ERR_INVALID_ARG, "moe_ep_pack_ids: arrays must be 4-byte aligned");
+  cudaError_t e = moe_host::launch_ep_pack_ids(ids, perm, offsets, n, E, world, local_ids,
+                                               static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_ep_pack_ids launch");
 }
 
 int moe_read_status(const int32_t* status, void* stream, int32_t* host_status) {

@@ -15,6 +15,13 @@
 // 16-byte vectors of the hidden dimension, so every load and store is a
 // 128-bit access.  The k source rows of a token are independent loads that
 // are all in flight together.
+//
+// Masked-local merge (expert parallelism, metrale ep_dispatch.rs: "the served
+// EP MoE is masked-local plus all-reduce"): with an expert range, only rows
+// of the experts [lo_e, hi_e) -- packed rows [offsets[lo_e], offsets[hi_e)) --
+// are added; a rank's other assignments belong to other ranks' experts.  The
+// partial sums of all ranks are then added across ranks and rounded once by
+// moe_finalize.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,11 +36,18 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
                                                       int T, int H, int k, int N,
                                                       const float* __restrict__ shared,
                                                       const float* __restrict__ sgate,
+                                                      const int32_t* __restrict__ range_offs,
+                                                      int lo_e, int hi_e,
                                                       void* __restrict__ outv, int32_t* status) {
   const int nvec = H / 8;                               // 8 outputs per thread step
   __shared__ int rows[moe::kMaxTopK];
   __shared__ float gate;
   moe::grid_dep_wait();
+  int rlo = 0, rhi = N;                                 // rows that contribute
+  if (range_offs != nullptr) {
+    rlo = range_offs[lo_e];
+    rhi = range_offs[hi_e];
+  }
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < k) {
@@ -41,6 +55,8 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
       if (p < 0 || p >= N) {
         moe::report(status, MOE_ERR_BAD_INDEX);
         p = -1;
+      } else if (p < rlo || p >= rhi) {
+        p = -1;                                         // another rank's expert
       }
       rows[threadIdx.x] = p;
     }
@@ -91,13 +107,46 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
   moe::grid_dep_launch();
 }
 
+// out = acc rounded once to the output type (bf16 or fp32 copy).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(CNT) finalize_kernel(const float4* __restrict__ acc,
+                                                       size_t nvec8, void* __restrict__ outv) {
+  moe::grid_dep_wait();
+  for (size_t v = blockIdx.x * static_cast<size_t>(CNT) + threadIdx.x; v < nvec8;
+       v += static_cast<size_t>(gridDim.x) * CNT) {
+    const float4 a = acc[2 * v], b = acc[2 * v + 1];
+    if (OUT_BF16) {
+      reinterpret_cast<uint4*>(outv)[v] =
+          make_uint4(moe::pack_bf16x2(a.x, a.y), moe::pack_bf16x2(a.z, a.w),
+                     moe::pack_bf16x2(b.x, b.y), moe::pack_bf16x2(b.z, b.w));
+    } else {
+      float4* d = reinterpret_cast<float4*>(outv) + 2 * v;
+      d[0] = a;
+      d[1] = b;
+    }
+  }
+  moe::grid_dep_launch();
+}
+
 }  // namespace
 
 namespace moe_host {
 
+cudaError_t launch_finalize(const float* acc, int T, int H, int dtype, void* out,
+                            cudaStream_t s) {
+  const size_t nvec8 = static_cast<size_t>(T) * H / 8;
+  const int grid = static_cast<int>(std::max<size_t>(
+      1, std::min<size_t>((nvec8 + CNT - 1) / CNT, static_cast<size_t>(num_sms()) * 8)));
+  const float4* a = reinterpret_cast<const float4*>(acc);
+  return dtype == MOE_BF16
+             ? launch_pdl(finalize_kernel<true>, dim3(grid), dim3(CNT), 0, s, 0, a, nvec8, out)
+             : launch_pdl(finalize_kernel<false>, dim3(grid), dim3(CNT), 0, s, 0, a, nvec8, out);
+}
+
 cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
                            const float* shared, const float* shared_gate, int dtype, void* out,
-                           int32_t* status, cudaStream_t s) {
+                           int32_t* status, cudaStream_t s, const int32_t* range_offs, int lo_e,
+                           int hi_e) {
   const int grid = std::max(1, std::min(T, num_sms() * 8));
   const int N = T * k;
   // k is a template parameter so that exactly k rows are loaded, all in flight.
@@ -105,9 +154,9 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
   case KV:                                                                                    \
     return dtype == MOE_BF16                                                                  \
                ? launch_pdl(combine_kernel<true, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,       \
-                            inv_perm, T, H, k, N, shared, shared_gate, out, status)           \
+                            inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out, status)           \
                : launch_pdl(combine_kernel<false, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,      \
-                            inv_perm, T, H, k, N, shared, shared_gate, out, status);
+                            inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out, status);
   switch (k) {
     MOE_COMBINE_K(1)
     MOE_COMBINE_K(2)

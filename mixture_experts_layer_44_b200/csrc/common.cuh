@@ -111,9 +111,26 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
 cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
                                 const float* packed_w, const void* w13, const void* w2, int N,
                                 int H, int I, int E, void* h, void* y, cudaStream_t s);
+// range_offs != NULL: only packed rows [range_offs[lo_e], range_offs[hi_e]) are added.
 cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
                            const float* shared, const float* shared_gate, int dtype, void* out,
-                           int32_t* status, cudaStream_t s);
+                           int32_t* status, cudaStream_t s, const int32_t* range_offs = nullptr,
+                           int lo_e = 0, int hi_e = 0);
+cudaError_t launch_finalize(const float* acc, int T, int H, int dtype, void* out,
+                            cudaStream_t s);
+// Rows [offsets[lo_e], offsets[hi_e]) of x_packed gathered from x by packed_tok.
+cudaError_t launch_gather(const void* x, const int32_t* packed_tok, const int32_t* offsets,
+                          int lo_e, int hi_e, int N, int H, int dtype, void* x_packed,
+                          int32_t* status, cudaStream_t s);
+size_t ep_partition_ws_bytes(long long n);
+cudaError_t launch_ep_partition(const int32_t* ids, const float* w, int n, int top_k,
+                                unsigned lo, unsigned hi, int32_t* l_tok, int32_t* l_eid,
+                                float* l_w, int32_t* r_tok, int32_t* r_eid, float* r_w,
+                                int32_t* bucket_counts, void* ws, cudaStream_t s);
+cudaError_t launch_ep_owner(const int32_t* ids, int n, int E, int R, int32_t* owner,
+                            int32_t* status, cudaStream_t s);
+cudaError_t launch_ep_pack_ids(const int32_t* ids, const int32_t* perm, const int32_t* offsets,
+                               int n, int E, int R, int32_t* local, cudaStream_t s);
 cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream_t s);
 int num_sms();
 void set_last_error(const std::string& msg);   // the message moe_last_error() returns

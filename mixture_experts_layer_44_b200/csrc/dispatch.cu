@@ -283,10 +283,12 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
 constexpr int GW = 4;      // warps per CTA, each an independent copy engine client
 constexpr int GSLOTS = 4;  // rows in flight per warp
 
+// Rows [offsets[lo_e], offsets[hi_e]) of x_packed: every valid row for the
+// dispatcher (lo_e = 0, hi_e = E), one rank's experts for an expert range.
 __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
     const uint8_t* __restrict__ x, const int32_t* __restrict__ packed_tok,
-    const int32_t* __restrict__ offsets, int E, int row_bytes, uint8_t* __restrict__ xp,
-    int32_t* status) {
+    const int32_t* __restrict__ offsets, int lo_e, int hi_e, int row_bytes,
+    uint8_t* __restrict__ xp, int32_t* status) {
   extern __shared__ __align__(128) uint8_t gsm[];
   __shared__ __align__(8) uint64_t bars[GW][GSLOTS];
   const int warp = threadIdx.x >> 5;
@@ -296,12 +298,13 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
   moe::fence_barrier_init();
   moe::grid_dep_wait();
 
-  const int nrows = offsets[E];            // valid rows (assignments with a valid id)
+  const int row0 = offsets[lo_e];
+  const int nrows = offsets[hi_e] - row0;  // valid rows (assignments with a valid id)
   const int stride = gridDim.x * GW;
   const int first = blockIdx.x * GW + warp;
   const int mine = first < nrows ? (nrows - first + stride - 1) / stride : 0;
   auto issue = [&](int i) {
-    const int p = first + i * stride;
+    const int p = row0 + first + i * stride;
     const int s = i % GSLOTS;
     const uint32_t bar = moe::smem_addr(&bars[warp][s]);
     moe::mbar_arrive_expect_tx(bar, row_bytes);
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
   for (int i = 0; i < prologue; ++i) issue(i);
   for (int i = 0; i < mine; ++i) {
     const int s = i % GSLOTS;
-    const int p = first + i * stride;
+    const int p = row0 + first + i * stride;
     if (!moe::mbar_wait(moe::smem_addr(&bars[warp][s]), (i / GSLOTS) & 1)) {
       moe::report(status, MOE_ERR_TIMEOUT);
       // Let every load already issued land before the CTA leaves.
@@ -336,11 +339,12 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
 // Rows too large for the shared-memory ring: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ packed_tok,
-    const int32_t* __restrict__ offsets, int E, int row_vecs, uint4* __restrict__ xp) {
+    const int32_t* __restrict__ offsets, int lo_e, int hi_e, int row_vecs,
+    uint4* __restrict__ xp) {
   moe::grid_dep_wait();
-  const int nrows = offsets[E];
+  const int row_end = offsets[hi_e];
   const int lane = threadIdx.x & 31;
-  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < nrows;
+  for (int p = offsets[lo_e] + ((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < row_end;
        p += (gridDim.x * blockDim.x) >> 5) {
     const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
@@ -411,22 +415,28 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
                        w ? packed_w : nullptr, status);
     if (err != cudaSuccess || x == nullptr) return err;
   }
-  cudaError_t err;
+  return launch_gather(x, packed_tok, offsets, 0, E, N, H, dtype, x_packed, status, s);
+}
+
+cudaError_t launch_gather(const void* x, const int32_t* packed_tok, const int32_t* offsets,
+                          int lo_e, int hi_e, int N, int H, int dtype, void* x_packed,
+                          int32_t* status, cudaStream_t s) {
+  const int es = dtype == MOE_BF16 ? 2 : 4;
+  const int row_bytes = H * es;
   const size_t gsm = static_cast<size_t>(GW) * GSLOTS * row_bytes;
   if (gsm > 200 * 1024) {
     const int grid = std::max(1, std::min((N + 7) / 8, num_sms() * 8));
     return launch_pdl(dispatch_gather_vec_kernel, dim3(grid), dim3(256), 0, s, 0,
-                      static_cast<const uint4*>(x), static_cast<const int32_t*>(packed_tok),
-                      static_cast<const int32_t*>(offsets), E, row_bytes / 16,
-                      static_cast<uint4*>(x_packed));
+                      static_cast<const uint4*>(x), packed_tok, offsets, lo_e, hi_e,
+                      row_bytes / 16, static_cast<uint4*>(x_packed));
   }
-  err = ensure_smem(reinterpret_cast<const void*>(dispatch_gather_kernel), static_cast<int>(gsm));
+  cudaError_t err =
+      ensure_smem(reinterpret_cast<const void*>(dispatch_gather_kernel), static_cast<int>(gsm));
   if (err != cudaSuccess) return err;
   const int ctas_per_sm = std::max(1, static_cast<int>((200 * 1024) / gsm));
   const int grid = std::max(1, std::min((N + GW - 1) / GW, num_sms() * ctas_per_sm));
   return launch_pdl(dispatch_gather_kernel, dim3(grid), dim3(GW * 32), gsm, s, 0,
-                    static_cast<const uint8_t*>(x), static_cast<const int32_t*>(packed_tok),
-                    static_cast<const int32_t*>(offsets), E, row_bytes,
+                    static_cast<const uint8_t*>(x), packed_tok, offsets, lo_e, hi_e, row_bytes,
                     static_cast<uint8_t*>(x_packed), status);
 }
 

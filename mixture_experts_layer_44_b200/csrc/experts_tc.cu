@@ -18,7 +18,9 @@
 // (MMA N) x K.  In pass 1 the 256 weight rows are 128 gate rows and the 128
 // matching up rows (one 3-D TMA box over [2E, I, H]), so column c and column
 // 128 + c of the accumulator are the gate and up value of the same feature
-// and the SwiGLU is thread-local.  The tile list is derived on the device from
+// and the SwiGLU is thread-local.  I is a multiple of 64: when it is not one
+// of 128, the last feature tile reaches 64 rows past I, which the box reads
+// as zeros and the epilogue does not store.  The tile list is derived on the device from
 // `offsets` (the scheduler of the README's "Scheduler Module", folded into
 // the kernel): expert e owns ceil(count_e / 128) token tiles x (rows / 256)
 // weight tiles, token tiles fastest, so CTAs running at the same time share a
@@ -549,6 +551,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(buf * BN);
       const int nvalid = rows_valid < BM ? rows_valid : BM;
+      // h columns of this feature tile that exist (pass 1: 64 or 128)
+      const int ncol = min(BN / 2, uldo - un.nt * (BN / 2));
       const bool staged = nvalid > STAGE_MIN_ROWS;    // same for all four epilogue warps
       const size_t row0 = static_cast<size_t>(un.row0);
       const int S = un.S;
@@ -558,7 +562,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __nv_bfloat16* dst =
               static_cast<__nv_bfloat16*>(uout) + grow * uldo + un.nt * (BN / 2);
 #pragma unroll 1
-          for (int cc = 0; cc < BN / 2; cc += 16) {
+          for (int cc = 0; cc < ncol; cc += 16) {
             uint32_t g[16], v[16];
             moe::tmem_ld16(taddr + cc, g);
             moe::tmem_ld16(taddr + BN / 2 + cc, v);
@@ -580,7 +584,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uint8_t* gtile = static_cast<uint8_t*>(uout) +
                            (row0 * uldo + un.nt * (BN / 2)) * sizeof(__nv_bfloat16);
 #pragma unroll 1
-          for (int hc = 0; hc < BN / 2; hc += 64) {
+          for (int hc = 0; hc < ncol; hc += 64) {        // same count in all four warps
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
               const int cc = hc + half * 32;
@@ -678,7 +682,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float* base = partials + static_cast<size_t>(u - un.ks) * (BM * BN);
           if (EPI == EPI_SWIGLU) {
             const int cg = et & 31;                       // h columns 4cg .. 4cg+3
-            for (int r = et >> 5; r < nrows; r += 4) {
+            for (int r = et >> 5; r < nrows && cg * 4 < ncol; r += 4) {
               float4 g = make_float4(0.f, 0.f, 0.f, 0.f), v = g;
               const float* pr = base + static_cast<size_t>(r) * BN + cg * 4;
 #pragma unroll
@@ -813,17 +817,20 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     max_units = static_cast<int>(std::min<size_t>((ws_bytes - cbytes) / PARTIAL_BYTES, 1 << 20));
   }
   const int sms = num_sms();
+  // Feature tiles of pass 1: 128 features each, the last one possibly half full.
+  const int ntw1 = (I + BN / 2 - 1) / (BN / 2);
+  const int ntw1s = (Is + BN / 2 - 1) / (BN / 2);
   int g1 = sms, g2 = sms;
   if (counters == nullptr) {   // no split possible: never more CTAs than tiles
     const int mt_bound = (N + BM - 1) / BM + E;
     const int mt2 = (T2 + BM - 1) / BM;
-    g1 = std::max(1, std::min(sms, mt_bound * (I / (BN / 2)) + mt2 * (Is / (BN / 2))));
+    g1 = std::max(1, std::min(sms, mt_bound * ntw1 + mt2 * ntw1s));
     g2 = std::max(1, std::min(sms, (mt_bound + mt2) * (H / BN)));
   }
   const float* no_w = nullptr;
   cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS),
-                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, offsets, E, H, I / (BN / 2),
-                               2 * I, no_w, h, I, T2, H, Is / (BN / 2), sh ? sh->h : nullptr, Is,
+                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, offsets, E, H, ntw1,
+                               2 * I, no_w, h, I, T2, H, ntw1s, sh ? sh->h : nullptr, Is,
                                counters, partials, max_units, status);
   if (err != cudaSuccess) return err;
   return launch_pdl(k2, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,

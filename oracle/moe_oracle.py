@@ -30,7 +30,8 @@ __all__ = [
     "route", "route_from_logits", "dispatch", "gather_rows", "silu", "w13_halves",
     "expert_hidden", "expert_output", "experts", "combine", "shared_expert",
     "shared_gate_logit", "moe_forward", "moe_forward_tokens", "ep_partition",
-    "rel_err_rms",
+    "expert_ranges", "expert_owner", "tp_slice", "moe_forward_tokens_ep",
+    "moe_forward_tokens_tp", "rel_err_rms",
 ]
 
 
@@ -345,6 +346,97 @@ def ep_partition(gate_indices, gate_weights, num_tokens: int, top_k: int,
             b[f"{side}_expert_ids"].append(e)
             b[f"{side}_weights"].append(gate_weights[f])
     return b
+
+
+# ------------------------------------- expert / tensor parallel forms ---
+
+def expert_ranges(E: int, world: int):
+    """Contiguous expert ranges of ``world`` ranks: rank q owns
+    [floor(E*q/world), floor(E*(q+1)/world)) -- the local_expert_start ..
+    local_expert_end of metrale's build_ep_routing_table, one range per rank,
+    every expert on exactly one rank (the pages leave the split open; this is
+    the plain even split)."""
+    return [(E * q // world, E * (q + 1) // world) for q in range(world)]
+
+
+def expert_owner(expert_ids, E: int, world: int) -> np.ndarray:
+    """Owning rank of each expert id: the range of expert_ranges() holding it,
+    found by a plain search."""
+    ids = _ints(expert_ids)
+    ranges = expert_ranges(E, world)
+    out = np.empty(ids.shape, dtype=np.int64)
+    for i, e in np.ndenumerate(ids):
+        out[i] = next(q for q, (a, b) in enumerate(ranges) if a <= e < b)
+    return out
+
+
+def tp_slice(w13_e, w2_e, rank: int, tp: int):
+    """One expert's tensor-parallel slice (modelexpress refit test,
+    ``FusedMoEModel._expert_loader``: take this rank's slice of the source --
+    rows [rank*I/tp, (rank+1)*I/tp) -- of w1 and of w3, and store them w1 low,
+    w3 high in the rank's [2*I/tp, H] slot).  The down projection w2 [H, I]
+    keeps the same I columns (the pages show only w13; splitting w2 along its
+    input dimension is the reading under which the ranks' outputs add up).
+    Returns (w13 slot [2*I/tp, H], w2 slice [H, I/tp]) in float64."""
+    w13_e = to_f64(w13_e)
+    w2_e = to_f64(w2_e)
+    I = w13_e.shape[0] // 2
+    it = I // tp
+    w1, w3 = w13_halves(w13_e, I)
+    slot = np.empty((2 * it, w13_e.shape[1]))
+    slot[0:it] = w1[rank * it:(rank + 1) * it]          # member 0 (w1): low half
+    slot[it:2 * it] = w3[rank * it:(rank + 1) * it]     # member 1 (w3): high half
+    return slot, w2_e[:, rank * it:(rank + 1) * it]
+
+
+def moe_forward_tokens_ep(params: dict, tokens, ids, w, start: int, end: int,
+                          with_shared: bool) -> np.ndarray:
+    """Masked-local partial of an expert-parallel rank owning experts
+    [start, end) (metrale ep_dispatch.rs, module doc: "masked-local plus
+    all-reduce"): out[t] = sum over j with start <= ids[t,j] < end of
+    w[t,j] * SwiGLU_{ids[t,j]}(x_t), plus the shared term on the one rank that
+    holds the shared expert.  The ranks' partials add up to the layer."""
+    tokens = _ints(tokens)
+    ids = _ints(ids)
+    w = to_f64(w)
+    xs = to_f64(params["x"])[tokens]
+    I = params["w13"].shape[1] // 2
+    H = params["w2"].shape[1]
+    out = np.zeros((len(tokens), H))
+    for e in np.unique(ids):
+        if not start <= e < end:
+            continue                                   # another rank's expert
+        rows, cols = np.nonzero(ids == e)
+        y = expert_output(xs[rows], params["w13"][int(e)], params["w2"][int(e)], I)
+        np.add.at(out, rows, w[rows, cols][:, None] * y)
+    if with_shared and params.get("w13s") is not None:
+        s = shared_expert(xs, params["w13s"], params["w2s"])
+        g = 1.0 / (1.0 + np.exp(-shared_gate_logit(xs, params["w_sg"])))
+        out += g[:, None] * s
+    return out
+
+
+def moe_forward_tokens_tp(params: dict, tokens, ids, w, rank: int, tp: int) -> np.ndarray:
+    """Partial of tensor-parallel rank ``rank`` of ``tp``: every selected
+    expert (and the shared one) run on the rank's I-slice (tp_slice); the
+    ranks' partials add up to the layer."""
+    tokens = _ints(tokens)
+    ids = _ints(ids)
+    w = to_f64(w)
+    xs = to_f64(params["x"])[tokens]
+    H = params["w2"].shape[1]
+    out = np.zeros((len(tokens), H))
+    for e in np.unique(ids):
+        rows, cols = np.nonzero(ids == e)
+        slot, w2r = tp_slice(params["w13"][int(e)], params["w2"][int(e)], rank, tp)
+        y = expert_output(xs[rows], slot, w2r, slot.shape[0] // 2)
+        np.add.at(out, rows, w[rows, cols][:, None] * y)
+    if params.get("w13s") is not None:
+        slot, w2r = tp_slice(params["w13s"], params["w2s"], rank, tp)
+        s = expert_output(xs, slot, w2r, slot.shape[0] // 2)
+        g = 1.0 / (1.0 + np.exp(-shared_gate_logit(xs, params["w_sg"])))
+        out += g[:, None] * s
+    return out
 
 
 # ------------------------------------------------------------- metrics ---

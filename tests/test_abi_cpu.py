@@ -52,7 +52,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_workspace_queries(lib):
-    assert M.moe_abi_version() == 2
+    assert M.moe_abi_version() == 3
     assert M.moe_launch_count() == 0     # nothing launched on a CPU-only host
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
