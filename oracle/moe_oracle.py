@@ -26,7 +26,8 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "to_f64", "router_logits", "softmax_rows", "topk_experts", "routing_weights",
+    "to_f64", "router_logits", "softmax_rows", "topk_experts", "topk_experts_grouped",
+    "routing_weights",
     "route", "route_from_logits", "dispatch", "gather_rows", "silu", "w13_halves",
     "expert_hidden", "expert_output", "experts", "combine", "shared_expert",
     "shared_gate_logit", "moe_forward", "moe_forward_tokens", "ep_partition",
@@ -94,6 +95,32 @@ def topk_experts(l: np.ndarray, k: int) -> np.ndarray:
     return order[:, :k].astype(np.int64)
 
 
+def topk_experts_grouped(l: np.ndarray, k: int, n_groups: int, topk_groups: int) -> np.ndarray:
+    """Group-limited top-k (diffulex.moe API reference, ``diffulex.moe.topk``:
+    ``GroupLimitedTopKRouter``, "router with group-limited expert selection";
+    the page gives no formula, so the plainest reading is taken):
+
+    1. the E experts form ``n_groups`` equal groups of consecutive ids,
+       group g = experts [g*E/G, (g+1)*E/G);
+    2. a group's score is the largest logit among its experts;
+    3. the ``topk_groups`` groups with the highest scores are kept (equal
+       scores -> lower group id first);
+    4. the k experts are chosen among the kept groups' experts exactly as
+       topk_experts chooses them among all (key (-logit, expert id)).
+    The routing weights stay the softmax over all E experts (routing_weights).
+    """
+    T, E = l.shape
+    gs = E // n_groups
+    out = np.empty((T, k), dtype=np.int64)
+    for t in range(T):
+        score = [max(l[t, g * gs:(g + 1) * gs]) for g in range(n_groups)]
+        groups = sorted(range(n_groups), key=lambda g: (-score[g], g))[:topk_groups]
+        cand = [e for g in sorted(groups) for e in range(g * gs, (g + 1) * gs)]
+        cand.sort(key=lambda e: (-l[t, e], e))
+        out[t] = cand[:k]
+    return out
+
+
 def routing_weights(l: np.ndarray, ids: np.ndarray, renormalize: bool) -> np.ndarray:
     """Routing weights of the selected experts (DWDP README, "Router Module":
     normalized routing weights).
@@ -115,10 +142,15 @@ def route(x, W_gate, bias, k: int, renormalize: bool):
     return l, ids, routing_weights(l, ids, renormalize)
 
 
-def route_from_logits(logits, k: int, renormalize: bool):
-    """Selection and weights from given logits (e.g. fp32 logits made elsewhere)."""
+def route_from_logits(logits, k: int, renormalize: bool, n_groups: int = 1,
+                      topk_groups: int = 1):
+    """Selection and weights from given logits (e.g. fp32 logits made elsewhere);
+    n_groups > 1 selects group-limited (topk_experts_grouped)."""
     l = to_f64(logits)
-    ids = topk_experts(l, k)
+    if n_groups > 1:
+        ids = topk_experts_grouped(l, k, n_groups, topk_groups)
+    else:
+        ids = topk_experts(l, k)
     return ids, routing_weights(l, ids, renormalize)
 
 
