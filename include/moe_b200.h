@@ -104,6 +104,27 @@ int moe_route(const void* x, const void* W_gate, const float* bias,
               float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
               void* stream);
 
+/*
+ * moe_route_grouped -- Router with group-limited expert selection
+ * (diffulex.moe API reference, "diffulex.moe.topk": GroupLimitedTopKRouter).
+ * The page gives no rule; the one implemented is the plainest reading:
+ *   the E experts form n_groups groups of E / n_groups consecutive ids;
+ *   a group's score is the largest logit among its experts;
+ *   the topk_groups groups with the highest scores are kept (equal scores:
+ *   lower group id first);
+ *   topk_ids = the k largest logits among the kept groups' experts, ordered
+ *   and tie-broken as in moe_route.
+ * logits and topk_w are defined as in moe_route (the softmax spans all E
+ * experts; renormalize divides by the k selected probabilities).
+ * n_groups == 1 is moe_route.  Needs n_groups <= 32, E % n_groups == 0,
+ * 1 <= topk_groups <= n_groups and 1 <= k <= topk_groups * E / n_groups;
+ * otherwise MOE_ERR_INVALID_ARG.  All other arguments as moe_route.
+ */
+int moe_route_grouped(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
+                      int k, int renormalize, int n_groups, int topk_groups, int dtype,
+                      float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                      void* stream);
+
 /* Bytes of device scratch moe_dispatch needs for (T, k, E). */
 size_t moe_dispatch_workspace_bytes(int T, int k, int E);
 

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "MoEError", "lib_path", "load_library", "moe_abi_version", "moe_launch_count",
     "moe_last_error",
-    "moe_route", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_dispatch_noalloc",
+    "moe_route", "moe_route_grouped", "moe_dispatch_workspace_bytes", "moe_dispatch", "moe_dispatch_noalloc",
     "moe_experts_workspace_bytes",
     "moe_experts", "moe_experts_shared", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
@@ -68,6 +68,7 @@ _SIGS = {
     "moe_read_status": (_I, [_P, _P, _P]),
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_combine_range": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_finalize": (_I, [_P, _I, _I, _I, _P, _P]),
     "moe_ep_partition_workspace_bytes": (_SZ, [_I, _I]),
@@ -139,6 +140,18 @@ def moe_route(x, W_gate, bias, k: int, renormalize: bool, logits, topk_ids=None,
                                     int(bool(renormalize)), _dtype_code(x), _ptr(logits),
                                     _ptr(topk_ids), _ptr(topk_w), _ptr(status),
                                     _stream(stream)))
+
+
+def moe_route_grouped(x, W_gate, bias, k: int, renormalize: bool, n_groups: int,
+                      topk_groups: int, logits, topk_ids, topk_w, status=None, stream=None):
+    """Group-limited router: top-k among the experts of the topk_groups best
+    of n_groups consecutive-expert groups (a group scored by its best logit)."""
+    T, H = x.shape
+    E = W_gate.shape[0]
+    _check(load_library().moe_route_grouped(
+        _ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k, int(bool(renormalize)), n_groups,
+        topk_groups, _dtype_code(x), _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _ptr(status),
+        _stream(stream)))
 
 
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
@@ -324,15 +337,21 @@ class MoELayerBuffers:
 
 
 def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
-                      stream=None):
+                      stream=None, n_groups: int = 1, topk_groups: int = 1):
     """Router -> dispatcher -> executor -> merger into ``buf.out`` (asynchronous).
 
     ``params``: W_gate [E,H], bias [E] f32 or None, w13 [E,2I,H], w2 [E,H,I] and,
-    for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].
+    for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].  n_groups > 1
+    routes group-limited (moe_route_grouped).
     """
     E = params["W_gate"].shape[0]
-    moe_route(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits, buf.ids,
-              buf.w, status=buf.status, stream=stream)
+    if n_groups > 1:
+        moe_route_grouped(x, params["W_gate"], params.get("bias"), k, renormalize, n_groups,
+                          topk_groups, buf.logits, buf.ids, buf.w, status=buf.status,
+                          stream=stream)
+    else:
+        moe_route(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits, buf.ids,
+                  buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
     shared = sg = None

@@ -88,29 +88,60 @@ unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_o
 
 const char* moe_last_error(void) { return g_err.c_str(); }
 
+namespace {
+
+int route_impl(const char* fn, const void* x, const void* W_gate, const float* bias, int T,
+               int H, int E, int k, int renormalize, int n_groups, int topk_groups, int dtype,
+               float* logits, int32_t* topk_ids, float* topk_w, int32_t* status, void* stream) {
+  const std::string f = std::string(fn) + ": ";
+  if (int r = check_dtype(dtype)) return r;
+  REQ(x && W_gate && logits, MOE_ERR_INVALID_ARG, f + "null x, W_gate or logits");
+  REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, f + "T and H must be >= 1");
+  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, f + "E must be in [1, 256]");
+  REQ(k >= 0 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
+      f + "k must be in [0, min(E, 8)]");
+  REQ(k == 0 || (topk_ids && topk_w), MOE_ERR_INVALID_ARG, f + "null topk_ids or topk_w");
+  REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, f + "H must be a multiple of 8");
+  REQ(aligned16(x) && aligned16(W_gate), MOE_ERR_INVALID_ARG,
+      f + "x and W_gate must be 16-byte aligned");
+  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias) &&
+          aligned4(status),
+      MOE_ERR_INVALID_ARG, f + "outputs, bias and status must be 4-byte aligned");
+  REQ(static_cast<long long>(T) * (H > E ? H : E) < (1ll << 31), MOE_ERR_INVALID_ARG,
+      f + "T*H too large");
+  if (n_groups > 1) {
+    REQ(n_groups <= 32 && E % n_groups == 0, MOE_ERR_INVALID_ARG,
+        f + "n_groups must divide E and be at most 32");
+    REQ(topk_groups >= 1 && topk_groups <= n_groups, MOE_ERR_INVALID_ARG,
+        f + "topk_groups must be in [1, n_groups]");
+    REQ(k >= 1 && k <= topk_groups * (E / n_groups), MOE_ERR_INVALID_ARG,
+        f + "k must be in [1, topk_groups * E / n_groups]");
+  }
+  cudaError_t e = moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
+                                         logits, topk_ids, topk_w, status,
+                                         static_cast<cudaStream_t>(stream), n_groups,
+                                         topk_groups);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, (f + "launch").c_str());
+}
+
+}  // namespace
+
 int moe_route(const void* x, const void* W_gate, const float* bias, int T, int H, int E, int k,
               int renormalize, int dtype, float* logits, int32_t* topk_ids, float* topk_w,
               int32_t* status, void* stream) {
   g_err.clear();
-  if (int r = check_dtype(dtype)) return r;
-  REQ(x && W_gate && logits, MOE_ERR_INVALID_ARG, "moe_route: null x, W_gate or logits");
-  REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_route: T and H must be >= 1");
-  REQ(E >= 1 && E <= moe::kMaxExperts, MOE_ERR_INVALID_ARG, "moe_route: E must be in [1, 256]");
-  REQ(k >= 0 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
-      "moe_route: k must be in [0, min(E, 8)]");
-  REQ(k == 0 || (topk_ids && topk_w), MOE_ERR_INVALID_ARG, "moe_route: null topk_ids or topk_w");
-  REQ(H % 8 == 0, MOE_ERR_INVALID_ARG, "moe_route: H must be a multiple of 8");
-  REQ(aligned16(x) && aligned16(W_gate), MOE_ERR_INVALID_ARG,
-      "moe_route: x and W_gate must be 16-byte aligned");
-  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias) &&
-          aligned4(status),
-      MOE_ERR_INVALID_ARG, "moe_route: outputs, bias and status must be 4-byte aligned");
-  REQ(static_cast<long long>(T) * (H > E ? H : E) < (1ll << 31), MOE_ERR_INVALID_ARG,
-      "moe_route: T*H too large");
-  cudaError_t e = moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
-                                         logits, topk_ids, topk_w, status,
-                                         static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+  return route_impl("moe_route", x, W_gate, bias, T, H, E, k, renormalize, 1, 1, dtype, logits,
+                    topk_ids, topk_w, status, stream);
+}
+
+int moe_route_grouped(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
+                      int k, int renormalize, int n_groups, int topk_groups, int dtype,
+                      float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
+                      void* stream) {
+  g_err.clear();
+  REQ(n_groups >= 1, MOE_ERR_INVALID_ARG, "moe_route_grouped: n_groups must be >= 1");
+  return route_impl("moe_route_grouped", x, W_gate, bias, T, H, E, k, renormalize, n_groups,
+                    topk_groups, dtype, logits, topk_ids, topk_w, status, stream);
 }
 
 size_t moe_dispatch_workspace_bytes(int T, int k, int E) {

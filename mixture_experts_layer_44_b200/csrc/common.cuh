@@ -79,12 +79,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Host-side internal launchers (one translation unit each).  They assume the
 // arguments were validated by the ABI layer and return a cudaError_t.
 namespace moe_host {
+// n_groups > 1: group-limited selection (topk_groups of n_groups groups kept).
 cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, int T, int H,
                          int E, int k, int renormalize, int dtype, float* logits,
-                         int32_t* ids, float* w, int32_t* status, cudaStream_t s);
+                         int32_t* ids, float* w, int32_t* status, cudaStream_t s,
+                         int n_groups = 1, int topk_groups = 1);
 cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
                             int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
-                            int32_t* status, cudaStream_t s);
+                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups);
 size_t dispatch_ws_bytes(int T, int k, int E);
 cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, int T, int H,
                             int E, int k, int dtype, int32_t* counts, int32_t* offsets,

@@ -74,7 +74,8 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
                                                          int E, int k, int renorm,
                                                          float* __restrict__ logits,
                                                          int32_t* __restrict__ ids,
-                                                         float* __restrict__ wout) {
+                                                         float* __restrict__ wout,
+                                                         moe::GroupLimit gl) {
   constexpr int NWARP = NS / 32;
   constexpr int EPW = EP > NWARP ? EP / NWARP : 1;       // experts per warp
   constexpr int WPE = EP >= NWARP ? 1 : NWARP / EP;      // warps (H slices) per expert
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict_
   }
   if (k == 0) return;
   moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
-                        wout + static_cast<size_t>(t) * k);
+                        wout + static_cast<size_t>(t) * k, gl);
 }
 
 // Token rows per thread: 8 when E <= 64 (more FMAs per shared-memory read),
@@ -193,7 +194,8 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
                                                    int E, int k, int renorm, int kc_per_cta,
                                                    float* __restrict__ logits,
                                                    int32_t* __restrict__ ids,
-                                                   float* __restrict__ wout) {
+                                                   float* __restrict__ wout,
+                                                   moe::GroupLimit gl) {
   constexpr int TT = Tile<EPAD>::TT;
   constexpr int BTC = Tile<EPAD>::BT;        // tokens per cluster
   constexpr int TE = Tile<EPAD>::TE;         // experts per thread
@@ -346,14 +348,15 @@ __global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
     }
     if (k == 0) continue;
     moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
-                     wout + static_cast<size_t>(t) * k);
+                          wout + static_cast<size_t>(t) * k, gl);
   }
   cluster.sync();   // no CTA leaves while another still reads its partial tile
 }
 
 template <int EPAD, bool BF16>
 cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H, int E, int k,
-                     int renorm, float* logits, int32_t* ids, float* w, cudaStream_t s) {
+                     int renorm, float* logits, int32_t* ids, float* w, moe::GroupLimit gl,
+                     cudaStream_t s) {
   constexpr int BTC = Tile<EPAD>::BT;
   const size_t smem =
       sizeof(float) * std::max(2 * (KC * BTC + KC * EPAD), BTC * (EPAD + 1));
@@ -367,7 +370,7 @@ cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H,
   S = std::max(1, std::min({S, MAX_S, chunks}));
   const int kc_per_cta = (chunks + S - 1) / S;
   return moe_host::launch_pdl(fn, dim3(S, tiles, 1), dim3(NT, 1, 1), smem, s, S, x, W, b, T, H,
-                              E, k, renorm, kc_per_cta, logits, ids, w);
+                              E, k, renorm, kc_per_cta, logits, ids, w, gl);
 }
 
 }  // namespace
@@ -376,8 +379,11 @@ namespace moe_host {
 
 cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, int T, int H,
                          int E, int k, int renormalize, int dtype, float* logits, int32_t* ids,
-                         float* w, int32_t* status, cudaStream_t s) {
+                         float* w, int32_t* status, cudaStream_t s, int n_groups,
+                         int topk_groups) {
   const bool bf = dtype == MOE_BF16;
+  const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
+                           n_groups > 1 ? topk_groups : 1};
   if (T <= 64 && E <= 64 && H <= 32768) {
 #define MOE_SMALL_CASE(EPV)                                                                   \
     if (E <= EPV) {                                                                         \
@@ -386,13 +392,13 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
             reinterpret_cast<const void*>(route_small_kernel<EPV, true>), H * 4);           \
         if (e != cudaSuccess) return e;                                                     \
         return launch_pdl(route_small_kernel<EPV, true>, dim3(T), dim3(NS), H * 4, s, 0, x,   \
-                          W_gate, bias, H, E, k, renormalize, logits, ids, w);              \
+                          W_gate, bias, H, E, k, renormalize, logits, ids, w, gl);          \
       }                                                                                     \
       cudaError_t e = ensure_smem(                                                          \
           reinterpret_cast<const void*>(route_small_kernel<EPV, false>), H * 4);            \
       if (e != cudaSuccess) return e;                                                       \
       return launch_pdl(route_small_kernel<EPV, false>, dim3(T), dim3(NS), H * 4, s, 0, x,    \
-                        W_gate, bias, H, E, k, renormalize, logits, ids, w);                \
+                        W_gate, bias, H, E, k, renormalize, logits, ids, w, gl);            \
     }
     MOE_SMALL_CASE(1)
     MOE_SMALL_CASE(2)
@@ -403,10 +409,12 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
     MOE_SMALL_CASE(64)
 #undef MOE_SMALL_CASE
   }
-  if (bf) return launch_route_tc(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
-  if (E <= 64) return launch_t<64, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
-  if (E <= 128) return launch_t<128, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
-  if (E <= 256) return launch_t<256, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, s);
+  if (bf)
+    return launch_route_tc(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s,
+                           n_groups, topk_groups);
+  if (E <= 64) return launch_t<64, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, gl, s);
+  if (E <= 128) return launch_t<128, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, gl, s);
+  if (E <= 256) return launch_t<256, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, gl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(RNT, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias,
                     int T, int E, int k, int renorm, int kblocks, float* __restrict__ logits,
-                    int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* status) {
+                    int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* status,
+                    moe::GroupLimit gl) {
   using C = RCfg<EPAD>;
   constexpr int LS = C::LS;
   extern __shared__ uint8_t smem_raw[];
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(RNT, 1)
       const size_t tb = static_cast<size_t>(t0 + rows[1]) * k;
       int32_t* const it[2] = {ids + ta, has_b ? ids + tb : nullptr};
       float* const wt[2] = {wout + ta, has_b ? wout + tb : nullptr};
-      moe::select_topk_n<PER, 2>(v, live, k, renorm, it, wt);
+      moe::select_topk_n<PER, 2>(v, live, k, renorm, it, wt, gl);
     }
   }
   cluster.sync();   // no CTA leaves while another still reads its partial tile
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(RNT, 1)
 template <int EPAD>
 cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H, int E, int k,
                      int renorm, float* logits, int32_t* ids, float* w, int32_t* status,
-                     cudaStream_t s) {
+                     moe::GroupLimit gl, cudaStream_t s) {
   auto fn = route_tc_kernel<EPAD>;
   constexpr size_t smem = smem_bytes<EPAD>();
   cudaError_t err = moe_host::ensure_smem(reinterpret_cast<const void*>(fn), (int)smem);
@@ -306,7 +307,7 @@ cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H,
   int S = moe_host::num_sms() / tiles;
   S = std::max(1, std::min({S, RMAX_S, kblocks}));
   return moe_host::launch_pdl(fn, dim3(S * tiles, 1, 1), dim3(RNT, 1, 1), smem, s, S, mx, mw, b,
-                              T, E, k, renorm, kblocks, logits, ids, w, status);
+                              T, E, k, renorm, kblocks, logits, ids, w, status, gl);
 }
 
 }  // namespace
@@ -315,11 +316,13 @@ namespace moe_host {
 
 cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
                             int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
-                            int32_t* status, cudaStream_t s) {
-  if (E <= 32) return launch_t<32>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
-  if (E <= 64) return launch_t<64>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
-  if (E <= 128) return launch_t<128>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
-  if (E <= 256) return launch_t<256>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s);
+                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups) {
+  const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
+                           n_groups > 1 ? topk_groups : 1};
+  if (E <= 32) return launch_t<32>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
+  if (E <= 64) return launch_t<64>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
+  if (E <= 128) return launch_t<128>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
+  if (E <= 256) return launch_t<256>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -24,6 +24,43 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
+// Group-limited selection (diffulex.moe.topk, GroupLimitedTopKRouter): the
+// experts form `count` groups of `gsize` consecutive ids, a group scores as
+// its best expert, and only the `keep` best groups (equal scores: lower group
+// id first) stay in the running.  count <= 1: no limit.
+struct GroupLimit {
+  int gsize;
+  int count;
+  int keep;
+};
+
+// Bit g of the result is set when group g is kept.  key[j] is the order key
+// of expert lane + 32 j (0 = no expert); gidx[j] its group.  Every lane
+// returns the same mask.
+template <int PER>
+__device__ __forceinline__ uint32_t kept_groups(const uint32_t (&key)[PER], const int (&gidx)[PER],
+                                                GroupLimit gl) {
+  const int lane = threadIdx.x & 31;
+  uint32_t mine = 0;                                   // score key of group `lane`
+  for (int g = 0; g < gl.count; ++g) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+      if (gidx[j] == g) m = key[j] > m ? key[j] : m;
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == g) mine = m;
+  }
+  uint32_t mask = 0;
+  for (int r = 0; r < gl.keep; ++r) {
+    const uint32_t best = __reduce_max_sync(0xffffffffu, mine);
+    const uint32_t who = __reduce_min_sync(
+        0xffffffffu, (lane < gl.count && mine == best) ? static_cast<uint32_t>(lane) : 32u);
+    mask |= 1u << who;
+    if (lane == static_cast<int>(who)) mine = 0;
+  }
+  return mask;
+}
+
 // Top-k selection and softmax weights for NTOK tokens at once, each held by
 // the whole warp (lane l holds the logits of experts l, l+32, ... of every
 // token; k >= 1).  Each lane first sorts its PER experts of a token by
@@ -35,19 +72,33 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 // reductions overlap.  The first round's logit is the row maximum m; the
 // weight of a selection is exp(l - m) divided by the sum over the k
 // selections (renormalize) or over all E experts.  Lane r < k writes
-// selection r of token n when ids_t[n] is not null.
+// selection r of token n when ids_t[n] is not null.  With a group limit the
+// experts of the groups left out are out of the running before the sort (the
+// softmax still spans all E; the group holding the row maximum is always
+// kept, so the first selection is still the row maximum m).
 template <int PER, int NTOK>
 __device__ __forceinline__ void select_topk_n(const float (&v)[NTOK][PER], const bool (&live)[PER],
                                               int k, int renorm, int32_t* const (&ids_t)[NTOK],
-                                              float* const (&w_t)[NTOK]) {
+                                              float* const (&w_t)[NTOK],
+                                              GroupLimit gl = GroupLimit{1, 1, 1}) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NTOK][PER], eid[NTOK][PER];
+  int gidx[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j)
+    gidx[j] = (gl.count > 1 && live[j]) ? (lane + 32 * j) / gl.gsize : -1;
 #pragma unroll
   for (int n = 0; n < NTOK; ++n) {
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
       key[n][j] = live[j] ? order_key(v[n][j]) : 0u;
       eid[n][j] = static_cast<uint32_t>(lane + 32 * j);
+    }
+    if (gl.count > 1) {
+      const uint32_t kept = kept_groups<PER>(key[n], gidx, gl);
+#pragma unroll
+      for (int j = 0; j < PER; ++j)
+        if (gidx[j] >= 0 && !((kept >> gidx[j]) & 1u)) key[n][j] = 0u;
     }
     // odd-even transposition sort, PER passes: (key descending, id ascending)
 #pragma unroll
@@ -125,7 +176,8 @@ __device__ __forceinline__ void select_topk_n(const float (&v)[NTOK][PER], const
 // One token per warp (see select_topk_n).
 template <int PER>
 __device__ __forceinline__ void select_topk(const float* v, const bool* live, int k, int renorm,
-                                            int32_t* ids_t, float* w_t) {
+                                            int32_t* ids_t, float* w_t,
+                                            GroupLimit gl = GroupLimit{1, 1, 1}) {
   float vv[1][PER];
   bool lv[PER];
 #pragma unroll
@@ -135,7 +187,7 @@ __device__ __forceinline__ void select_topk(const float* v, const bool* live, in
   }
   int32_t* const it[1] = {ids_t};
   float* const wt[1] = {w_t};
-  select_topk_n<PER, 1>(vv, lv, k, renorm, it, wt);
+  select_topk_n<PER, 1>(vv, lv, k, renorm, it, wt, gl);
 }
 
 }  // namespace moe

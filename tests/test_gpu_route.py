@@ -151,3 +151,76 @@ def test_route_ties_on_the_tensor_core_path():
                           torch.randn(80, 64, generator=g).to(torch.bfloat16), None, 4, True)
     assert ids.tolist() == [[0, 1, 2, 3]] * 130
     np.testing.assert_allclose(w.numpy(), 0.25, rtol=1e-6)
+
+
+# ------------------------------------------------ group-limited router ---
+
+def _run_grouped(x, W, b, k, renorm, G, M):
+    T, E = x.shape[0], W.shape[0]
+    logits = torch.empty(T, E, device=DEV)
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, device=DEV)
+    M_ = M
+    import mixture_experts_layer_44_b200 as MM
+    MM.moe_route_grouped(dev(x), dev(W), dev(b), k, renorm, G, M_, logits, ids, w)
+    torch.cuda.synchronize()
+    return logits.cpu(), ids.cpu(), w.cpu()
+
+
+@pytest.mark.parametrize("E,k,G,Mg", [(8, 2, 4, 2), (64, 6, 8, 3), (60, 4, 6, 2), (128, 8, 8, 4),
+                                      (256, 8, 8, 4), (32, 4, 32, 4), (64, 2, 2, 1)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [7, 131])       # one-CTA-per-token path / cluster or tensor-core path
+def test_route_grouped_shapes(E, k, G, Mg, dtype, T):
+    cfg = LayerConfig("g", T=T, H=96, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 3 != 0))
+    p = make_layer(cfg, seed=E + G)
+    logits, ids, w = _run_grouped(p["x"], p["W_gate"], None, k, cfg.renormalize, G, Mg)
+    l64 = O.router_logits(p["x"], p["W_gate"], None)
+    assert rel(logits, l64) <= 1e-5
+    ids_o, w_o = O.route_from_logits(logits, k, cfg.renormalize, G, Mg)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    np.testing.assert_allclose(w.numpy(), w_o, rtol=1e-5, atol=0)
+    assert max(len(set((r // (E // G)).tolist())) for r in ids.numpy()) <= Mg
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [5, 200])
+def test_route_grouped_ties_between_groups(dtype, T):
+    # groups of 4 over 16 experts; experts 1, 6 and 13 share one W_gate row, so
+    # groups 0, 1 and 3 tie whenever that row wins its group
+    cfg = LayerConfig("gt", T=T, H=64, E=16, k=3, I=8, dtype=dtype, renormalize=True)
+    p = make_layer(cfg, seed=99)
+    W = p["W_gate"].clone()
+    W[6] = W[1]
+    W[13] = W[1]
+    W[1] *= 3                   # make the shared row win its group most of the time
+    W[6] = W[1]
+    W[13] = W[1]
+    logits, ids, w = _run_grouped(p["x"], W, None, 3, True, 4, 2)
+    ids_o, w_o = O.route_from_logits(logits, 3, True, 4, 2)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    np.testing.assert_allclose(w.numpy(), w_o, rtol=1e-5, atol=0)
+    # the tie really happens and goes to the lower groups
+    l = logits.numpy()
+    tied = (l[:, 1] == l[:, 6]) & (l[:, 1] == l[:, 13]) & (l[:, 1] == l.max(axis=1))
+    assert tied.sum() > 0
+    assert all(set(r.tolist()) >= {1, 6} for r in ids.numpy()[tied])
+
+
+def test_grouped_routing_through_the_whole_layer():
+    cfg = LayerConfig("g_layer", T=300, H=512, E=64, k=6, I=256, dtype="bf16", renormalize=True)
+    p = make_layer(cfg, seed=5)
+    dp = {k_: (dev(v) if v is not None else None) for k_, v in p.items()}
+    import mixture_experts_layer_44_b200 as MM
+    buf = MM.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, torch.bfloat16)
+    out = MM.moe_layer_forward(dp["x"], dp, cfg.k, True, buf, n_groups=8, topk_groups=3)
+    torch.cuda.synchronize()
+    assert int(buf.status.item()) == 0
+    ids = buf.ids.cpu().numpy()
+    ids_o, _ = O.route_from_logits(buf.logits.cpu(), cfg.k, True, 8, 3)
+    np.testing.assert_array_equal(ids, ids_o)
+    l64 = O.router_logits(p["x"], p["W_gate"], None)
+    w64 = O.routing_weights(l64, ids, True)
+    want = O.moe_forward_tokens(p, np.arange(cfg.T), ids, w64)
+    from tests.gpu_util import err_bf16_out
+    assert err_bf16_out(out.cpu(), want) <= 2e-2
