@@ -402,6 +402,78 @@ int moe_ep_owner(const int32_t* ids, int n, int E, int world, int32_t* owner, in
 int moe_ep_pack_ids(const int32_t* ids, const int32_t* perm, const int32_t* offsets, int n,
                     int E, int world, int32_t* local_ids, void* stream);
 
+/*
+ * ---- The whole layer behind one handle -----------------------------------
+ *
+ * DWDP README, "Runtime Integration Layer": router -> dispatcher ->
+ * executor -> merger, each stage consuming the previous stage's output.  A
+ * moe_layer holds a layer's shapes and weights (device pointers the caller
+ * keeps alive) and every intermediate buffer, carved from ONE device block
+ * the caller allocates (moe_layer_workspace_bytes; 256-byte aligned): the
+ * library allocates no device memory here either.  It owns three CUDA
+ * streams and a few events (host objects) for moe_layer_forward_host.
+ */
+typedef struct moe_layer_desc {
+  int T, H, E, k, I;          /* tokens per call, hidden, experts, top-k, expert width */
+  int dtype;                  /* MOE_F32 or MOE_BF16 */
+  int renormalize;            /* divide the k weights by their sum */
+  int n_groups, topk_groups;  /* group-limited routing when n_groups > 1 */
+  const void* W_gate;         /* device [E,H] */
+  const float* bias;          /* device [E] fp32 or NULL */
+  const void* w13;            /* device [E,2I,H] */
+  const void* w2;             /* device [E,H,I] */
+  int I_s;                    /* shared expert width (when w13s != NULL) */
+  const void* w13s;           /* device [2I_s,H] or NULL: no shared expert */
+  const void* w2s;            /* device [H,I_s] */
+  const void* w_sg;           /* device [H]: the shared expert's gate vector */
+} moe_layer_desc;
+
+typedef struct moe_layer moe_layer;   /* opaque */
+
+/* Device bytes moe_layer_create needs for `d` (0 if d is invalid). */
+size_t moe_layer_workspace_bytes(const moe_layer_desc* d);
+
+/* Check `d` once (the rules of the stage calls), carve the buffers out of
+ * `workspace` and zero what must start at zero (enqueued on `stream`, which
+ * is then synchronised once).  *out receives the handle. */
+int moe_layer_create(const moe_layer_desc* d, void* workspace, size_t workspace_bytes,
+                     void* stream, moe_layer** out);
+
+/* Wait for the handle's streams and free its host objects (not the workspace). */
+int moe_layer_destroy(moe_layer* L);
+
+/* The layer on device activations: x device [T,H] (dtype) -> out device
+ * [T,H] (dtype), enqueued on `stream`, as moe_route, moe_dispatch,
+ * moe_experts(_shared) and moe_combine chained. */
+int moe_layer_forward(moe_layer* L, const void* x, void* out, void* stream);
+
+/*
+ * The layer on HOST activations: x_host [T,H] -> out_host [T,H], both host
+ * memory of the activation type (pinned, so that the copies run
+ * asynchronously).  Enqueues, without waiting for completion:
+ *   upload x_host into one of two device copies of x (one cudaMemcpyAsync,
+ *   after the work already on `stream` and after the step that last used
+ *   that copy), the layer, and the download into out_host (one
+ *   cudaMemcpyAsync), on three internal streams.  Consecutive calls
+ *   therefore overlap: one step uploads while the previous one computes and
+ *   the one before it downloads.
+ * x_host must stay unchanged and out_host unread until the step is done:
+ * moe_layer_join(L, s) makes stream s wait for every step enqueued so far.
+ */
+int moe_layer_forward_host(moe_layer* L, const void* x_host, void* out_host, void* stream);
+
+/* Make `stream` wait for all work enqueued on L so far. */
+int moe_layer_join(moe_layer* L, void* stream);
+
+/* moe_layer_join, then copy L's device status word to *host_status
+ * (synchronises `stream`). */
+int moe_layer_status(moe_layer* L, void* stream, int32_t* host_status);
+
+/* Device address of one of L's intermediate buffers, for inspection:
+ * "logits", "ids", "w", "counts", "offsets", "inv_perm", "status"; NULL for
+ * any other name. */
+void* moe_layer_buffer(moe_layer* L, const char* name);
+
 /* Copy the device status word to *host_status after the stream's prior work
  * (synchronises `stream`).  Returns MOE_OK or MOE_ERR_CUDA. */
 int moe_read_status(const int32_t* status, void* stream, int32_t* host_status);

@@ -29,6 +29,7 @@ __all__ = [
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
     "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
     "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
+    "MoELayerDesc", "MoELayer",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
@@ -69,6 +70,14 @@ _SIGS = {
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "moe_layer_workspace_bytes": (_SZ, [_P]),
+    "moe_layer_create": (_I, [_P, _P, _SZ, _P, _P]),
+    "moe_layer_destroy": (_I, [_P]),
+    "moe_layer_forward": (_I, [_P, _P, _P, _P]),
+    "moe_layer_forward_host": (_I, [_P, _P, _P, _P]),
+    "moe_layer_join": (_I, [_P, _P]),
+    "moe_layer_status": (_I, [_P, _P, _P]),
+    "moe_layer_buffer": (_P, [_P, ctypes.c_char_p]),
     "moe_combine_range": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_finalize": (_I, [_P, _I, _I, _I, _P, _P]),
     "moe_ep_partition_workspace_bytes": (_SZ, [_I, _I]),
@@ -289,6 +298,96 @@ def moe_read_status(status, stream=None) -> int:
 
 def moe_probe_wait_timeout(status, budget_us: int, stream=None):
     _check(load_library().moe_probe_wait_timeout(_ptr(status), budget_us, _stream(stream)))
+
+
+class MoELayerDesc(ctypes.Structure):
+    """ctypes mirror of moe_layer_desc (include/moe_b200.h)."""
+    _fields_ = [("T", _I), ("H", _I), ("E", _I), ("k", _I), ("I", _I), ("dtype", _I),
+                ("renormalize", _I), ("n_groups", _I), ("topk_groups", _I), ("W_gate", _P),
+                ("bias", _P), ("w13", _P), ("w2", _P), ("I_s", _I), ("w13s", _P), ("w2s", _P),
+                ("w_sg", _P)]
+
+
+def _desc(params: dict, T: int, k: int, renormalize: bool, n_groups: int, topk_groups: int):
+    W = params["W_gate"]
+    E, H = W.shape
+    I = params["w13"].shape[1] // 2
+    d = MoELayerDesc(T=T, H=H, E=E, k=k, I=I, dtype=_dtype_code(W),
+                     renormalize=int(bool(renormalize)), n_groups=n_groups,
+                     topk_groups=topk_groups, W_gate=W.data_ptr(),
+                     bias=params["bias"].data_ptr() if params.get("bias") is not None else None,
+                     w13=params["w13"].data_ptr(), w2=params["w2"].data_ptr())
+    if params.get("w13s") is not None:
+        d.I_s = params["w13s"].shape[0] // 2
+        d.w13s = params["w13s"].data_ptr()
+        d.w2s = params["w2s"].data_ptr()
+        d.w_sg = params["w_sg"].data_ptr()
+    return d
+
+
+class MoELayer:
+    """moe_layer handle: the whole layer for batches of T tokens, its buffers in
+    one device block (a torch tensor this object keeps).  ``params`` (device
+    tensors) must stay alive as long as the layer."""
+
+    def __init__(self, params: dict, T: int, k: int, renormalize: bool, n_groups: int = 1,
+                 topk_groups: int = 1, stream=None):
+        lib = load_library()
+        self.params = params
+        self.desc = _desc(params, T, k, renormalize, n_groups, topk_groups)
+        nbytes = lib.moe_layer_workspace_bytes(ctypes.byref(self.desc))
+        if nbytes == 0:
+            raise MoEError(MOE_ERR_INVALID_ARG, "moe_layer_workspace_bytes: invalid layer")
+        self.ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=params["W_gate"].device)
+        off = (-self.ws.data_ptr()) % 256
+        self.block = self.ws[off:off + nbytes]
+        h = ctypes.c_void_p()
+        _check(lib.moe_layer_create(ctypes.byref(self.desc), _ptr(self.block), nbytes,
+                                    _stream(stream), ctypes.byref(h)))
+        self.handle = h
+        self.T, self.H = T, self.desc.H
+        self.dtype = params["W_gate"].dtype
+
+    def forward(self, x, out, stream=None):
+        _check(load_library().moe_layer_forward(self.handle, _ptr(x), _ptr(out), _stream(stream)))
+        return out
+
+    def forward_host(self, x_host, out_host, stream=None):
+        _check(load_library().moe_layer_forward_host(self.handle, ctypes.c_void_p(x_host.data_ptr()),
+                                                     ctypes.c_void_p(out_host.data_ptr()),
+                                                     _stream(stream)))
+        return out_host
+
+    def join(self, stream=None):
+        _check(load_library().moe_layer_join(self.handle, _stream(stream)))
+
+    def status(self, stream=None) -> int:
+        v = ctypes.c_int32(0)
+        _check(load_library().moe_layer_status(self.handle, _stream(stream), ctypes.byref(v)))
+        return int(v.value)
+
+    def buffer(self, name: str, shape, dtype) -> torch.Tensor:
+        """A view of one of the layer's intermediate buffers (see moe_layer_buffer)."""
+        p = load_library().moe_layer_buffer(self.handle, name.encode())
+        if not p:
+            raise MoEError(MOE_ERR_INVALID_ARG, f"no layer buffer named {name!r}")
+        n = 1
+        for d in shape:
+            n *= d
+        off = p - self.block.data_ptr()
+        es = torch.empty(0, dtype=dtype).element_size()
+        return self.block[off:off + n * es].view(dtype).view(*shape)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load_library().moe_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class MoELayerBuffers:

@@ -145,3 +145,27 @@ def test_python_binding_raises_with_the_library_message(lib):
     x = torch.empty(0, 64)
     with pytest.raises(M.MoEError, match="moe_route: "):
         M.moe_route(x, torch.empty(8, 64), None, 2, True, torch.empty(0, 8), stream=0)
+
+
+def test_layer_descriptor_is_checked_on_the_host(lib):
+    d = M.MoELayerDesc(T=64, H=256, E=8, k=2, I=128, dtype=M.MOE_BF16, renormalize=1,
+                       n_groups=1, topk_groups=1, W_gate=256, bias=None, w13=512, w2=768)
+    n = lib.moe_layer_workspace_bytes(ctypes.byref(d))
+    # two copies each of x and out, the packed buffers, fp32 y_packed, the workspaces
+    assert n >= 4 * 64 * 256 * 2 + 128 * 256 * 2 + 128 * 128 * 2 + 128 * 256 * 4
+    for field, bad in (("I", 100), ("k", 9), ("E", 0), ("dtype", 7), ("H", 200)):
+        b = M.MoELayerDesc.from_buffer_copy(d)
+        setattr(b, field, bad)
+        assert lib.moe_layer_workspace_bytes(ctypes.byref(b)) == 0, field
+    g = M.MoELayerDesc.from_buffer_copy(d)
+    g.n_groups, g.topk_groups = 4, 1            # k = 2 <= 1 * 8 / 4: fine
+    assert lib.moe_layer_workspace_bytes(ctypes.byref(g)) == n
+    g.n_groups, g.topk_groups = 8, 1            # k = 2 > 1 * 8 / 8
+    assert lib.moe_layer_workspace_bytes(ctypes.byref(g)) == 0
+    h = ctypes.c_void_p()
+    assert lib.moe_layer_create(ctypes.byref(d), None, n, None, ctypes.byref(h)) == M.MOE_ERR_INVALID_ARG
+    assert "workspace" in M.moe_last_error()
+    assert lib.moe_layer_create(ctypes.byref(d), ctypes.c_void_p(4096 + 16), n, None,
+                                ctypes.byref(h)) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_forward(None, P, P, None) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_destroy(None) == M.MOE_OK
