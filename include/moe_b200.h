@@ -488,6 +488,20 @@ int moe_read_status(const int32_t* status, void* stream, int32_t* host_status);
  */
 int moe_probe_wait_timeout(int32_t* status, int budget_us, void* stream);
 
+/*
+ * moe_test_set_wait_budget_ns -- testing hook for failure detection.  Sets the
+ * budget of the main-loop waits of the tensor-core kernels (the grouped GEMM
+ * and the tensor-core router) for launches made after the call, process
+ * wide: 0 restores the default (2 s); otherwise 1000 <= ns <= 2e9.  With a
+ * budget of a few microseconds ordinary waits for copies and MMAs run out,
+ * so the kernels report MOE_ERR_TIMEOUT and take their abort path (their
+ * drain waits keep the full budget: every issued copy and MMA completes
+ * before a CTA leaves, and TMEM is freed).  Results of such launches are
+ * undefined; re-zero a moe_experts workspace used by one.  Not for
+ * production use.
+ */
+int moe_test_set_wait_budget_ns(unsigned long long ns);
+
 #ifdef __cplusplus
 }
 #endif

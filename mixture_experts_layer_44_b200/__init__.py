@@ -29,7 +29,7 @@ __all__ = [
     "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
     "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
     "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
-    "MoELayerDesc", "MoELayer",
+    "MoELayerDesc", "MoELayer", "moe_test_set_wait_budget_ns",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
@@ -71,6 +71,7 @@ _SIGS = {
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "moe_layer_workspace_bytes": (_SZ, [_P]),
+    "moe_test_set_wait_budget_ns": (_I, [ctypes.c_ulonglong]),
     "moe_layer_create": (_I, [_P, _P, _SZ, _P, _P]),
     "moe_layer_destroy": (_I, [_P]),
     "moe_layer_forward": (_I, [_P, _P, _P, _P]),
@@ -294,6 +295,11 @@ def moe_read_status(status, stream=None) -> int:
     v = ctypes.c_int32(0)
     _check(load_library().moe_read_status(_ptr(status), _stream(stream), ctypes.byref(v)))
     return int(v.value)
+
+
+def moe_test_set_wait_budget_ns(ns: int):
+    """Testing hook: budget of the tensor-core kernels' main-loop waits (0 = default)."""
+    _check(load_library().moe_test_set_wait_budget_ns(ns))
 
 
 def moe_probe_wait_timeout(status, budget_us: int, stream=None):

@@ -17,6 +17,7 @@ namespace {
 
 thread_local std::string g_err;
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned long long> g_main_wait_ns{moe::kWaitBudgetNs};
 
 int fail(int code, const std::string& msg) {
   g_err = msg;
@@ -57,6 +58,7 @@ __global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
 namespace moe_host {
 void set_last_error(const std::string& msg) { g_err = msg; }
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+uint64_t main_wait_budget_ns() { return g_main_wait_ns.load(std::memory_order_relaxed); }
 
 cudaError_t ensure_smem(const void* kernel, int bytes) {
   static std::mutex mu;
@@ -417,6 +419,15 @@ int moe_read_status(const int32_t* status, void* stream, int32_t* host_status) {
   cudaError_t e = cudaMemcpyAsync(host_status, status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_read_status");
+}
+
+int moe_test_set_wait_budget_ns(unsigned long long ns) {
+  g_err.clear();
+  if (ns == 0) ns = moe::kWaitBudgetNs;
+  REQ(ns >= 1000 && ns <= moe::kWaitBudgetNs, MOE_ERR_INVALID_ARG,
+      "moe_test_set_wait_budget_ns: budget must be 0 (default) or in [1000, 2e9] ns");
+  g_main_wait_ns.store(ns, std::memory_order_relaxed);
+  return MOE_OK;
 }
 
 int moe_probe_wait_timeout(int32_t* status, int budget_us, void* stream) {

@@ -142,6 +142,10 @@ cudaError_t ensure_smem(const void* kernel, int bytes);
 // Count one kernel enqueued by this library (moe_launch_count).
 void note_launch();
 
+// Budget of the main-loop waits of the tensor-core kernels (nanoseconds):
+// kWaitBudgetNs unless moe_test_set_wait_budget_ns shortened it.
+uint64_t main_wait_budget_ns();
+
 // Launch with programmatic stream serialization (and a cluster of cluster_x
 // CTAs along x when cluster_x > 0).
 template <typename... KArgs, typename... Args>

@@ -50,6 +50,12 @@
 // of them; the last CTA to exit resets the ticket for the next launch.
 // Without one, CTA b takes units b, b+grid, b+2*grid, ...
 //
+// Waits.  The waits of the main loops (unit ring, stage ring, accumulators)
+// are bounded by `wait_ns` (normally the 2 s budget; a test hook shortens it
+// so that ordinary waits run out and the abort path runs).  The drain waits
+// at the end -- every issued copy landed, every issued MMA completed -- always
+// keep the full budget, so nothing is in flight when the CTA leaves.
+//
 // CTA = 6 warps, one CTA per SM, persistent over units:
 //   warp 0    TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
 //   warp 1    MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
@@ -109,7 +115,9 @@ struct Ctl {
 };
 
 constexpr int STAGE_OUT_BYTES = BM * 128;                  // epilogue staging: 128 rows x 128 B
-constexpr size_t CTL_BYTES = (sizeof(Ctl) + 127) / 128 * 128;
+// The staging buffer starts on a 1024-byte boundary: TMA stores read it with
+// the 128-byte swizzle, whose pattern is anchored there.
+constexpr size_t CTL_BYTES = (sizeof(Ctl) + 1023) / 1024 * 1024;
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTL_BYTES + STAGE_OUT_BYTES;
 
 // A work unit: tile (group g, expert e, weight tile nt, token tile mt) and
@@ -276,11 +284,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB2,
+                        const __grid_constant__ CUtensorMap tmY,
+                        const __grid_constant__ CUtensorMap tmY2,
                         const int32_t* __restrict__ offsets, int E, int K, int ntw,
                         int rows_per_expert, const float* __restrict__ packed_w,
                         void* __restrict__ out, int ldo, int rows2, int K2, int ntw2,
                         void* __restrict__ out2, int ldo2, int* __restrict__ counters,
-                        float* __restrict__ partials, int max_units, int32_t* status) {
+                        float* __restrict__ partials, int max_units, int32_t* status,
+                        uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -402,7 +413,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int next_static = blockIdx.x;
       for (;;) {
         // Take the next unit and publish its id (-1: no more work) to the consumers.
-        if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1)) {
+        if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1, wait_ns)) {
           set_abort(c, status);
           break;
         }
@@ -427,7 +438,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const CUtensorMap* ma = g1 ? &tmA2 : &tmA;
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
-          if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
+          if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1, wait_ns)) {
             set_abort(c, status);
             ok = false;
             break;
@@ -467,7 +478,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int uslot = 0;
       uint32_t uphase = 0;
       for (;; ++i) {
-        if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase)) {
+        if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns)) {
           set_abort(c, status);
           break;
         }
@@ -480,7 +491,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (u < 0) break;
         const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int buf = i & 1;
-        if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1)) {
+        if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1, wait_ns)) {
           set_abort(c, status);
           break;
         }
@@ -488,7 +499,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
-          if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase)) {
+          if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase, wait_ns)) {
             set_abort(c, status);
             ok = false;
             break;
@@ -522,7 +533,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int uslot = 0;
     uint32_t uphase = 0;
     for (;; ++i) {
-      if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase)) {
+      if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns)) {
         set_abort(c, status);
         break;
       }
@@ -535,7 +546,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (u < 0) break;
       const int buf = i & 1;
-      if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1)) {
+      if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1, wait_ns)) {
         set_abort(c, status);
         break;
       }
@@ -615,21 +626,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             epi_bar();
           }
         } else {
+          // fp32 output, 32 columns per step.  Each warp works alone on its
+          // 32-row quarter: when all 32 rows belong to the unit it stages
+          // them (the 128-byte-swizzled layout a TMA store reads) and one lane
+          // hands the 32 x 32 block to the TMA engine, so no thread waits on
+          // global stores and no barrier spans the warps; a partly valid
+          // quarter stores its valid rows directly.
           const float sc = live ? (upw ? upw[grow] : 1.f) : 0.f;
           uint8_t* gtile =
               static_cast<uint8_t*>(uout) + (row0 * uldo + un.nt * BN) * sizeof(float);
+          const int qrows = min(max(nvalid - q * 32, 0), 32);
+          const CUtensorMap* ym = g1 ? &tmY2 : &tmY;
+          const uint32_t wstg = moe::smem_addr(stg + q * 32 * 128);
 #pragma unroll 1
           for (int cc = 0; cc < BN; cc += 32) {
             uint32_t a[16], b[16];
             moe::tmem_ld16(taddr + cc, a);
             moe::tmem_ld16(taddr + cc + 16, b);
             moe::tmem_ld_wait();
-            if (staged) {
+            if (qrows == 32) {
+              if (lane == 0) moe::bulk_wait_read_all();   // the last store has read the stage
+              __syncwarp();
               stage_f32x32(stg, row, a, b, sc);
-              epi_bar();
-              stage_flush(stg, q, lane, nvalid, gtile + cc * sizeof(float),
-                          static_cast<size_t>(uldo) * sizeof(float));
-              epi_bar();
+              moe::fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                moe::tma_store_2d(ym, wstg, un.nt * BN + cc, static_cast<int>(row0) + q * 32);
+                moe::bulk_commit();
+              }
             } else if (live) {
               store_f32x32(reinterpret_cast<float*>(gtile) + static_cast<size_t>(row) * uldo + cc,
                            a, b, sc);
@@ -641,6 +665,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
       } else {
         // Partial of one K-slice: valid rows to this unit's workspace slot.
+        // (In the w2 pass a TMA store of an earlier unit may still be reading
+        // this warp's quarter of the staging buffer: let it finish first.)
+        if (EPI == EPI_SCALE) {
+          if (lane == 0) moe::bulk_wait_read_all();
+          __syncwarp();
+        }
         uint8_t* gtile = reinterpret_cast<uint8_t*>(partials + static_cast<size_t>(u) * (BM * BN));
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 32) {
@@ -724,6 +754,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
 
+  if (EPI == EPI_SCALE && warp >= 2 && lane == 0)
+    moe::bulk_wait_all();          // this warp's TMA stores are complete before the grid ends
   moe::grid_dep_launch();
   moe::tc_fence_before();
   __syncthreads();
@@ -745,6 +777,15 @@ bool map_rows(CUtensorMap* m, const void* p, int rows, int K) {
   const cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
   const cuuint32_t box[2] = {BK, BM};
   return moe_host::encode_bf16_sw128(m, p, 2, dims, str, box);
+}
+
+// fp32 outputs [rows, cols], the target of the w2 pass's TMA stores: box of 32
+// columns (128 bytes, one swizzle row) x 32 rows.
+bool map_out_f32(CUtensorMap* m, const void* p, int rows, int cols) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t str[1] = {static_cast<cuuint64_t>(cols) * 4};
+  const cuuint32_t box[2] = {32, 32};
+  return moe_host::encode_f32_sw128(m, p, 2, dims, str, box);
 }
 
 }  // namespace
@@ -802,6 +843,11 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     const cuuint32_t b2[2] = {BK, BN};
     ok = ok && encode_bf16_sw128(&sB2, sh->w2, 2, d2, s2, b2);
   }
+  // the w2 pass's fp32 outputs (the shared expert's own, or the routed map standing in)
+  CUtensorMap mY, sY;
+  ok = ok && map_out_f32(&mY, y, nmap, H);
+  sY = mY;
+  if (sh) ok = ok && map_out_f32(&sY, sh->y, T2, H);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
     return cudaErrorInvalidValue;
@@ -829,13 +875,14 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   }
   const float* no_w = nullptr;
   cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS),
-                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, offsets, E, H, ntw1,
+                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, mY, sY, offsets, E, H, ntw1,
                                2 * I, no_w, h, I, T2, H, ntw1s, sh ? sh->h : nullptr, Is,
-                               counters, partials, max_units, status);
+                               counters, partials, max_units, status, main_wait_budget_ns());
   if (err != cudaSuccess) return err;
   return launch_pdl(k2, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
-                    mA2, mB2, sA2, sB2, offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
-                    sh ? sh->y : nullptr, H, counters, partials, max_units, status);
+                    mA2, mB2, sA2, sB2, mY, sY, offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
+                    sh ? sh->y : nullptr, H, counters, partials, max_units, status,
+                    main_wait_budget_ns());
 }
 
 }  // namespace moe_host

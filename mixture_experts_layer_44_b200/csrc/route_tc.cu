@@ -27,7 +27,9 @@
 // (warp w: TMEM lanes 32*(w%4) .. +31, column half w/4) and finalise tokens.
 // Every wait is bounded; one that runs out reports MOE_ERR_TIMEOUT in the
 // status word and the CTA still takes part in both cluster barriers, so its
-// peers finish too.
+// peers finish too.  The stage-ring waits are bounded by `wait_ns` (a test
+// hook can shorten it); the drain of issued copies and the wait for the
+// issued MMAs (accf) always keep the full budget.
 #include <cooperative_groups.h>
 #include <cuda.h>
 
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(RNT, 1)
                     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias,
                     int T, int E, int k, int renorm, int kblocks, float* __restrict__ logits,
                     int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* status,
-                    moe::GroupLimit gl) {
+                    moe::GroupLimit gl, uint64_t wait_ns) {
   using C = RCfg<EPAD>;
   constexpr int LS = C::LS;
   extern __shared__ uint8_t smem_raw[];
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(RNT, 1)
     uint32_t phase = 0;
     int issued[C::STAGES] = {};
     for (int kb = kb0; kb < kb1; ++kb) {
-      if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1)) {
+      if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1, wait_ns)) {
         set_abort(c, status);
         break;
       }
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(RNT, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int i = 0; i < nkb; ++i) {
-      if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase)) {
+      if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase, wait_ns)) {
         set_abort(c, status);
         break;
       }
@@ -307,7 +309,8 @@ cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H,
   int S = moe_host::num_sms() / tiles;
   S = std::max(1, std::min({S, RMAX_S, kblocks}));
   return moe_host::launch_pdl(fn, dim3(S * tiles, 1, 1), dim3(RNT, 1, 1), smem, s, S, mx, mw, b,
-                              T, E, k, renorm, kblocks, logits, ids, w, status, gl);
+                              T, E, k, renorm, kblocks, logits, ids, w, status, gl,
+                              moe_host::main_wait_budget_ns());
 }
 
 }  // namespace

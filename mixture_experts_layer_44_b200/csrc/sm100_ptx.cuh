@@ -107,6 +107,22 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* m, int c0, in
                : "memory");
 }
 
+// shared -> global tensor store of one box at (c0, c1), tracked by the issuing
+// thread's bulk groups.  The shared source must be written through the
+// generic proxy first and then fenced (fence_proxy_async_smem).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Make this thread's shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // --------------------------------------------- bulk (non-tensor) copies ---
 
 // global -> shared, completion counted on `bar` (bytes % 16 == 0, both 16B aligned)

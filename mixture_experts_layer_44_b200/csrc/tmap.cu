@@ -23,12 +23,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-bool encode_uncached(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                     const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+bool encode_uncached(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank,
+                     const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+                     const cuuint32_t* box) {
   auto fn = get_encode();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+  CUresult r = fn(m, dt, rank, const_cast<void*>(base), dims,
                   strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -39,7 +40,7 @@ bool encode_uncached(CUtensorMap* m, const void* base, int rank, const cuuint64_
 // buffers reuses its descriptors instead of encoding four per call.  The map
 // depends only on the key (device, base, rank, dims, strides, box).
 struct MapKey {
-  int dev, rank;
+  int dev, rank, dtype;
   const void* base;
   cuuint64_t dims[3], strides[2];
   cuuint32_t box[3];
@@ -49,8 +50,11 @@ struct MapKey {
 
 namespace moe_host {
 
-bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-                       const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+namespace {
+
+bool encode_cached(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank,
+                   const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+                   const cuuint32_t* box) {
   constexpr int kSlots = 64;
   static std::mutex mu;
   static MapKey keys[kSlots];
@@ -60,6 +64,7 @@ bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint6
   std::memset(&k, 0, sizeof(k));
   cudaGetDevice(&k.dev);
   k.rank = rank;
+  k.dtype = static_cast<int>(dt);
   k.base = base;
   for (int i = 0; i < rank; ++i) {
     k.dims[i] = dims[i];
@@ -72,11 +77,23 @@ bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint6
       *m = maps[i];
       return true;
     }
-  if (!encode_uncached(m, base, rank, dims, strides_bytes, box)) return false;
+  if (!encode_uncached(m, dt, base, rank, dims, strides_bytes, box)) return false;
   const int slot = used < kSlots ? used++ : (next++ % kSlots);
   keys[slot] = k;
   maps[slot] = *m;
   return true;
+}
+
+}  // namespace
+
+bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box);
+}
+
+bool encode_f32_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                      const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, rank, dims, strides_bytes, box);
 }
 
 }  // namespace moe_host
