@@ -169,3 +169,36 @@ def test_layer_descriptor_is_checked_on_the_host(lib):
                                 ctypes.byref(h)) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_forward(None, P, P, None) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_destroy(None) == M.MOE_OK
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
+    B = M.MOE_BF16
+    # group-limited router: groups must divide E, at most 32, enough experts kept
+    assert lib.moe_route_grouped(P, P, NULL, 4, 64, 12, 2, 1, 5, 1, B, P, P, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert "n_groups must divide E" in M.moe_last_error()
+    assert lib.moe_route_grouped(P, P, NULL, 4, 64, 64, 2, 1, 64, 2, B, P, P, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_grouped(P, P, NULL, 4, 64, 16, 8, 1, 8, 3, B, P, P, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert "topk_groups * E / n_groups" in M.moe_last_error()
+    assert lib.moe_route_grouped(P, P, NULL, 4, 64, 16, 2, 1, 8, 9, B, P, P, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_grouped(P, P, NULL, 4, 64, 16, 2, 1, 0, 1, B, P, P, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    # range gather / merge: 0 <= start <= end <= E
+    assert lib.moe_gather(P, P, P, 8, 3, 9, 16, 64, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather(P, P, P, 8, 5, 4, 16, 64, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_range(P, P, P, 8, -1, 4, 4, 64, 2, NULL, NULL, M.MOE_F32, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_finalize(NULL, 4, 64, B, P, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_finalize(P, 4, 60, B, P, NULL) == M.MOE_ERR_INVALID_ARG
+    # owner ids: at most one rank per expert
+    assert lib.moe_ep_owner(P, 8, 4, 5, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_pack_ids(P, P, P, 8, 4, 0, P, NULL) == M.MOE_ERR_INVALID_ARG
+    # routing table: the page's panics, and a missing workspace for a large table
+    assert lib.moe_ep_partition(P, 3, P, 4, 2, 2, 0, 256, P, P, P, P, P, P, P, NULL, 0, NULL) == M.MOE_ERR_INVALID_ARG
+    assert M.moe_last_error() == "gate_indices length mismatch"
+    assert lib.moe_ep_partition(P, 4, P, 3, 2, 2, 0, 256, P, P, P, P, P, P, P, NULL, 0, NULL) == M.MOE_ERR_INVALID_ARG
+    assert M.moe_last_error() == "gate_weights length mismatch"
+    assert lib.moe_ep_partition(P, 8000, P, 8000, 1000, 8, 0, 4, P, P, P, P, P, P, P, NULL, 0, NULL) == M.MOE_ERR_INVALID_ARG
+    assert M.moe_ep_partition_workspace_bytes(1000, 8) >= 4 * 4
+    # dispatch takes repeated ids (all-to-all by owner) but still k <= 8
+    assert lib.moe_dispatch(P, P, NULL, 4, 0, 2, 9, B, P, P, P, P, P, P, NULL, P, 256, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    # the testing hook's bounds
+    assert lib.moe_test_set_wait_budget_ns(10) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_test_set_wait_budget_ns(0) == M.MOE_OK

@@ -35,6 +35,32 @@ PROGRAM = textwrap.dedent(r"""
       if (moe_dispatch_workspace_bytes(16384, 8, 128) < (size_t)64 * 128 * 4) {
         puts("dispatch ws"); ++fails;
       }
+      /* the layer handle's descriptor, checked on the host */
+      moe_layer_desc d;
+      memset(&d, 0, sizeof d);
+      d.T = 64; d.H = 256; d.E = 8; d.k = 2; d.I = 128; d.dtype = MOE_BF16; d.renormalize = 1;
+      d.W_gate = dummy; d.w13 = dummy; d.w2 = dummy;
+      size_t need = moe_layer_workspace_bytes(&d);
+      if (need < (size_t)4 * 64 * 256 * 2) { puts("layer ws"); ++fails; }
+      d.I = 100;
+      if (moe_layer_workspace_bytes(&d) != 0) { puts("layer desc check"); ++fails; }
+      moe_layer* L = NULL;
+      if (moe_layer_create(&d, NULL, need, NULL, &L) != MOE_ERR_INVALID_ARG || L != NULL) {
+        puts("layer create check"); ++fails;
+      }
+      /* the page's length-mismatch rule, on the host */
+      r = moe_ep_partition((const int32_t*)dummy, 3, (const float*)dummy, 4, 2, 2, 0, 256,
+                           dummy, dummy, (float*)dummy, dummy, dummy, (float*)dummy, dummy,
+                           NULL, 0, NULL);
+      if (r != MOE_ERR_INVALID_ARG || strcmp(moe_last_error(), "gate_indices length mismatch")) {
+        puts("ep length"); ++fails;
+      }
+      r = moe_ep_partition((const int32_t*)dummy, 4, (const float*)dummy, 3, 2, 2, 0, 256,
+                           dummy, dummy, (float*)dummy, dummy, dummy, (float*)dummy, dummy,
+                           NULL, 0, NULL);
+      if (r != MOE_ERR_INVALID_ARG || strcmp(moe_last_error(), "gate_weights length mismatch")) {
+        puts("ep weights length"); ++fails;
+      }
       printf("%s\n", fails ? "FAIL" : "OK");
       return fails;
     }
