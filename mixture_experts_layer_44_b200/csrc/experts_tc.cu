@@ -330,7 +330,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
     moe::tmem_relinquish();
   }
-  moe::grid_dep_wait();        // offsets and the A operand come from the previous kernels
+  // Pass 1 reads offsets and x_packed, both written by the kernels just before
+  // it, so it waits for them first.  Pass 2's inputs other than h are older:
+  // its offsets were final before pass 1 could start (pass 1 waited for them,
+  // and pass 2 starts only once every pass-1 CTA has passed that wait), and
+  // the weights are constant.  So pass 2 builds its tile table and requests
+  // the weights of its first unit while pass 1 still finishes, and waits only
+  // before its first read of h.
+  constexpr bool EARLY = EPI == EPI_SCALE;
+  if (!EARLY) moe::grid_dep_wait();
   if (warp == 2) {
     // Tile table: per-expert token-tile counts, exclusive scan, x ntw.
     // Lane l owns experts [8l, 8l+8); lane 31 also writes the end entries.
@@ -342,8 +350,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int e = lane * 8 + j;
       int m = 0;
       if (e < E) {
-        c.offs[e] = offsets[e];
-        const int rows = offsets[e + 1] - offsets[e];
+        // read at L2, the point of coherence (pass 2 reads before its wait)
+        const int o0 = __ldcg(offsets + e), o1 = __ldcg(offsets + e + 1);
+        c.offs[e] = o0;
+        const int rows = o1 - o0;
         m = (rows + BM - 1) / BM;
         rmax = max(rmax, min(rows, BM));
       }
@@ -367,7 +377,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       run += cnt[j];
     }
     if (lane == 31) {
-      c.offs[E] = offsets[E];
+      c.offs[E] = __ldcg(offsets + E);
       const int tiles = n2 + incl * ntw;
       c.tstart[E] = tiles;
       c.n2 = n2;
@@ -402,15 +412,57 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int total = c.n2 * c.splits2 + (c.tstart[E] - c.n2) * c.splits;   // units
   const uint32_t tmem = c.tmem_base;
 
+  // The B operand (weights) of k-block kb of unit un into stage buffer sa,
+  // completing on barrier fb.
+  auto load_b = [&](const Unit& un, int kb, uint32_t sa, uint32_t fb) {
+    if (SHARED && un.g) {
+      if (EPI == EPI_SWIGLU)
+        moe::tma_load_3d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), 0);
+      else
+        moe::tma_load_2d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * BN);
+    } else if (EPI == EPI_SWIGLU) {
+      moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, un.nt * (BN / 2), 2 * un.e);
+    } else {
+      moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, un.e * rows_per_expert + un.nt * BN);
+    }
+  };
+
+  // Pass 2, before waiting for pass 1: the weights of this CTA's first unit
+  // (static: unit blockIdx.x) into the first stages, and the next k-blocks
+  // into L2.  Each such stage's barrier expects the whole stage; the A half
+  // follows after the wait.
+  int pre = 0;                                   // stages whose B half is on its way
+  int pre_issued[STAGES] = {};
+  if (EARLY && warp == 0 && lane == 0 && static_cast<int>(blockIdx.x) < total) {
+    const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, blockIdx.x);
+    pre = min(STAGES, un.kb1 - un.kb0);
+    for (int s = 0; s < pre; ++s) {
+      const uint32_t fb = moe::smem_addr(&c.full[s]);
+      moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+      load_b(un, un.kb0 + s, moe::smem_addr(smem + s * STAGE_BYTES), fb);
+      pre_issued[s] = 1;
+    }
+    const int l2_end = min(un.kb1, un.kb0 + pre + 8);
+    for (int kb = un.kb0 + pre; kb < l2_end; ++kb) {
+      if (SHARED && un.g)
+        moe::tma_prefetch_2d(&tmB2, kb * BK, un.nt * BN);
+      else
+        moe::tma_prefetch_2d(&tmB, kb * BK, un.e * rows_per_expert + un.nt * BN);
+    }
+  }
+  if (EARLY) moe::grid_dep_wait();               // h comes from pass 1
+
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------ producer ---
       int stage = 0;
       uint32_t phase = 0;
       int issued[STAGES] = {};
+      for (int s = 0; s < STAGES; ++s) issued[s] = pre_issued[s];
       int uslot = 0;
       uint32_t uphase = 0;
       int next_static = blockIdx.x;
+      int npre = pre;                              // the first unit's prefetched k-blocks
       for (;;) {
         // Take the next unit and publish its id (-1: no more work) to the consumers.
         if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1, wait_ns)) {
@@ -438,31 +490,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const CUtensorMap* ma = g1 ? &tmA2 : &tmA;
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
-          if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1, wait_ns)) {
-            set_abort(c, status);
-            ok = false;
-            break;
-          }
           const uint32_t fb = moe::smem_addr(&c.full[stage]);
           const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
-          moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
-          if (g1) {
-            if (EPI == EPI_SWIGLU)
-              moe::tma_load_3d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), 0);
-            else
-              moe::tma_load_2d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * BN);
-          } else if (EPI == EPI_SWIGLU) {
-            moe::tma_load_3d(sa + A_BYTES, &tmB, fb, kb * BK, un.nt * (BN / 2), 2 * un.e);
+          if (kb - un.kb0 < npre) {
+            // B already requested before the wait (fresh stage, nothing to wait for)
+            moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
           } else {
-            moe::tma_load_2d(sa + A_BYTES, &tmB, fb, kb * BK, un.e * rows_per_expert + un.nt * BN);
+            if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1, wait_ns)) {
+              set_abort(c, status);
+              ok = false;
+              break;
+            }
+            moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
+            load_b(un, kb, sa, fb);
+            ++issued[stage];
           }
-          ++issued[stage];
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+        npre = 0;
         if (!ok) break;
       }
       // Drain: every load issued has landed before the CTA can leave.
