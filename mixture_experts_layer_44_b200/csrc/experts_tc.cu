@@ -107,6 +107,7 @@ struct Ctl {
   int splits;          // S: K-slices per routed tile (1 = no split)
   int splits2;         // K-slices per shared-expert tile
   int last_flag;       // epilogue: this unit is the last of its tile
+  int slot_rows;       // rows of one split-K partial slot (the fullest tile's valid rows)
   int n2;              // tiles of the second group (a shared expert), numbered first
   int mte2;            // its token tiles
   int rows2;           // its rows
@@ -178,9 +179,9 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
 
 // Split count: 1 when there are at least two tiles per CTA; otherwise the
 // smallest S whose units fill the grid's waves to >= 90% (else the best one),
-// with >= 4 K-blocks per unit, the units within the workspace, and at most
-// 128 partial rows per tile (S x the fullest tile's valid rows), since one
-// CTA reads them all back.
+// with >= 4 K-blocks per unit, the units within the workspace's partial slots
+// (max_units), and at most 128 partial rows per tile (S x the fullest tile's
+// valid rows), since one CTA reads them all back.
 __device__ int choose_splits(int tiles, int grid, int kblocks, int max_units, int rows_max) {
   if (tiles <= 0 || tiles >= 2 * grid) return 1;
   int smax = min(MAX_SPLITS, kblocks / 4);
@@ -384,18 +385,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       c.mte2 = mte2;
       c.rows2 = rows2;
       const int rt = incl * ntw;                  // routed tiles
+      // A partial slot holds only the rows a tile can have (the fullest
+      // tile's, rounded up to 8), so decode batches, whose tiles have a row
+      // or two, fit many more slots in the workspace and can split finer.
+      const int slot_rows = min(BM, max(8, (max(rmax, min(rows2, BM)) + 7) / 8 * 8));
+      const int units_cap = static_cast<int>(
+          min(static_cast<long long>(max_units) * BM / slot_rows, 1ll << 30));
       int sp = 1, sp2 = 1;
       if (counters != nullptr && partials != nullptr && tiles <= SCHED_TICKET) {
         if (rt == 0) {
-          sp2 = choose_splits(n2, gridDim.x, kblocks2, max_units, min(rows2, BM));
+          sp2 = choose_splits(n2, gridDim.x, kblocks2, units_cap, min(rows2, BM));
         } else {
-          sp = choose_splits(tiles, gridDim.x, kblocks, max_units, max(rmax, min(rows2, BM)));
+          sp = choose_splits(tiles, gridDim.x, kblocks, units_cap, max(rmax, min(rows2, BM)));
           if (n2 > 0 && kblocks2 > kblocks) {
             // a longer shared K is cut into slices about as long as the routed units
             sp2 = min(sp * ((kblocks2 + kblocks - 1) / kblocks), MAX_SPLITS);
             sp2 = min(sp2, max(1, kblocks2 / 4));
             sp2 = min(sp2, max(2, BM / max(1, min(rows2, BM))));
-            if (n2 * sp2 + rt * sp > max_units) sp2 = sp;
+            if (n2 * sp2 + rt * sp > units_cap) sp2 = sp;
           } else {
             sp2 = sp;
           }
@@ -403,6 +410,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       c.splits = sp;
       c.splits2 = sp2;
+      c.slot_rows = slot_rows;
     }
   }
   moe::tc_fence_before();
@@ -720,7 +728,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (lane == 0) moe::bulk_wait_read_all();
           __syncwarp();
         }
-        uint8_t* gtile = reinterpret_cast<uint8_t*>(partials + static_cast<size_t>(u) * (BM * BN));
+        const size_t slot = static_cast<size_t>(c.slot_rows) * BN;   // floats per slot
+        uint8_t* gtile = reinterpret_cast<uint8_t*>(partials + static_cast<size_t>(u) * slot);
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 32) {
           uint32_t a[16], b[16];
@@ -758,7 +767,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __threadfence();
           const int et = threadIdx.x - 64;                // 0..127
           const int nrows = nvalid;
-          const float* base = partials + static_cast<size_t>(u - un.ks) * (BM * BN);
+          const float* base = partials + static_cast<size_t>(u - un.ks) * slot;
           if (EPI == EPI_SWIGLU) {
             const int cg = et & 31;                       // h columns 4cg .. 4cg+3
             for (int r = et >> 5; r < nrows && cg * 4 < ncol; r += 4) {
@@ -767,9 +776,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
               for (int s = 0; s < MAX_SPLITS; ++s) {
                 if (s < S) {
-                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN)));
+                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * slot));
                   const float4 b =
-                      __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN) + BN / 2));
+                      __ldcg(reinterpret_cast<const float4*>(pr + s * slot + BN / 2));
                   g.x += a.x; g.y += a.y; g.z += a.z; g.w += a.w;
                   v.x += b.x; v.y += b.y; v.z += b.z; v.w += b.w;
                 }
@@ -788,7 +797,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
               for (int s = 0; s < MAX_SPLITS; ++s) {
                 if (s < S) {
-                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * (BM * BN)));
+                  const float4 a = __ldcg(reinterpret_cast<const float4*>(pr + s * slot));
                   v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
                 }
               }

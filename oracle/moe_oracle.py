@@ -29,7 +29,7 @@ __all__ = [
     "to_f64", "router_logits", "softmax_rows", "topk_experts", "topk_experts_grouped",
     "routing_weights",
     "route", "route_from_logits", "dispatch", "gather_rows", "silu", "w13_halves",
-    "expert_hidden", "expert_output", "experts", "combine", "shared_expert",
+    "expert_hidden", "expert_output", "experts", "experts_down", "combine", "shared_expert",
     "shared_gate_logit", "moe_forward", "moe_forward_tokens", "ep_partition",
     "expert_ranges", "expert_owner", "tp_slice", "moe_forward_tokens_ep",
     "moe_forward_tokens_tp", "rel_err_rms",
@@ -234,6 +234,26 @@ def expert_output(x_rows: np.ndarray, w13_e, w2_e, I: int) -> np.ndarray:
     return expert_hidden(x_rows, w13_e, I) @ to_f64(w2_e).T
 
 
+def experts_down(h, offsets, packed_w, w2):
+    """The Executor's second product alone, fed a given hidden h [N, I]: for
+    each expert e and position p in its range, y_packed[p] = packed_w[p] *
+    (h[p] W2e^T).  experts() is expert_hidden followed by this step; fed the
+    hidden of a device, it checks that device's second product by itself."""
+    hh = to_f64(h)
+    offs = _ints(offsets)
+    E = len(offs) - 1
+    N = hh.shape[0]
+    H = w2.shape[1]
+    y = np.zeros((N, H))
+    pw = np.ones(N) if packed_w is None else to_f64(packed_w)
+    for e in range(E):
+        a, b = offs[e], offs[e + 1]
+        if b == a:
+            continue
+        y[a:b] = pw[a:b, None] * (hh[a:b] @ to_f64(w2[e]).T)
+    return y
+
+
 def experts(x_packed, offsets, packed_w, w13, w2):
     """Expert execution over expert-major ranges (DWDP README, "Executor
     Module": execute expert modules, apply routing weights, write packed
@@ -252,15 +272,12 @@ def experts(x_packed, offsets, packed_w, w13, w2):
     I = w13.shape[1] // 2
     H = w2.shape[1]
     h = np.zeros((N, I))
-    y = np.zeros((N, H))
-    pw = np.ones(N) if packed_w is None else to_f64(packed_w)
     for e in range(E):
         a, b = offs[e], offs[e + 1]
         if b == a:
             continue
         h[a:b] = expert_hidden(xp[a:b], w13[e], I)
-        y[a:b] = pw[a:b, None] * (h[a:b] @ to_f64(w2[e]).T)
-    return h, y
+    return h, experts_down(h, offs, packed_w, w2)
 
 
 # ---------------------------------------------------------------- Merger ---

@@ -7,10 +7,13 @@ benchmark times (moe_layer_forward over MoELayerBuffers), for every workload.
   two experts' fp64 logits differ by less than 1e-5;
 * dispatch: identical to the oracle's stable sort of the GPU's ids, and
   x_packed byte-identical to x gathered by packed_tok;
-* experts, at full size: EVERY row of h and of y_packed (and of the shared
-  expert's h_s / y_s) against the oracle's experts() fed the GPU's own
-  x_packed, offsets and packed_w: y_packed (fp32) within 2e-2 of the rms,
-  h (bf16) within 2e-2 beyond its own final rounding;
+* experts, at full size, stage by stage: EVERY row of h (and of the shared
+  expert's h_s) against the oracle's experts() fed the GPU's own x_packed,
+  offsets and packed_w -- h is bf16: within 2e-2 of the rms beyond its own
+  final rounding; and EVERY row of y_packed (and y_s) against the oracle's
+  second product fed the GPU's own h (experts_down) -- an fp32 result of an
+  fp32-accumulated product: within STAGED_Y_TOL of the rms.  Their distance
+  from the all-fp64 chain (h never rounded) is recorded too;
 * output, at full size: every token of the merged output, against the
   oracle's merge of its own expert outputs: the fp32 merge within 2e-2 of the
   rms, the bf16 output within 2e-2 beyond its final rounding (the plain
@@ -82,6 +85,10 @@ def test_tiny_f32_every_stage_and_every_token():
     assert rel(out, direct) <= TOL["f32"]
 
 
+# y_packed against the oracle's second product fed the GPU's own h: the
+# tensor cores' fp32 accumulation over K = I terms is all that separates them.
+STAGED_Y_TOL = 1e-3
+
 FULL = ["builder_bf16", "qwen15_t32", "qwen15_t8192", "qwen3_t16384", "decode_t1", "decode_t8",
         "decode_t64"]
 
@@ -106,24 +113,32 @@ def test_full_size_workload(name):
     assert torch.equal(x_packed.view(torch.int16), p["x"][packed_tok.long()].view(torch.int16))
     # every row of both expert passes, fed the GPU's own packed inputs
     offsets = buf.offsets.cpu().numpy()
-    h_o, y_o = O.experts(x_packed, offsets, buf.packed_w.cpu(), p["w13"], p["w2"])
+    packed_w = buf.packed_w.cpu()
+    h_o, y_o = O.experts(x_packed, offsets, packed_w, p["w13"], p["w2"])
     del x_packed
-    rec["h_err"] = err_bf16_out(buf.h.cpu(), h_o)
-    rec["h_err_plain"] = rel(buf.h.cpu(), h_o)
+    h_gpu = buf.h.cpu()
+    rec["h_err"] = err_bf16_out(h_gpu, h_o)
+    rec["h_err_plain"] = rel(h_gpu, h_o)
     del h_o
-    rec["y_packed_err"] = rel(buf.y_packed.cpu(), y_o)
+    y_gpu = buf.y_packed.cpu()
+    rec["y_packed_err_chain"] = rel(y_gpu, y_o)                   # vs h never rounded
+    rec["y_packed_err_staged"] = rel(y_gpu, O.experts_down(h_gpu, offsets, packed_w, p["w2"]))
+    del h_gpu, y_gpu
     assert rec["h_err"] <= TOL["bf16"], rec
-    assert rec["y_packed_err"] <= TOL["bf16"], rec
+    assert rec["y_packed_err_staged"] <= STAGED_Y_TOL, rec
     shared = sg = None
     if cfg.shared_I:
-        hs_o, shared = O.experts(p["x"], np.array([0, cfg.T]), None, p["w13s"].unsqueeze(0),
-                                 p["w2s"].unsqueeze(0))
+        one = np.array([0, cfg.T])
+        w13s, w2s = p["w13s"].unsqueeze(0), p["w2s"].unsqueeze(0)
+        hs_o, shared = O.experts(p["x"], one, None, w13s, w2s)
         sg = O.shared_gate_logit(p["x"], p["w_sg"])
-        rec["shared_h_err"] = err_bf16_out(buf.sh_h.cpu(), hs_o)
-        rec["shared_y_err"] = rel(buf.sh_y.cpu(), shared)
+        sh_h = buf.sh_h.cpu()
+        rec["shared_h_err"] = err_bf16_out(sh_h, hs_o)
+        rec["shared_y_err_chain"] = rel(buf.sh_y.cpu(), shared)
+        rec["shared_y_err_staged"] = rel(buf.sh_y.cpu(), O.experts_down(sh_h, one, None, w2s))
         rec["shared_gate_logit_err"] = rel(buf.sg_logit.cpu().reshape(-1), sg)
         assert rec["shared_h_err"] <= TOL["bf16"], rec
-        assert rec["shared_y_err"] <= TOL["bf16"], rec
+        assert rec["shared_y_err_staged"] <= STAGED_Y_TOL, rec
         assert rec["shared_gate_logit_err"] <= 1e-5, rec
         del hs_o
     # every token of the merged output
