@@ -121,3 +121,68 @@ def test_wrong_shared_gate_is_caught(monkeypatch, bad_gate):
         return orig(y_packed, inv_perm, T, k, shared, shared_gate)
     monkeypatch.setattr(M, "combine", bad)
     assert _fails(P.test_shared_expert_and_sigmoid_gate)
+
+
+# --------------------------- the sharded forms and group-limited selection ---
+
+import tests.test_oracle_grouped as G          # noqa: E402
+import tests.test_oracle_parallel as PP        # noqa: E402
+
+
+def test_group_scored_by_its_worst_expert_is_caught(monkeypatch):
+    def bad(l, k, n_groups, topk_groups):
+        T, E = l.shape
+        gs = E // n_groups
+        out = np.empty((T, k), dtype=np.int64)
+        for t in range(T):
+            score = [min(l[t, g * gs:(g + 1) * gs]) for g in range(n_groups)]    # min, not max
+            groups = sorted(range(n_groups), key=lambda g: (-score[g], g))[:topk_groups]
+            cand = sorted((e for g in groups for e in range(g * gs, (g + 1) * gs)),
+                          key=lambda e: (-l[t, e], e))
+            out[t] = cand[:k]
+        return out
+    monkeypatch.setattr(M, "topk_experts_grouped", bad)
+    assert _fails(G.test_brute_force_on_tiny_layers, 8, 3, 4, 2)
+    assert _fails(G.test_a_case_where_group_limiting_changes_the_choice)
+
+
+def test_group_ties_to_the_higher_group_are_caught(monkeypatch):
+    orig = M.topk_experts_grouped
+
+    def bad(l, k, n_groups, topk_groups):
+        E = l.shape[1]
+        gs = E // n_groups
+        flip = np.concatenate([np.arange((n_groups - 1 - g) * gs, (n_groups - g) * gs)
+                               for g in range(n_groups)])
+        got = orig(l[:, flip], k, n_groups, topk_groups)        # groups numbered backwards
+        return flip[got]
+    monkeypatch.setattr(M, "topk_experts_grouped", bad)
+    assert _fails(G.test_equal_group_scores_keep_the_lower_group)
+
+
+def test_tp_slice_with_swapped_members_is_caught(monkeypatch):
+    orig = M.tp_slice
+
+    def bad(w13_e, w2_e, rank, tp):
+        slot, w2r = orig(w13_e, w2_e, rank, tp)
+        it = slot.shape[0] // 2
+        return np.concatenate([slot[it:], slot[:it]]), w2r         # w3 low, w1 high
+    monkeypatch.setattr(M, "tp_slice", bad)
+    assert _fails(PP.test_tp_slice_reproduces_the_refit_tests_worked_example)
+    assert _fails(PP.test_tensor_parallel_partials_add_up_to_the_layer, 2, False)
+
+
+def test_tp_slice_from_the_wrong_rank_is_caught(monkeypatch):
+    orig = M.tp_slice
+    monkeypatch.setattr(M, "tp_slice", lambda a, b, rank, tp: orig(a, b, (rank + 1) % tp, tp))
+    assert _fails(PP.test_tp_slice_of_every_rank_tiles_w13_and_w2) or \
+        _fails(PP.test_tensor_parallel_partials_add_up_to_the_layer, 2, True)
+    assert _fails(PP.test_tp_slice_reproduces_the_refit_tests_worked_example)
+
+
+def test_expert_range_off_by_one_is_caught(monkeypatch):
+    monkeypatch.setattr(M, "expert_ranges",
+                        lambda E, world: [(E * q // world, E * (q + 1) // world + (q == 0))
+                                          for q in range(world)])
+    assert _fails(PP.test_expert_ranges_partition_the_experts, 8, 3)
+    assert _fails(PP.test_masked_local_partials_add_up_to_the_layer, 3, False)
