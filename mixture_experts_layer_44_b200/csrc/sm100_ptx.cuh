@@ -49,17 +49,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the same phase (no suspension inside the instruction).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with parity `parity` of `bar` has completed, for at
 // most `budget_ns` of %globaltimer time (and, as a second guard should the
 // timer ever stall, at most budget_ns / 2 polls).  Returns false when the
-// budget ran out.
+// budget ran out.  With the default budget the first 32 polls skip the clock;
+// a shorter budget (a testing hook) polls without suspending and reads the
+// clock from the start, so that it really runs out after budget_ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           uint64_t budget_ns = kWaitBudgetNs) {
+  const uint64_t max_polls = budget_ns / 2 + 1;
+  if (budget_ns < kWaitBudgetNs) {
+    const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+    for (uint64_t n = 0; n < max_polls; ++n) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (globaltimer_ns() - t0 > budget_ns) return false;
+    }
+    return false;
+  }
 #pragma unroll 1
   for (int i = 0; i < 32; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  const uint64_t max_polls = budget_ns / 2 + 1;
 #pragma unroll 1
   for (uint64_t n = 0; n < max_polls; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
