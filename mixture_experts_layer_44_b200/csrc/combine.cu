@@ -31,12 +31,12 @@ namespace {
 constexpr int CNT = 256;
 
 template <bool OUT_BF16, int KT>
-__global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ y,
-                                                      const int32_t* __restrict__ inv_perm,
+__global__ void __launch_bounds__(CNT) combine_kernel(const float* y,
+                                                      const int32_t* inv_perm,
                                                       int T, int H, int k, int N,
-                                                      const float* __restrict__ shared,
-                                                      const float* __restrict__ sgate,
-                                                      const int32_t* __restrict__ range_offs,
+                                                      const float* shared,
+                                                      const float* sgate,
+                                                      const int32_t* range_offs,
                                                       int lo_e, int hi_e,
                                                       void* __restrict__ outv, int32_t* status) {
   const int nvec = H / 8;                               // 8 outputs per thread step
@@ -45,13 +45,13 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
   moe::grid_dep_wait();
   int rlo = 0, rhi = N;                                 // rows that contribute
   if (range_offs != nullptr) {
-    rlo = range_offs[lo_e];
-    rhi = range_offs[hi_e];
+    rlo = moe::ld_prod(range_offs + lo_e);
+    rhi = moe::ld_prod(range_offs + hi_e);
   }
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < k) {
-      int p = inv_perm[static_cast<size_t>(t) * k + threadIdx.x];
+      int p = moe::ld_prod(inv_perm + static_cast<size_t>(t) * k + threadIdx.x);
       if (p < 0 || p >= N) {
         moe::report(status, MOE_ERR_BAD_INDEX);
         p = -1;
@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
       }
       rows[threadIdx.x] = p;
     }
-    if (threadIdx.x == 0) gate = shared ? (sgate ? 1.f / (1.f + expf(-sgate[t])) : 1.f) : 0.f;
+    if (threadIdx.x == 0)
+      gate = shared ? (sgate ? 1.f / (1.f + expf(-moe::ld_prod(sgate + t))) : 1.f) : 0.f;
     __syncthreads();
     for (int v = threadIdx.x; v < nvec; v += CNT) {
       float acc[8];
@@ -73,8 +74,8 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
         if (rows[j] >= 0) {
           const float4* src =
               reinterpret_cast<const float4*>(y + static_cast<size_t>(rows[j]) * H) + 2 * v;
-          a[j] = src[0];
-          b[j] = src[1];
+          a[j] = moe::ld_prod(src);
+          b[j] = moe::ld_prod(src + 1);
         }
       }
 #pragma unroll
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
       if (shared) {
         const float g = gate;
         const float4* src = reinterpret_cast<const float4*>(shared + static_cast<size_t>(t) * H) + 2 * v;
-        const float4 a = src[0], b = src[1];
+        const float4 a = moe::ld_prod(src), b = moe::ld_prod(src + 1);
         acc[0] = fmaf(g, a.x, acc[0]); acc[1] = fmaf(g, a.y, acc[1]);
         acc[2] = fmaf(g, a.z, acc[2]); acc[3] = fmaf(g, a.w, acc[3]);
         acc[4] = fmaf(g, b.x, acc[4]); acc[5] = fmaf(g, b.y, acc[5]);
@@ -109,12 +110,12 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* __restrict__ 
 
 // out = acc rounded once to the output type (bf16 or fp32 copy).
 template <bool OUT_BF16>
-__global__ void __launch_bounds__(CNT) finalize_kernel(const float4* __restrict__ acc,
+__global__ void __launch_bounds__(CNT) finalize_kernel(const float4* acc,
                                                        size_t nvec8, void* __restrict__ outv) {
   moe::grid_dep_wait();
   for (size_t v = blockIdx.x * static_cast<size_t>(CNT) + threadIdx.x; v < nvec8;
        v += static_cast<size_t>(gridDim.x) * CNT) {
-    const float4 a = acc[2 * v], b = acc[2 * v + 1];
+    const float4 a = moe::ld_prod(acc + 2 * v), b = moe::ld_prod(acc + 2 * v + 1);
     if (OUT_BF16) {
       reinterpret_cast<uint4*>(outv)[v] =
           make_uint4(moe::pack_bf16x2(a.x, a.y), moe::pack_bf16x2(a.z, a.w),

@@ -48,6 +48,17 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Loads of data that an earlier kernel of the stream produced.  Every kernel
+// here is launched with programmatic dependent launch, so it can be resident
+// while its producer still runs; the read-only data path (ld.global.nc) is
+// only valid for data that stays constant for a kernel's whole lifetime.
+// Such data is therefore read at L2, the point of coherence (ld.global.cg),
+// after griddepcontrol.wait.  Constant weights keep the read-only path.
+template <typename T>
+__device__ __forceinline__ T ld_prod(const T* p) {
+  return __ldcg(p);
+}
+
 // Unpack 8 bf16 (one 16-byte vector) into floats.
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);

@@ -43,7 +43,7 @@ constexpr int PER_WARP = CHUNK / DWARPS;
 
 // Per-warp per-expert counts of this CTA's slice.  Invalid ids (outside
 // [0,E)) are reported and skipped.  wc: [DWARPS][E] in shared memory.
-__device__ __forceinline__ void warp_counts(const int32_t* __restrict__ ids, int N, int E,
+__device__ __forceinline__ void warp_counts(const int32_t* ids, int N, int E,
                                             int base, int* wc, int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < DWARPS * E; i += DNT) wc[i] = 0;
@@ -54,7 +54,7 @@ __device__ __forceinline__ void warp_counts(const int32_t* __restrict__ ids, int
     const int f = w0 + r + lane;
     int e = -1;
     if (f < N) {
-      e = ids[f];
+      e = moe::ld_prod(ids + f);
       if (e < 0 || e >= E) {
         moe::report(status, MOE_ERR_BAD_INDEX);
         e = -1;
@@ -69,7 +69,7 @@ __device__ __forceinline__ void warp_counts(const int32_t* __restrict__ ids, int
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* __restrict__ ids,
+__global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* ids,
                                                              int N, int E,
                                                              int32_t* __restrict__ bc,
                                                              int32_t* status) {
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
   moe::grid_dep_wait();
   int total = 0;
   if (e < E)
-    for (int b = 0; b < B; ++b) total += bc[static_cast<size_t>(b) * E + e];
+    for (int b = 0; b < B; ++b) total += moe::ld_prod(bc + static_cast<size_t>(b) * E + e);
   // Exclusive scan over experts (Hillis-Steele on 256 entries).
   s_scan[e] = total;
   __syncthreads();
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
     int run = excl;
     for (int b = 0; b < B; ++b) {
       const size_t i = static_cast<size_t>(b) * E + e;
-      const int c = bc[i];
+      const int c = moe::ld_prod(bc + i);
       bc[i] = run;
       run += c;
     }
@@ -120,14 +120,14 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
 }
 
 __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ w, int N, int E, int k,
-    const int32_t* __restrict__ bc, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+    const int32_t* ids, const float* w, int N, int E, int k,
+    const int32_t* bc, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
     int32_t* __restrict__ packed_tok, float* __restrict__ packed_w, int32_t* status) {
   extern __shared__ int wc[];  // [DWARPS][E] counts, then bases
   const int base = blockIdx.x * CHUNK;
   warp_counts(ids, N, E, base, wc, nullptr);
   for (int e = threadIdx.x; e < E; e += DNT) {
-    int run = bc[static_cast<size_t>(blockIdx.x) * E + e];
+    int run = moe::ld_prod(bc + static_cast<size_t>(blockIdx.x) * E + e);
 #pragma unroll
     for (int ww = 0; ww < DWARPS; ++ww) {
       const int c = wc[ww * E + e];
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     const int f = w0 + r + lane;
     int e = -1;
     if (f < N) {
-      e = ids[f];
+      e = moe::ld_prod(ids + f);
       if (e < 0 || e >= E) {
         e = -1;
         inv_perm[f] = -1;
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
       perm[p] = f;
       inv_perm[f] = p;
       packed_tok[p] = f / k;
-      if (packed_w) packed_w[p] = w[f];
+      if (packed_w) packed_w[p] = moe::ld_prod(w + f);
     }
     __syncwarp();
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
@@ -172,10 +172,10 @@ constexpr int SMALL_PER_WARP = 256;
 constexpr int SMALL_N = SMALL_WARPS * SMALL_PER_WARP;   // 8192 assignments
 
 __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ w, int N, int E, int k,
+    const int32_t* ids, const float* w, int N, int E, int k,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv_perm, int32_t* __restrict__ packed_tok,
-    float* __restrict__ packed_w, const uint4* __restrict__ x, int row_vecs,
+    float* __restrict__ packed_w, const uint4* x, int row_vecs,
     uint4* __restrict__ xp, int32_t* status) {
   extern __shared__ int wc[];                  // [SMALL_WARPS][E]
   __shared__ int s_scan[moe::kMaxExperts];
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
 #pragma unroll
   for (int i = 0; i < ROUNDS; ++i) {
     const int f = w0 + 32 * i + lane;
-    eid[i] = f < w1 ? ids[f] : -1;
+    eid[i] = f < w1 ? moe::ld_prod(ids + f) : -1;
   }
   // 1. per-warp counts over this warp's contiguous slice
 #pragma unroll
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
       perm[p] = f;
       inv_perm[f] = p;
       packed_tok[p] = f / k;
-      if (packed_w) packed_w[p] = w[f];
+      if (packed_w) packed_w[p] = moe::ld_prod(w + f);
     }
     __syncwarp();
     if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
@@ -264,13 +264,13 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
   //    flight per lane before the stores
   const int nrows = s_scan[moe::kMaxExperts - 1];
   for (int p = warp; p < nrows; p += SMALL_WARPS) {
-    const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
+    const uint4* src = x + static_cast<size_t>(moe::ld_prod(packed_tok + p)) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
     for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
       uint4 q[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (v0 + 32 * j < row_vecs) q[j] = src[v0 + 32 * j];
+        if (v0 + 32 * j < row_vecs) q[j] = moe::ld_prod(src + v0 + 32 * j);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];
@@ -286,8 +286,8 @@ constexpr int GSLOTS = 4;  // rows in flight per warp
 // Rows [offsets[lo_e], offsets[hi_e]) of x_packed: every valid row for the
 // dispatcher (lo_e = 0, hi_e = E), one rank's experts for an expert range.
 __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
-    const uint8_t* __restrict__ x, const int32_t* __restrict__ packed_tok,
-    const int32_t* __restrict__ offsets, int lo_e, int hi_e, int row_bytes,
+    const uint8_t* x, const int32_t* packed_tok,
+    const int32_t* offsets, int lo_e, int hi_e, int row_bytes,
     uint8_t* __restrict__ xp, int32_t* status) {
   extern __shared__ __align__(128) uint8_t gsm[];
   __shared__ __align__(8) uint64_t bars[GW][GSLOTS];
@@ -298,8 +298,8 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
   moe::fence_barrier_init();
   moe::grid_dep_wait();
 
-  const int row0 = offsets[lo_e];
-  const int nrows = offsets[hi_e] - row0;  // valid rows (assignments with a valid id)
+  const int row0 = moe::ld_prod(offsets + lo_e);
+  const int nrows = moe::ld_prod(offsets + hi_e) - row0;  // valid rows (assignments with a valid id)
   const int stride = gridDim.x * GW;
   const int first = blockIdx.x * GW + warp;
   const int mine = first < nrows ? (nrows - first + stride - 1) / stride : 0;
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
     const uint32_t bar = moe::smem_addr(&bars[warp][s]);
     moe::mbar_arrive_expect_tx(bar, row_bytes);
     moe::bulk_g2s(moe::smem_addr(ring + static_cast<size_t>(s) * row_bytes),
-                  x + static_cast<size_t>(packed_tok[p]) * row_bytes, row_bytes, bar);
+                  x + static_cast<size_t>(moe::ld_prod(packed_tok + p)) * row_bytes, row_bytes, bar);
   };
   const int prologue = mine < GSLOTS ? mine : GSLOTS;
   for (int i = 0; i < prologue; ++i) issue(i);
@@ -338,21 +338,21 @@ __global__ void __launch_bounds__(GW * 32) dispatch_gather_kernel(
 
 // Rows too large for the shared-memory ring: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256) dispatch_gather_vec_kernel(
-    const uint4* __restrict__ x, const int32_t* __restrict__ packed_tok,
-    const int32_t* __restrict__ offsets, int lo_e, int hi_e, int row_vecs,
+    const uint4* x, const int32_t* packed_tok,
+    const int32_t* offsets, int lo_e, int hi_e, int row_vecs,
     uint4* __restrict__ xp) {
   moe::grid_dep_wait();
-  const int row_end = offsets[hi_e];
+  const int row_end = moe::ld_prod(offsets + hi_e);
   const int lane = threadIdx.x & 31;
-  for (int p = offsets[lo_e] + ((blockIdx.x * blockDim.x + threadIdx.x) >> 5); p < row_end;
-       p += (gridDim.x * blockDim.x) >> 5) {
-    const uint4* src = x + static_cast<size_t>(packed_tok[p]) * row_vecs;
+  for (int p = moe::ld_prod(offsets + lo_e) + ((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+       p < row_end; p += (gridDim.x * blockDim.x) >> 5) {
+    const uint4* src = x + static_cast<size_t>(moe::ld_prod(packed_tok + p)) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
     for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
       uint4 q[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (v0 + 32 * j < row_vecs) q[j] = src[v0 + 32 * j];
+        if (v0 + 32 * j < row_vecs) q[j] = moe::ld_prod(src + v0 + 32 * j);
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];

@@ -34,7 +34,7 @@ __device__ __forceinline__ bool is_local(int32_t id, uint32_t lo, uint32_t hi) {
   return u >= lo && u < hi;
 }
 
-__global__ void __launch_bounds__(EP_NT) ep_count_kernel(const int32_t* __restrict__ ids, int n,
+__global__ void __launch_bounds__(EP_NT) ep_count_kernel(const int32_t* ids, int n,
                                                          uint32_t lo, uint32_t hi,
                                                          int32_t* __restrict__ block_local) {
   __shared__ int s_warp[EP_NT / 32];
@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(EP_NT) ep_count_kernel(const int32_t* __restri
   int c = 0;
   for (int i = threadIdx.x; i < EP_CHUNK; i += EP_NT) {
     const int f = base + i;
-    if (f < n && is_local(ids[f], lo, hi)) ++c;
+    if (f < n && is_local(moe::ld_prod(ids + f), lo, hi)) ++c;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
@@ -59,8 +59,8 @@ __global__ void __launch_bounds__(EP_NT) ep_count_kernel(const int32_t* __restri
 }
 
 __global__ void __launch_bounds__(EP_NT) ep_scatter_kernel(
-    const int32_t* __restrict__ ids, const float* __restrict__ w, int n, int top_k, uint32_t lo,
-    uint32_t hi, const int32_t* __restrict__ block_local, int32_t* __restrict__ l_tok,
+    const int32_t* ids, const float* w, int n, int top_k, uint32_t lo,
+    uint32_t hi, const int32_t* block_local, int32_t* __restrict__ l_tok,
     int32_t* __restrict__ l_eid, float* __restrict__ l_w, int32_t* __restrict__ r_tok,
     int32_t* __restrict__ r_eid, float* __restrict__ r_w, int32_t* __restrict__ bucket_counts) {
   __shared__ int s_warp[EP_NT / 32];
@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(EP_NT) ep_scatter_kernel(
   // First local position of this CTA: the local entries of all earlier CTAs.
   int before = 0;
   if (block_local != nullptr)
-    for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += EP_NT) before += block_local[b];
+    for (int b = threadIdx.x; b < static_cast<int>(blockIdx.x); b += EP_NT)
+      before += moe::ld_prod(block_local + b);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
   if (lane == 0) s_warp[warp] = before;
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(EP_NT) ep_scatter_kernel(
 #pragma unroll
   for (int i = 0; i < EP_PER; ++i) {
     const int f = f0 + i;
-    id[i] = f < n ? ids[f] : 0;
+    id[i] = f < n ? moe::ld_prod(ids + f) : 0;
     if (f < n && is_local(id[i], lo, hi)) ++mine;
   }
   // Block-wide exclusive scan of the per-thread local counts.
@@ -116,12 +117,12 @@ __global__ void __launch_bounds__(EP_NT) ep_scatter_kernel(
     if (is_local(id[i], lo, hi)) {
       l_tok[lp] = tok;
       l_eid[lp] = id[i];
-      l_w[lp] = w[f];
+      l_w[lp] = moe::ld_prod(w + f);
       ++lp;
     } else {
       r_tok[rp] = tok;
       r_eid[rp] = id[i];
-      r_w[rp] = w[f];
+      r_w[rp] = moe::ld_prod(w + f);
       ++rp;
     }
   }
@@ -145,12 +146,12 @@ __device__ __forceinline__ int owner_of(int id, int E, int R) {
   return static_cast<int>((static_cast<long long>(R) * (id + 1) - 1) / E);
 }
 
-__global__ void __launch_bounds__(256) ep_owner_kernel(const int32_t* __restrict__ ids, int n,
+__global__ void __launch_bounds__(256) ep_owner_kernel(const int32_t* ids, int n,
                                                        int E, int R, int32_t* __restrict__ owner,
                                                        int32_t* status) {
   moe::grid_dep_wait();
   for (int f = blockIdx.x * 256 + threadIdx.x; f < n; f += gridDim.x * 256) {
-    const int id = ids[f];
+    const int id = moe::ld_prod(ids + f);
     if (id < 0 || id >= E) {
       moe::report(status, MOE_ERR_BAD_INDEX);
       owner[f] = -1;                         // left out by the dispatcher, reported there too
@@ -163,15 +164,15 @@ __global__ void __launch_bounds__(256) ep_owner_kernel(const int32_t* __restrict
 
 // local[p] = ids[perm[p]] - (first expert of its owner), for the rows
 // p < offsets[R] that a dispatch by owner wrote.
-__global__ void __launch_bounds__(256) ep_pack_ids_kernel(const int32_t* __restrict__ ids,
-                                                          const int32_t* __restrict__ perm,
-                                                          const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(256) ep_pack_ids_kernel(const int32_t* ids,
+                                                          const int32_t* perm,
+                                                          const int32_t* offsets,
                                                           int E, int R,
                                                           int32_t* __restrict__ local) {
   moe::grid_dep_wait();
-  const int nrows = offsets[R];
+  const int nrows = moe::ld_prod(offsets + R);
   for (int p = blockIdx.x * 256 + threadIdx.x; p < nrows; p += gridDim.x * 256) {
-    const int id = ids[perm[p]];
+    const int id = moe::ld_prod(ids + moe::ld_prod(perm + p));
     const int q = owner_of(id, E, R);
     local[p] = id - static_cast<int>(static_cast<long long>(E) * q / R);
   }

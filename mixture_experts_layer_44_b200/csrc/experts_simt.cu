@@ -26,22 +26,23 @@ __device__ void build_tiles(const int32_t* offsets, int E, int* offs, int* tstar
   if (threadIdx.x == 0) {
     int run = 0;
     for (int e = 0; e < E; ++e) {
-      offs[e] = offsets[e];
+      const int o0 = moe::ld_prod(offsets + e), o1 = moe::ld_prod(offsets + e + 1);
+      offs[e] = o0;
       tstart[e] = run;
-      run += (offsets[e + 1] - offsets[e] + SBM - 1) / SBM;
+      run += (o1 - o0 + SBM - 1) / SBM;
     }
-    offs[E] = offsets[E];
+    offs[E] = moe::ld_prod(offsets + E);
     tstart[E] = run;
   }
   __syncthreads();
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* __restrict__ A, int K,
-                                                        const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* A, int K,
+                                                        const int32_t* offsets,
                                                         int E, const float* __restrict__ B,
                                                         int rows_per_expert, int I,
-                                                        const float* __restrict__ pw,
+                                                        const float* pw,
                                                         float* __restrict__ out, int ldo) {
   __shared__ int offs[moe::kMaxExperts + 1];
   __shared__ int tstart[moe::kMaxExperts + 1];
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* __restrict_
     for (int i = threadIdx.x; i < SBM * SBK; i += SNT) {
       const int r = i / SBK, kk = i % SBK;
       const int gr = r0 + r, gk = k0 + kk;
-      As[kk][r] = (gr < rend && gk < K) ? A[static_cast<size_t>(gr) * K + gk] : 0.f;
+      As[kk][r] = (gr < rend && gk < K) ? moe::ld_prod(A + static_cast<size_t>(gr) * K + gk) : 0.f;
     }
     for (int i = threadIdx.x; i < NB * SBK; i += SNT) {
       const int r = i / SBK, kk = i % SBK;
@@ -105,7 +106,7 @@ __global__ void __launch_bounds__(SNT) simt_gemm_kernel(const float* __restrict_
   for (int i = 0; i < 4; ++i) {
     const int gr = r0 + ty * 4 + i;
     if (gr >= rend) continue;
-    const float sc = EPI == EPI_SCALE ? (pw ? pw[gr] : 1.f) : 1.f;
+    const float sc = EPI == EPI_SCALE ? (pw ? moe::ld_prod(pw + gr) : 1.f) : 1.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int gc = c0 + tx * 4 + j;

@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const __grid_constant__ CUtensorMap tmY,
                         const __grid_constant__ CUtensorMap tmY2,
                         const int32_t* __restrict__ offsets, int E, int K, int ntw,
-                        int rows_per_expert, const float* __restrict__ packed_w,
+                        int rows_per_expert, const float* packed_w,
                         void* __restrict__ out, int ldo, int rows2, int K2, int ntw2,
                         void* __restrict__ out2, int ldo2, int* __restrict__ counters,
                         float* __restrict__ partials, int max_units, int32_t* status,
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // hands the 32 x 32 block to the TMA engine, so no thread waits on
           // global stores and no barrier spans the warps; a partly valid
           // quarter stores its valid rows directly.
-          const float sc = live ? (upw ? upw[grow] : 1.f) : 0.f;
+          const float sc = live ? (upw ? moe::ld_prod(upw + grow) : 1.f) : 0.f;
           uint8_t* gtile =
               static_cast<uint8_t*>(uout) + (row0 * uldo + un.nt * BN) * sizeof(float);
           const int qrows = min(max(nvalid - q * 32, 0), 32);
@@ -801,7 +801,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
                 }
               }
-              const float sc = upw ? upw[row0 + r] : 1.f;
+              const float sc = upw ? moe::ld_prod(upw + row0 + r) : 1.f;
               *reinterpret_cast<float4*>(static_cast<float*>(uout) + (row0 + r) * uldo +
                                          un.nt * BN + cg * 4) =
                   make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);

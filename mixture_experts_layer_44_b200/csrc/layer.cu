@@ -228,8 +228,10 @@ int moe_layer_create(const moe_layer_desc* d, void* workspace, size_t workspace_
     so[0] = 0;
     so[1] = d->T;
     e = cudaMemcpyAsync(L->sh_offsets, so, 8, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);   // `so` must outlive the copy
   }
+  // Set-up done before the first forward call can be enqueued (and `so` must
+  // outlive its copy).
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   const unsigned fl = cudaStreamNonBlocking;
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->s_in, fl);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->s_comp, fl);

@@ -37,6 +37,8 @@ constexpr int KC = 32;    // H chunk
 constexpr int NT = 256;   // threads per CTA
 constexpr int MAX_S = 8;  // CTAs per cluster
 
+// Eight elements at base + off (activations may come from the kernel before:
+// read at L2, see moe::ld_prod).
 template <bool BF16>
 __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, float* f) {
   if (!ok) {
@@ -45,11 +47,12 @@ __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, flo
     return;
   }
   if (BF16) {
-    const uint4 q = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + off);
+    const uint4 q =
+        moe::ld_prod(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + off));
     moe::unpack8(q, f);
   } else {
     const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
-    const float4 a = p[0], b = p[1];
+    const float4 a = moe::ld_prod(p), b = moe::ld_prod(p + 1);
     f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
   }
@@ -68,7 +71,7 @@ __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, flo
 constexpr int NS = 512;   // threads per CTA of the small-batch router
 
 template <int EP, bool BF16>
-__global__ void __launch_bounds__(NS) route_small_kernel(const void* __restrict__ xv,
+__global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
                                                          const void* __restrict__ wv,
                                                          const float* __restrict__ bias, int H,
                                                          int E, int k, int renorm,
@@ -188,7 +191,7 @@ struct Tile {
 };
 
 template <int EPAD, bool BF16>
-__global__ void __launch_bounds__(NT) route_kernel(const void* __restrict__ xv,
+__global__ void __launch_bounds__(NT) route_kernel(const void* xv,
                                                    const void* __restrict__ wv,
                                                    const float* __restrict__ bias, int T, int H,
                                                    int E, int k, int renorm, int kc_per_cta,
