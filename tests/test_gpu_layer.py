@@ -87,6 +87,8 @@ def test_tiny_f32_every_stage_and_every_token():
 
 # y_packed against the oracle's second product fed the GPU's own h: the
 # tensor cores' fp32 accumulation over K = I terms is all that separates them.
+# Measured at full size: 8e-6 (decode, T = 1) to 1.3e-4 (decode, T = 64, K =
+# 14336 split in 16 slices); the bound leaves a margin of ~8x over the worst.
 STAGED_Y_TOL = 1e-3
 
 FULL = ["builder_bf16", "qwen15_t32", "qwen15_t8192", "qwen3_t16384", "decode_t1", "decode_t8",
