@@ -193,6 +193,37 @@ int moe_dispatch_noalloc(const int32_t* topk_ids, const float* topk_w, const voi
                          int32_t* packed_tok, float* packed_w, void* x_packed,
                          int32_t* status, void* stream);
 
+/*
+ * moe_route_dispatch -- moe_route_grouped followed by moe_dispatch, in one
+ * launch, for small batches (decode).  The Router and the Dispatcher of the
+ * DWDP README ("Router Module", "Dispatcher Module", chained as its "Runtime
+ * Integration Layer" gives) produce exactly the outputs of the two separate
+ * calls on the same arguments (bit for bit: the same routing arithmetic and
+ * the same stable order).
+ *
+ * One CTA per token routes it; the CTA that finishes last (found with an
+ * atomic ticket on `counter`: no CTA waits for another) then counts, scans
+ * and scatters all T*k assignments, and gathers x_packed when the rows total
+ * at most 128 KiB (a second, multi-CTA gather kernel otherwise).
+ *
+ *   Arguments as moe_route_grouped (n_groups = 1: plain top-k) and
+ *   moe_dispatch, with topk_ids / topk_w as the routed outputs it writes and
+ *   then reads back (both required, k >= 1).
+ *   x_packed  device [N,H] (dtype), or NULL to skip the gather.
+ *   counter   device int32, zero before the first call; every call leaves it
+ *             at zero again.  Calls that may overlap on the GPU (different
+ *             streams) need different counters.
+ *   Needs 1 <= T <= 64, 1 <= E <= 64, H <= 32768 and 1 <= k <= min(E, 8):
+ *   other shapes return MOE_ERR_INVALID_ARG (use the two separate calls).
+ *   No workspace.
+ */
+int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
+                       int k, int renormalize, int n_groups, int topk_groups, int dtype,
+                       float* logits, int32_t* topk_ids, float* topk_w,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
+                       int32_t* packed_tok, float* packed_w, void* x_packed,
+                       int32_t* counter, int32_t* status, void* stream);
+
 /* Bytes of device scratch moe_experts can use (bf16 path: per-tile counters
  * plus 128 KiB partial slots, 4 per SM; fp32 path: 0). */
 size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);

@@ -70,6 +70,8 @@ _SIGS = {
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "moe_route_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                                _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_layer_workspace_bytes": (_SZ, [_P]),
     "moe_test_set_wait_budget_ns": (_I, [ctypes.c_ulonglong]),
     "moe_layer_create": (_I, [_P, _P, _SZ, _P, _P]),
@@ -162,6 +164,25 @@ def moe_route_grouped(x, W_gate, bias, k: int, renormalize: bool, n_groups: int,
         _ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k, int(bool(renormalize)), n_groups,
         topk_groups, _dtype_code(x), _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _ptr(status),
         _stream(stream)))
+
+
+def route_dispatch_fits(T: int, H: int, E: int, k: int) -> bool:
+    """Shapes moe_route_dispatch takes (one launch for router + dispatcher)."""
+    return 1 <= T <= 64 and 1 <= E <= 64 and H <= 32768 and 1 <= k <= min(E, 8)
+
+
+def moe_route_dispatch(x, W_gate, bias, k: int, renormalize: bool, logits, topk_ids, topk_w,
+                       counts, offsets, perm, inv_perm, packed_tok, packed_w, x_packed, counter,
+                       status=None, stream=None, n_groups: int = 1, topk_groups: int = 1):
+    """moe_route_grouped then moe_dispatch in one launch (T <= 64, E <= 64).
+    ``counter``: one int32 on the device, zero before the first call."""
+    T, H = x.shape
+    E = W_gate.shape[0]
+    _check(load_library().moe_route_dispatch(
+        _ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k, int(bool(renormalize)), n_groups,
+        topk_groups, _dtype_code(x), _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _ptr(counts),
+        _ptr(offsets), _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w),
+        _ptr(x_packed), _ptr(counter), _ptr(status), _stream(stream)))
 
 
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
@@ -430,6 +451,8 @@ class MoELayerBuffers:
             max(16, moe_experts_workspace_bytes(N, H, I, E, MOE_BF16 if dtype == torch.bfloat16
                                                 else MOE_F32)), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
+        self.rd_counter = torch.zeros(1, **i32)    # ticket of moe_route_dispatch
+        self.route_dispatch = route_dispatch_fits(T, H, E, k)
         self.shared_I = shared_I
         # bf16 tensor-core layers run the shared expert inside the routed launches
         self.fuse_shared = bool(shared_I) and dtype == torch.bfloat16 and H % 256 == 0 and \
@@ -441,15 +464,18 @@ class MoELayerBuffers:
             self.sh_y = torch.empty(T, H, **f32)
 
 
-def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
-                      stream=None, n_groups: int = 1, topk_groups: int = 1):
-    """Router -> dispatcher -> executor -> merger into ``buf.out`` (asynchronous).
-
-    ``params``: W_gate [E,H], bias [E] f32 or None, w13 [E,2I,H], w2 [E,H,I] and,
-    for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].  n_groups > 1
-    routes group-limited (moe_route_grouped).
-    """
+def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
+                       stream=None, n_groups: int = 1, topk_groups: int = 1):
+    """Router then dispatcher into ``buf``: one launch for decode batches
+    (moe_route_dispatch), else moe_route[_grouped] and moe_dispatch."""
     E = params["W_gate"].shape[0]
+    if buf.route_dispatch:
+        moe_route_dispatch(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits,
+                           buf.ids, buf.w, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
+                           buf.packed_tok, buf.packed_w, buf.x_packed, buf.rd_counter,
+                           status=buf.status, stream=stream, n_groups=n_groups,
+                           topk_groups=topk_groups)
+        return
     if n_groups > 1:
         moe_route_grouped(x, params["W_gate"], params.get("bias"), k, renormalize, n_groups,
                           topk_groups, buf.logits, buf.ids, buf.w, status=buf.status,
@@ -459,6 +485,18 @@ def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerB
                   buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
+
+
+def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
+                      stream=None, n_groups: int = 1, topk_groups: int = 1):
+    """Router -> dispatcher -> executor -> merger into ``buf.out`` (asynchronous).
+
+    ``params``: W_gate [E,H], bias [E] f32 or None, w13 [E,2I,H], w2 [E,H,I] and,
+    for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].  n_groups > 1
+    routes group-limited (moe_route_grouped).
+    """
+    E = params["W_gate"].shape[0]
+    route_and_dispatch(x, params, k, renormalize, buf, stream, n_groups, topk_groups)
     shared = sg = None
     if params.get("w13s") is None:
         moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,

@@ -185,6 +185,47 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x, in
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch launch");
 }
 
+int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
+                       int k, int renormalize, int n_groups, int topk_groups, int dtype,
+                       float* logits, int32_t* topk_ids, float* topk_w, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
+                       float* packed_w, void* x_packed, int32_t* counter, int32_t* status,
+                       void* stream) {
+  g_err.clear();
+  if (int r = check_dtype(dtype)) return r;
+  const std::string f = "moe_route_dispatch: ";
+  REQ(x && W_gate && logits && topk_ids && topk_w, MOE_ERR_INVALID_ARG,
+      f + "null x, W_gate, logits, topk_ids or topk_w");
+  REQ(counts && offsets && perm && inv_perm && packed_tok && packed_w && counter,
+      MOE_ERR_INVALID_ARG, f + "null dispatch output or counter");
+  REQ(T >= 1 && T <= 64, MOE_ERR_INVALID_ARG, f + "T must be in [1, 64]");
+  REQ(E >= 1 && E <= 64, MOE_ERR_INVALID_ARG, f + "E must be in [1, 64]");
+  REQ(H >= 8 && H % 8 == 0 && H <= 32768, MOE_ERR_INVALID_ARG,
+      f + "H must be a multiple of 8 in [8, 32768]");
+  REQ(k >= 1 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
+      f + "k must be in [1, min(E, 8)]");
+  REQ(n_groups >= 1, MOE_ERR_INVALID_ARG, f + "n_groups must be >= 1");
+  if (n_groups > 1) {
+    REQ(n_groups <= 32 && E % n_groups == 0, MOE_ERR_INVALID_ARG,
+        f + "n_groups must divide E and be at most 32");
+    REQ(topk_groups >= 1 && topk_groups <= n_groups, MOE_ERR_INVALID_ARG,
+        f + "topk_groups must be in [1, n_groups]");
+    REQ(k <= topk_groups * (E / n_groups), MOE_ERR_INVALID_ARG,
+        f + "k must be in [1, topk_groups * E / n_groups]");
+  }
+  REQ(aligned16(x) && aligned16(W_gate) && aligned16(x_packed), MOE_ERR_INVALID_ARG,
+      f + "x, W_gate and x_packed must be 16-byte aligned");
+  REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias) &&
+          aligned4(counts) && aligned4(offsets) && aligned4(perm) && aligned4(inv_perm) &&
+          aligned4(packed_tok) && aligned4(packed_w) && aligned4(counter) && aligned4(status),
+      MOE_ERR_INVALID_ARG, f + "index arrays, bias, counter and status must be 4-byte aligned");
+  cudaError_t e = moe_host::launch_route_dispatch(
+      x, W_gate, bias, T, H, E, k, renormalize != 0, dtype, logits, topk_ids, topk_w, counts,
+      offsets, perm, inv_perm, packed_tok, packed_w, x_packed, counter, status,
+      static_cast<cudaStream_t>(stream), n_groups, n_groups > 1 ? topk_groups : 1);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_dispatch launch");
+}
+
 size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype) {
   (void)N; (void)H; (void)I; (void)E;
   return dtype == MOE_BF16 ? moe_host::experts_ws_bytes() : 0;

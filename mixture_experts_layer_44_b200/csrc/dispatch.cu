@@ -32,6 +32,7 @@
 #include <string>
 
 #include "common.cuh"
+#include "dispatch_cta.cuh"
 #include "sm100_ptx.cuh"
 
 namespace {
@@ -179,103 +180,12 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
     uint4* __restrict__ xp, int32_t* status) {
   extern __shared__ int wc[];                  // [SMALL_WARPS][E]
   __shared__ int s_scan[moe::kMaxExperts];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
   for (int i = threadIdx.x; i < SMALL_WARPS * E; i += blockDim.x) wc[i] = 0;
   moe::grid_dep_wait();
   __syncthreads();
-  const int per = (N + SMALL_WARPS - 1) / SMALL_WARPS;
-  const int w0 = warp * per, w1 = min(N, w0 + per);
-  // The warp's slice of ids, read once (all loads in flight together) and
-  // kept in registers for both passes; -1 marks no assignment / a bad id.
-  constexpr int ROUNDS = SMALL_PER_WARP / 32;
-  const int nr = w1 > w0 ? (w1 - w0 + 31) / 32 : 0;   // rounds this warp needs
-  int eid[ROUNDS];
-#pragma unroll
-  for (int i = 0; i < ROUNDS; ++i) {
-    const int f = w0 + 32 * i + lane;
-    eid[i] = f < w1 ? moe::ld_prod(ids + f) : -1;
-  }
-  // 1. per-warp counts over this warp's contiguous slice
-#pragma unroll
-  for (int i = 0; i < ROUNDS; ++i) {
-    if (i >= nr) break;
-    const int f = w0 + 32 * i + lane;
-    if (f < w1 && (eid[i] < 0 || eid[i] >= E)) {
-      moe::report(status, MOE_ERR_BAD_INDEX);
-      inv_perm[f] = -1;
-      eid[i] = -1;
-    }
-    const int e = eid[i];
-    const int key = e >= 0 ? e : -1 - lane;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
-  }
-  __syncthreads();
-  // 2. counts, exclusive scan over experts, per-warp bases
-  const int e = threadIdx.x;
-  int total = 0;
-  if (e < E)
-    for (int ww = 0; ww < SMALL_WARPS; ++ww) total += wc[ww * E + e];
-  if (e < moe::kMaxExperts) s_scan[e] = total;
-  __syncthreads();
-  for (int o = 1; o < moe::kMaxExperts; o <<= 1) {
-    const int v = (e < moe::kMaxExperts && e >= o) ? s_scan[e - o] : 0;
-    __syncthreads();
-    if (e < moe::kMaxExperts) s_scan[e] += v;
-    __syncthreads();
-  }
-  if (e < E) {
-    const int excl = s_scan[e] - total;
-    counts[e] = total;
-    offsets[e] = excl;
-    int run = excl;
-    for (int ww = 0; ww < SMALL_WARPS; ++ww) {
-      const int c = wc[ww * E + e];
-      wc[ww * E + e] = run;
-      run += c;
-    }
-  }
-  if (e == 0) offsets[E] = s_scan[moe::kMaxExperts - 1];
-  __syncthreads();
-  // 3. stable scatter: slices in warp order, rounds in order, lanes in order
-#pragma unroll
-  for (int i = 0; i < ROUNDS; ++i) {
-    if (i >= nr) break;
-    const int f = w0 + 32 * i + lane;
-    const int ex = eid[i];
-    const int key = ex >= 0 ? ex : -1 - lane;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (ex >= 0) {
-      const int p = wc[warp * E + ex] + __popc(peers & lt);
-      perm[p] = f;
-      inv_perm[f] = p;
-      packed_tok[p] = f / k;
-      if (packed_w) packed_w[p] = moe::ld_prod(w + f);
-    }
-    __syncwarp();
-    if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
-    __syncwarp();
-  }
-  moe::grid_dep_launch();
-  if (x == nullptr) return;
-  __syncthreads();
-  // 4. gather (small total): one warp per row, 16-byte vectors, 8 loads in
-  //    flight per lane before the stores
-  const int nrows = s_scan[moe::kMaxExperts - 1];
-  for (int p = warp; p < nrows; p += SMALL_WARPS) {
-    const uint4* src = x + static_cast<size_t>(moe::ld_prod(packed_tok + p)) * row_vecs;
-    uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
-    for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
-      uint4 q[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (v0 + 32 * j < row_vecs) q[j] = moe::ld_prod(src + v0 + 32 * j);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];
-    }
-  }
+  moe::dispatch_cta<SMALL_WARPS, SMALL_PER_WARP / 32>(ids, w, N, E, k, counts, offsets, perm,
+                                                      inv_perm, packed_tok, packed_w, x,
+                                                      row_vecs, xp, status, wc, s_scan);
 }
 
 // ------------------------------------------------------------- gather ---

@@ -1,0 +1,121 @@
+// One CTA dispatching a small batch: per-warp counts, exclusive scan over the
+// experts, stable scatter, and (when given x) the gather of the rows.
+//
+// DWDP-Triton-MoE-Inference-Engine README, "Dispatcher Module" and "Executor
+// Module" (gather token activations).  Inside an expert the assignments keep
+// ascending f = t*k + j, the flat order of metrale's ep_dispatch.rs
+// (build_ep_routing_table).  Warp w owns a contiguous slice of the N
+// assignments; inside a 32-lane round a lane's rank among equal experts is the
+// popcount of the lower lanes in its match mask, so positions grow with f
+// inside an expert and the result does not depend on the warp count.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// NW warps; up to NW * 32 * ROUNDS assignments.  wc: shared [NW][E], zeroed
+// by the caller before a __syncthreads; s_scan: shared [kMaxExperts].  Every
+// thread of the CTA calls this (it synchronises the CTA).  Ids outside [0,E)
+// are reported (MOE_ERR_BAD_INDEX), given inv_perm -1 and left out.
+template <int NW, int ROUNDS>
+__device__ __forceinline__ void dispatch_cta(
+    const int32_t* ids, const float* w, int N, int E, int k, int32_t* counts, int32_t* offsets,
+    int32_t* perm, int32_t* inv_perm, int32_t* packed_tok, float* packed_w, const uint4* x,
+    int row_vecs, uint4* xp, int32_t* status, int* wc, int* s_scan) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int per = (N + NW - 1) / NW;
+  const int w0 = warp * per, w1 = min(N, w0 + per);
+  // The warp's slice of ids, read once (all loads in flight together) and
+  // kept in registers for both passes; -1 marks no assignment / a bad id.
+  const int nr = w1 > w0 ? (w1 - w0 + 31) / 32 : 0;   // rounds this warp needs
+  int eid[ROUNDS];
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    const int f = w0 + 32 * i + lane;
+    eid[i] = f < w1 ? ld_prod(ids + f) : -1;
+  }
+  // 1. per-warp counts over this warp's contiguous slice
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    if (i >= nr) break;
+    const int f = w0 + 32 * i + lane;
+    if (f < w1 && (eid[i] < 0 || eid[i] >= E)) {
+      report(status, MOE_ERR_BAD_INDEX);
+      inv_perm[f] = -1;
+      eid[i] = -1;
+    }
+    const int e = eid[i];
+    const int key = e >= 0 ? e : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
+  }
+  __syncthreads();
+  // 2. counts, exclusive scan over experts, per-warp bases (blockDim >= 256)
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int ww = 0; ww < NW; ++ww) total += wc[ww * E + e];
+  if (e < kMaxExperts) s_scan[e] = total;
+  __syncthreads();
+  for (int o = 1; o < kMaxExperts; o <<= 1) {
+    const int v = (e < kMaxExperts && e >= o) ? s_scan[e - o] : 0;
+    __syncthreads();
+    if (e < kMaxExperts) s_scan[e] += v;
+    __syncthreads();
+  }
+  if (e < E) {
+    const int excl = s_scan[e] - total;
+    counts[e] = total;
+    offsets[e] = excl;
+    int run = excl;
+    for (int ww = 0; ww < NW; ++ww) {
+      const int c = wc[ww * E + e];
+      wc[ww * E + e] = run;
+      run += c;
+    }
+  }
+  if (e == 0) offsets[E] = s_scan[kMaxExperts - 1];
+  __syncthreads();
+  // 3. stable scatter: slices in warp order, rounds in order, lanes in order
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    if (i >= nr) break;
+    const int f = w0 + 32 * i + lane;
+    const int ex = eid[i];
+    const int key = ex >= 0 ? ex : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (ex >= 0) {
+      const int p = wc[warp * E + ex] + __popc(peers & lt);
+      perm[p] = f;
+      inv_perm[f] = p;
+      packed_tok[p] = f / k;
+      if (packed_w) packed_w[p] = ld_prod(w + f);
+    }
+    __syncwarp();
+    if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
+    __syncwarp();
+  }
+  grid_dep_launch();
+  if (x == nullptr) return;
+  __syncthreads();
+  // 4. gather (small total): one warp per row, 16-byte vectors, 8 loads in
+  //    flight per lane before the stores
+  const int nrows = s_scan[kMaxExperts - 1];
+  for (int p = warp; p < nrows; p += NW) {
+    const uint4* src = x + static_cast<size_t>(ld_prod(packed_tok + p)) * row_vecs;
+    uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
+    for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) q[j] = ld_prod(src + v0 + 32 * j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (v0 + 32 * j < row_vecs) dst[v0 + 32 * j] = q[j];
+    }
+  }
+}
+
+}  // namespace moe

@@ -85,6 +85,11 @@ constexpr int NTHREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
 constexpr int MAX_SPLITS = 16;
+// Weights that one unit alone reads (an expert whose rows fit one token tile:
+// decode batches) stream from HBM exactly once, and the stage ring alone
+// keeps too few bytes in flight per SM to reach full bandwidth.  Such units
+// also ask L2 for the k-block L2_AHEAD ahead of each one they load.
+constexpr int L2_AHEAD = 4;
 constexpr int COUNTER_INTS = 4096;                        // per-tile arrival counters, then
 constexpr int SCHED_TICKET = COUNTER_INTS - 2;            // the unit ticket and the
 constexpr int SCHED_DONE = COUNTER_INTS - 1;              // CTA exit count of dynamic scheduling
@@ -126,6 +131,7 @@ constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTL_BYTES + STAGE_OU
 // its own input), group 0 the routed experts.  Its rows are [row0, rend).
 struct Unit {
   int tile, g, e, nt, mt, ks, S, kb0, kb1, row0, rend;
+  bool stream;   // the group's rows fit one token tile: no other unit reads these weights
 };
 
 template <bool SHARED>
@@ -154,6 +160,7 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     r.mt = r.tile - r.nt * c.mte2;
     r.row0 = r.mt * BM;
     r.rend = c.rows2;
+    r.stream = c.mte2 == 1;
     kb = kblocks2;
   } else {
     // largest e with tstart[e] <= tile (experts without tiles share their successor's start)
@@ -170,6 +177,7 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     r.mt = local - r.nt * mte;
     r.row0 = c.offs[r.e] + r.mt * BM;
     r.rend = c.offs[r.e + 1];
+    r.stream = mte == 1;
     kb = kblocks;
   }
   r.kb0 = (r.ks * kb) / r.S;
@@ -435,6 +443,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   };
 
+  // The same k-block of the B operand, requested into L2 only.
+  auto prefetch_b = [&](const Unit& un, int kb) {
+    if (SHARED && un.g) {
+      if (EPI == EPI_SWIGLU)
+        moe::tma_prefetch_3d(&tmB2, kb * BK, un.nt * (BN / 2), 0);
+      else
+        moe::tma_prefetch_2d(&tmB2, kb * BK, un.nt * BN);
+    } else if (EPI == EPI_SWIGLU) {
+      moe::tma_prefetch_3d(&tmB, kb * BK, un.nt * (BN / 2), 2 * un.e);
+    } else {
+      moe::tma_prefetch_2d(&tmB, kb * BK, un.e * rows_per_expert + un.nt * BN);
+    }
+  };
+
   // Pass 2, before waiting for pass 1: the weights of this CTA's first unit
   // (static: unit blockIdx.x) into the first stages, and the next k-blocks
   // into L2.  Each such stage's barrier expects the whole stage; the A half
@@ -451,12 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       pre_issued[s] = 1;
     }
     const int l2_end = min(un.kb1, un.kb0 + pre + 8);
-    for (int kb = un.kb0 + pre; kb < l2_end; ++kb) {
-      if (SHARED && un.g)
-        moe::tma_prefetch_2d(&tmB2, kb * BK, un.nt * BN);
-      else
-        moe::tma_prefetch_2d(&tmB, kb * BK, un.e * rows_per_expert + un.nt * BN);
-    }
+    for (int kb = un.kb0 + pre; kb < l2_end; ++kb) prefetch_b(un, kb);
   }
   if (EARLY) moe::grid_dep_wait();               // h comes from pass 1
 
@@ -513,6 +530,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
             load_b(un, kb, sa, fb);
             ++issued[stage];
+            if (L2_AHEAD > 0 && un.stream && kb + L2_AHEAD < un.kb1) prefetch_b(un, kb + L2_AHEAD);
           }
           if (++stage == STAGES) {
             stage = 0;

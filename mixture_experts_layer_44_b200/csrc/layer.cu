@@ -43,6 +43,7 @@ struct moe_layer {
   void* ews;
   size_t ews_bytes;
   int32_t* status;
+  int32_t* counter;              // ticket of the fused small-batch route+dispatch
   float* sg_logit;
   void* sh_h;
   float* sh_y;
@@ -92,7 +93,8 @@ size_t layout(moe_layer* L, uint8_t* base) {
   L->dws = c.take(L->dws_bytes);
   L->ews_bytes = d.dtype == MOE_BF16 ? moe_host::experts_ws_bytes() : 0;
   L->ews = L->ews_bytes ? c.take(L->ews_bytes) : nullptr;
-  L->status = static_cast<int32_t*>(c.take(4));
+  L->status = static_cast<int32_t*>(c.take(8));   // status, then the route+dispatch ticket
+  L->counter = L->status + 1;
   if (d.w13s != nullptr) {
     L->sg_logit = static_cast<float*>(c.take(T * 4));
     L->sh_h = c.take(T * static_cast<size_t>(d.I_s) * es);
@@ -130,14 +132,24 @@ const char* check_desc(const moe_layer_desc* d) {
 
 cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
   const moe_layer_desc& d = L->d;
-  cudaError_t e = moe_host::launch_route(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k,
-                                         d.renormalize != 0, d.dtype, L->logits, L->ids, L->w,
-                                         L->status, s, d.n_groups > 1 ? d.n_groups : 1,
-                                         d.topk_groups);
-  if (e != cudaSuccess) return e;
-  e = moe_host::launch_dispatch(L->ids, L->w, x, d.T, d.H, d.E, d.k, d.dtype, L->counts,
-                                L->offsets, L->perm, L->inv_perm, L->packed_tok, L->packed_w,
-                                L->x_packed, L->dws, L->status, s);
+  const int ng = d.n_groups > 1 ? d.n_groups : 1;
+  cudaError_t e;
+  if (moe_host::route_dispatch_fits(d.T, d.H, d.E, d.k)) {
+    // decode batches: router and dispatcher in one launch
+    e = moe_host::launch_route_dispatch(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k,
+                                        d.renormalize != 0, d.dtype, L->logits, L->ids, L->w,
+                                        L->counts, L->offsets, L->perm, L->inv_perm,
+                                        L->packed_tok, L->packed_w, L->x_packed, L->counter,
+                                        L->status, s, ng, d.topk_groups);
+  } else {
+    e = moe_host::launch_route(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k, d.renormalize != 0,
+                               d.dtype, L->logits, L->ids, L->w, L->status, s, ng,
+                               d.topk_groups);
+    if (e == cudaSuccess)
+      e = moe_host::launch_dispatch(L->ids, L->w, x, d.T, d.H, d.E, d.k, d.dtype, L->counts,
+                                    L->offsets, L->perm, L->inv_perm, L->packed_tok,
+                                    L->packed_w, L->x_packed, L->dws, L->status, s);
+  }
   if (e != cudaSuccess) return e;
   const char* why = "";
   const bool shared = d.w13s != nullptr;
@@ -222,7 +234,7 @@ int moe_layer_create(const moe_layer_desc* d, void* workspace, size_t workspace_
   cudaError_t e = cudaSuccess;
   // the experts' split-K counters and the status word start at zero
   if (L->ews) e = cudaMemsetAsync(L->ews, 0, L->ews_bytes, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(L->status, 0, 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(L->status, 0, 8, s);   // status and ticket
   if (e == cudaSuccess && L->sh_offsets) {
     static thread_local int32_t so[2];
     so[0] = 0;

@@ -27,6 +27,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "dispatch_cta.cuh"
 #include "select.cuh"
 
 namespace cg = cooperative_groups;
@@ -70,15 +71,37 @@ __device__ __forceinline__ void load8(const void* base, size_t off, bool ok, flo
 // order, so the logits do not depend on timing.  Warp 0 then selects.
 constexpr int NS = 512;   // threads per CTA of the small-batch router
 
-template <int EP, bool BF16>
+// With FUSED, the router also dispatches: after its token is routed, each
+// CTA makes its writes visible (__threadfence) and takes a ticket from a
+// device counter; the CTA that takes the last ticket (no CTA ever waits for
+// another) reads every token's selection at L2 and runs the single-CTA
+// dispatch (per-warp counts, scan, stable scatter, and the gather of the rows
+// when they total at most 128 KiB), then puts the counter back to zero for
+// the next launch.
+struct SmallDispatch {
+  int32_t* counter;            // zero before the launch; zero again after it
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  int32_t* packed_tok;
+  float* packed_w;
+  const uint4* x;              // null: no fused gather
+  int row_vecs;
+  uint4* x_packed;
+  int32_t* status;
+};
+
+constexpr int kFusedRounds = 1;                       // N <= 16 warps x 32 = 512
+
+template <int EP, bool BF16, bool FUSED>
 __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
                                                          const void* __restrict__ wv,
                                                          const float* __restrict__ bias, int H,
                                                          int E, int k, int renorm,
                                                          float* __restrict__ logits,
-                                                         int32_t* __restrict__ ids,
-                                                         float* __restrict__ wout,
-                                                         moe::GroupLimit gl) {
+                                                         int32_t* ids, float* wout,
+                                                         moe::GroupLimit gl, SmallDispatch dd) {
   constexpr int NWARP = NS / 32;
   constexpr int EPW = EP > NWARP ? EP / NWARP : 1;       // experts per warp
   constexpr int WPE = EP >= NWARP ? 1 : NWARP / EP;      // warps (H slices) per expert
@@ -159,26 +182,47 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
   }
   __syncthreads();
   moe::grid_dep_launch();
-  if (warp != 0) return;
-  constexpr int PER = 2;                       // experts lane, lane + 32
-  float v[PER];
-  bool live[PER];
+  if (warp == 0) {
+    constexpr int PER = 2;                     // experts lane, lane + 32
+    float v[PER];
+    bool live[PER];
 #pragma unroll
-  for (int j = 0; j < PER; ++j) {
-    const int ex = lane + 32 * j;
-    live[j] = ex < E;
-    float s = 0.f;
-    if (live[j]) {
+    for (int j = 0; j < PER; ++j) {
+      const int ex = lane + 32 * j;
+      live[j] = ex < E;
+      float s = 0.f;
+      if (live[j]) {
 #pragma unroll
-      for (int sl = 0; sl < WPE; ++sl) s += part[ex][sl];
-      s += bias ? bias[ex] : 0.f;
-      logits[static_cast<size_t>(t) * E + ex] = s;
+        for (int sl = 0; sl < WPE; ++sl) s += part[ex][sl];
+        s += bias ? bias[ex] : 0.f;
+        logits[static_cast<size_t>(t) * E + ex] = s;
+      }
+      v[j] = live[j] ? s : -FLT_MAX;
     }
-    v[j] = live[j] ? s : -FLT_MAX;
+    if (k > 0)
+      moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
+                            wout + static_cast<size_t>(t) * k, gl);
   }
-  if (k == 0) return;
-  moe::select_topk<PER>(v, live, k, renorm, ids + static_cast<size_t>(t) * k,
-                        wout + static_cast<size_t>(t) * k, gl);
+  if constexpr (FUSED) {
+    __shared__ int s_last;
+    __shared__ int s_scan[moe::kMaxExperts];
+    __syncthreads();                           // this token's ids and weights are written
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(dd.counter, 1) == static_cast<int>(gridDim.x) - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();                           // every other token's writes are now visible
+    int* wc = reinterpret_cast<int*>(xs);      // [NWARP][E]: x is no longer needed
+    for (int i = threadIdx.x; i < NWARP * E; i += NS) wc[i] = 0;
+    __syncthreads();
+    moe::dispatch_cta<NWARP, kFusedRounds>(ids, wout, static_cast<int>(gridDim.x) * k, E, k,
+                                           dd.counts, dd.offsets, dd.perm, dd.inv_perm,
+                                           dd.packed_tok, dd.packed_w, dd.x, dd.row_vecs,
+                                           dd.x_packed, dd.status, wc, s_scan);
+    if (threadIdx.x == 0) *dd.counter = 0;
+  }
 }
 
 // Token rows per thread: 8 when E <= 64 (more FMAs per shared-memory read),
@@ -376,6 +420,32 @@ cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H,
                               E, k, renorm, kc_per_cta, logits, ids, w, gl);
 }
 
+template <int EP, bool FUSED>
+cudaError_t launch_small_ep(const void* x, const void* W, const float* b, int T, int H, int E,
+                            int k, int renorm, bool bf, float* logits, int32_t* ids, float* w,
+                            moe::GroupLimit gl, const SmallDispatch& dd, cudaStream_t s) {
+  // The fused dispatch reuses the x row's shared memory for its [16][E] counts.
+  const int smem = std::max(H, FUSED ? (NS / 32) * E : 0) * 4;
+  auto fn = bf ? route_small_kernel<EP, true, FUSED> : route_small_kernel<EP, false, FUSED>;
+  cudaError_t e = moe_host::ensure_smem(reinterpret_cast<const void*>(fn), smem);
+  if (e != cudaSuccess) return e;
+  return moe_host::launch_pdl(fn, dim3(T), dim3(NS), smem, s, 0, x, W, b, H, E, k, renorm,
+                              logits, ids, w, gl, dd);
+}
+
+template <bool FUSED>
+cudaError_t launch_small(const void* x, const void* W, const float* b, int T, int H, int E, int k,
+                         int renorm, bool bf, float* logits, int32_t* ids, float* w,
+                         moe::GroupLimit gl, const SmallDispatch& dd, cudaStream_t s) {
+  if (E <= 1) return launch_small_ep<1, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (E <= 2) return launch_small_ep<2, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (E <= 4) return launch_small_ep<4, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (E <= 8) return launch_small_ep<8, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (E <= 16) return launch_small_ep<16, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (E <= 32) return launch_small_ep<32, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  return launch_small_ep<64, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+}
+
 }  // namespace
 
 namespace moe_host {
@@ -387,31 +457,9 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
   const bool bf = dtype == MOE_BF16;
   const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
                            n_groups > 1 ? topk_groups : 1};
-  if (T <= 64 && E <= 64 && H <= 32768) {
-#define MOE_SMALL_CASE(EPV)                                                                   \
-    if (E <= EPV) {                                                                         \
-      if (bf) {                                                                             \
-        cudaError_t e = ensure_smem(                                                        \
-            reinterpret_cast<const void*>(route_small_kernel<EPV, true>), H * 4);           \
-        if (e != cudaSuccess) return e;                                                     \
-        return launch_pdl(route_small_kernel<EPV, true>, dim3(T), dim3(NS), H * 4, s, 0, x,   \
-                          W_gate, bias, H, E, k, renormalize, logits, ids, w, gl);          \
-      }                                                                                     \
-      cudaError_t e = ensure_smem(                                                          \
-          reinterpret_cast<const void*>(route_small_kernel<EPV, false>), H * 4);            \
-      if (e != cudaSuccess) return e;                                                       \
-      return launch_pdl(route_small_kernel<EPV, false>, dim3(T), dim3(NS), H * 4, s, 0, x,    \
-                        W_gate, bias, H, E, k, renormalize, logits, ids, w, gl);            \
-    }
-    MOE_SMALL_CASE(1)
-    MOE_SMALL_CASE(2)
-    MOE_SMALL_CASE(4)
-    MOE_SMALL_CASE(8)
-    MOE_SMALL_CASE(16)
-    MOE_SMALL_CASE(32)
-    MOE_SMALL_CASE(64)
-#undef MOE_SMALL_CASE
-  }
+  if (T <= 64 && E <= 64 && H <= 32768)
+    return launch_small<false>(x, W_gate, bias, T, H, E, k, renormalize, bf, logits, ids, w, gl,
+                               SmallDispatch{}, s);
   if (bf)
     return launch_route_tc(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, s,
                            n_groups, topk_groups);
@@ -419,6 +467,33 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
   if (E <= 128) return launch_t<128, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, gl, s);
   if (E <= 256) return launch_t<256, false>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, gl, s);
   return cudaErrorInvalidValue;
+}
+
+bool route_dispatch_fits(int T, int H, int E, int k) {
+  return T >= 1 && T <= 64 && E >= 1 && E <= 64 && H <= 32768 && k >= 1 && k <= moe::kMaxTopK &&
+         T * k <= (NS / 32) * 32 * kFusedRounds;
+}
+
+cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float* bias, int T,
+                                  int H, int E, int k, int renormalize, int dtype, float* logits,
+                                  int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
+                                  int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
+                                  float* packed_w, void* x_packed, int32_t* counter,
+                                  int32_t* status, cudaStream_t s, int n_groups,
+                                  int topk_groups) {
+  const bool bf = dtype == MOE_BF16;
+  const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
+                           n_groups > 1 ? topk_groups : 1};
+  const int row_bytes = H * (bf ? 2 : 4);
+  const bool fuse_gather = x_packed != nullptr &&
+                           static_cast<size_t>(T) * k * row_bytes <= (static_cast<size_t>(128) << 10);
+  const SmallDispatch dd{counter, counts, offsets, perm, inv_perm, packed_tok, packed_w,
+                         fuse_gather ? static_cast<const uint4*>(x) : nullptr, row_bytes / 16,
+                         static_cast<uint4*>(x_packed), status};
+  cudaError_t e = launch_small<true>(x, W_gate, bias, T, H, E, k, renormalize, bf, logits, ids, w,
+                                     gl, dd, s);
+  if (e != cudaSuccess || x_packed == nullptr || fuse_gather) return e;
+  return launch_gather(x, packed_tok, offsets, 0, E, T * k, H, dtype, x_packed, status, s);
 }
 
 }  // namespace moe_host

@@ -100,6 +100,27 @@ def test_dispatch_rejects_bad_arguments_on_the_host(lib):
     assert lib.moe_dispatch(*a) == M.MOE_ERR_INVALID_ARG
 
 
+def test_route_dispatch_rejects_bad_arguments_on_the_host(lib):
+    # x, W, bias, T, H, E, k, renorm, G, Mg, dtype, logits, ids, w, counts, offsets, perm,
+    # inv_perm, packed_tok, packed_w, x_packed, counter, status, stream
+    args = [P, P, NULL, 4, 64, 8, 2, 1, 1, 1, M.MOE_BF16, P, P, P, P, P, P, P, P, P, P, P, NULL,
+            NULL]
+    a = list(args); a[3] = 65             # more tokens than the one-launch path takes
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "T must be" in _err(lib)
+    a = list(args); a[5] = 65; a[6] = 2   # more experts than it takes
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "E must be" in _err(lib)
+    a = list(args); a[6] = 0              # it always dispatches: k >= 1
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "k must be" in _err(lib)
+    a = list(args); a[21] = NULL          # no ticket word
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "counter" in _err(lib)
+    a = list(args); a[8] = 3              # 3 groups do not divide 8 experts
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "n_groups" in _err(lib)
+    a = list(args); a[4] = 32776          # H above 32768
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "H must be" in _err(lib)
+    a = list(args); a[10] = 7
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG
+
+
 def test_experts_rejects_bad_arguments_on_the_host(lib):
     base = [P, P, P, P, P, 100, 256, 128, 4, M.MOE_BF16, P, P, NULL, 0, NULL, NULL]
     a = list(base); a[6] = 200            # H not a multiple of 256 on the bf16 path
