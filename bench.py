@@ -28,7 +28,7 @@ sample per step; rank 0 only).
 Roofline of the grouped GEMM (``roofline``): its algorithmic bytes are the
 weights of the experts that received tokens (plus a shared expert's); its
 flops 2*N*3*H*I (+ the shared expert's).  The packed intermediates it also
-moves (x_packed, h, fp32 y_packed) are reported beside it
+moves (x_packed, h, y_packed) are reported beside it
 (``bytes_incl_packed``, ``frac_incl_packed``), not in ``frac``.
 """
 from __future__ import annotations
@@ -93,16 +93,17 @@ def expert_weight_work(cfg, counts):
 
 def expert_stage_work(cfg, counts):
     """The same stage's bytes INCLUDING the materialised intermediates (x_packed
-    read, h written and read back, fp32 y_packed written, routing weights;
-    with a shared expert also its x read, h_s written and read, fp32 output
-    written), and its flops."""
+    read, h written and read back, y_packed written -- 2 bytes per element
+    (fp16) in bf16 layers, as the layer stores it --, routing weights; with a
+    shared expert also its x read, h_s written and read, output written), and
+    its flops."""
     es = 2 if cfg.dtype == "bf16" else 4
     N = int(sum(counts))
     H, I = cfg.H, cfg.I
     wbytes, flops = expert_weight_work(cfg, counts)
-    abytes = N * H * es + 2 * N * I * es + N * H * 4 + N * 4
+    abytes = N * H * es + 2 * N * I * es + N * H * es + N * 4
     if cfg.shared_I:
-        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * 4
+        abytes += cfg.T * H * es + 2 * cfg.T * cfg.shared_I * es + cfg.T * H * es
     return wbytes + abytes, flops
 
 

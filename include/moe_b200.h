@@ -50,12 +50,16 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented for this shape    */
   MOE_ERR_CUDA = 3,         /* a CUDA launch / runtime call failed         */
   MOE_ERR_TIMEOUT = 4,      /* (device status) a bounded wait ran out      */
-  MOE_ERR_BAD_INDEX = 5     /* (device status) an index was out of range   */
+  MOE_ERR_BAD_INDEX = 5,    /* (device status) an index was out of range   */
+  MOE_ERR_OVERFLOW = 6      /* (device status) a value beyond the fp16 range
+                               was stored in an fp16 y_packed (it became inf) */
 } moe_status_t;
 
 typedef enum {
   MOE_F32 = 0,   /* activations, weights and outputs in fp32              */
-  MOE_BF16 = 1   /* activations, weights and outputs in bf16, fp32 inside  */
+  MOE_BF16 = 1,  /* activations, weights and outputs in bf16, fp32 inside  */
+  MOE_F16 = 2    /* fp16: only as the type of y_packed and of the shared
+                    expert's output (y_dtype) of a bf16 layer               */
 } moe_dtype_t;
 
 /* Version of this ABI (bumped on any added entry point or signature change). */
@@ -241,15 +245,22 @@ size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
  *   y_packed[p,c] = packed_w[p] * (h[p,:] . w2[e,c,:])
  * with silu(z) = z / (1 + exp(-z)), fp32 accumulation, and (bf16) h
  * rounded to bf16 before the second product (it is the operand of a bf16
- * tensor-core product).  y_packed is always fp32: the merger adds the k
- * terms of a token before the output's one rounding.
+ * tensor-core product).  y_packed is stored in y_dtype: fp16 (each element
+ * rounded once, to nearest, after the fp32 accumulation and the
+ * routing-weight scale: a relative error of at most 2^-11, half the bytes to
+ * write here and to read in the merger) or fp32 (the merger then adds the k
+ * fp32 terms before the output's only rounding).  An fp16 element whose
+ * magnitude exceeds 65504 becomes inf and sets MOE_ERR_OVERFLOW in status.
+ * fp32 layers take y_dtype = MOE_F32 only.
  *
  *   x_packed device [N,H]       offsets device [E+1] int32 (read on the
  *   device; the host never needs the split)
  *   packed_w device [N] fp32, or NULL for all-ones (e.g. a shared expert)
  *   w13 device [E,2I,H]         w2 device [E,H,I]
  *   h        device [N,I] (dtype) scratch, written
- *   y_packed device [N,H] fp32, written; rows outside every expert's
+ *   y_dtype  MOE_F16 or MOE_F32 (bf16 layers), MOE_F32 (fp32 layers);
+ *            otherwise MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED
+ *   y_packed device [N,H] (y_dtype), written; rows outside every expert's
  *            range are left untouched
  *   ws/ws_bytes  device scratch of moe_experts_workspace_bytes() bytes,
  *            ZERO-FILLED before its first use (the kernels leave it zeroed
@@ -257,13 +268,13 @@ size_t moe_experts_workspace_bytes(int N, int H, int I, int E, int dtype);
  *            fewer tiles than two per SM splits K and reduces the fp32
  *            partials in a fixed order (deterministic).  NULL / 0 is allowed:
  *            no split.  Calls that share one ws must not overlap on the GPU.
- *   status   device int32 or NULL (timeouts)
+ *   status   device int32 or NULL (timeouts, fp16 overflow)
  * offsets must be non-decreasing with offsets[E] <= N (as moe_dispatch
  * writes them); rows are trusted to lie in [0, N).
  */
 int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
                 const void* w13, const void* w2, int N, int H, int I, int E, int dtype,
-                void* h, void* y_packed, void* ws, size_t ws_bytes,
+                int y_dtype, void* h, void* y_packed, void* ws, size_t ws_bytes,
                 int32_t* status, void* stream);
 
 /*
@@ -278,14 +289,14 @@ int moe_experts(const void* x_packed, const int32_t* offsets, const float* packe
  * bf16 only (fp32 returns MOE_ERR_UNSUPPORTED: call moe_experts twice).
  *
  *   x    device [T,H] bf16          w13s device [2*I_s,H]   w2s device [H,I_s]
- *   h_s  device [T,I_s] bf16, written   y_s device [T,H] fp32, written
+ *   h_s  device [T,I_s] bf16, written   y_s device [T,H] (y_dtype), written
  *   I_s % 64 == 0; all other arguments, results and rules as moe_experts.
  */
 int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float* packed_w,
                        const void* w13, const void* w2, int N, int H, int I, int E,
                        const void* x, int T, const void* w13s, const void* w2s, int I_s,
-                       int dtype, void* h, void* y_packed, void* h_s, float* y_s, void* ws,
-                       size_t ws_bytes, int32_t* status, void* stream);
+                       int dtype, int y_dtype, void* h, void* y_packed, void* h_s, void* y_s,
+                       void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
 /*
  * moe_combine -- Merger.  DWDP README, "Merger Module": restore token-major
@@ -296,8 +307,9 @@ int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float
  *              fp32 sum, one rounding to the output type)
  *            + sigmoid(shared_gate_logit[t]) * shared[t,:]   (if shared)
  *
- *   y_packed device [N,H] fp32, N = T*k      inv_perm device [N] int32
- *   shared   device [T,H] fp32 or NULL (a moe_experts output with E = 1);
+ *   y_packed device [N,H] (y_dtype: MOE_F16 or MOE_F32), N = T*k
+ *   inv_perm device [N] int32
+ *   shared   device [T,H] (y_dtype) or NULL (a moe_experts output with E = 1);
  *            shared_gate_logit device [T] fp32 or NULL (gate 1 when shared
  *            is given without it): the always-on shared expert of
  *            diffulex.moe.layer (SharedExpertMLP)
@@ -306,8 +318,8 @@ int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float
  *   status   device int32 or NULL: an inv_perm entry outside [0,N) sets
  *            MOE_ERR_BAD_INDEX and contributes nothing.
  */
-int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,
-                const float* shared, const float* shared_gate_logit, int dtype,
+int moe_combine(const void* y_packed, int y_dtype, const int32_t* inv_perm, int T, int H, int k,
+                const void* shared, const float* shared_gate_logit, int dtype,
                 void* out, int32_t* status, void* stream);
 
 /*
@@ -362,10 +374,10 @@ int moe_gather(const void* x, const int32_t* packed_tok, const int32_t* offsets,
  * Arguments and errors as moe_combine, plus offsets (device [E+1] int32)
  * and 0 <= expert_start <= expert_end <= E.
  */
-int moe_combine_range(const float* y_packed, const int32_t* inv_perm, const int32_t* offsets,
-                      int E, int expert_start, int expert_end, int T, int H, int k,
-                      const float* shared, const float* shared_gate_logit, int dtype, void* out,
-                      int32_t* status, void* stream);
+int moe_combine_range(const void* y_packed, int y_dtype, const int32_t* inv_perm,
+                      const int32_t* offsets, int E, int expert_start, int expert_end, int T,
+                      int H, int k, const void* shared, const float* shared_gate_logit,
+                      int dtype, void* out, int32_t* status, void* stream);
 
 /*
  * moe_finalize -- the one rounding after the ranks' partial outputs were
@@ -457,6 +469,8 @@ typedef struct moe_layer_desc {
   const void* w13s;           /* device [2I_s,H] or NULL: no shared expert */
   const void* w2s;            /* device [H,I_s] */
   const void* w_sg;           /* device [H]: the shared expert's gate vector */
+  int y_f32;                  /* bf16 layers: keep y_packed and the shared expert's
+                                 output in fp32 (0: in fp16, see moe_experts) */
 } moe_layer_desc;
 
 typedef struct moe_layer moe_layer;   /* opaque */

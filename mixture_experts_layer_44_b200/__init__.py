@@ -26,14 +26,16 @@ __all__ = [
     "moe_experts_workspace_bytes",
     "moe_experts", "moe_experts_shared", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
-    "MOE_ERR_BAD_INDEX", "MOE_F32", "MOE_BF16", "MoELayerBuffers", "moe_layer_forward",
+    "MOE_ERR_BAD_INDEX", "MOE_ERR_OVERFLOW", "MOE_F32", "MOE_BF16", "MOE_F16", "MoELayerBuffers",
+    "moe_layer_forward", "moe_route_dispatch", "route_dispatch_fits", "route_and_dispatch",
     "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
     "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
     "MoELayerDesc", "MoELayer", "moe_test_set_wait_budget_ns",
 ]
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, MOE_ERR_BAD_INDEX = range(6)
-MOE_F32, MOE_BF16 = 0, 1
+(MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
+ MOE_ERR_BAD_INDEX, MOE_ERR_OVERFLOW) = range(7)
+MOE_F32, MOE_BF16, MOE_F16 = 0, 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -62,10 +64,10 @@ _SIGS = {
     "moe_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "moe_dispatch_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_experts_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
-    "moe_experts": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
-    "moe_experts_shared": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _I, _P, _P,
-                                _P, _P, _P, _SZ, _P, _P]),
-    "moe_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
+    "moe_experts": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
+    "moe_experts_shared": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _I, _I, _I,
+                                _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "moe_combine": (_I, [_P, _I, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_read_status": (_I, [_P, _P, _P]),
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
@@ -81,7 +83,7 @@ _SIGS = {
     "moe_layer_join": (_I, [_P, _P]),
     "moe_layer_status": (_I, [_P, _P, _P]),
     "moe_layer_buffer": (_P, [_P, ctypes.c_char_p]),
-    "moe_combine_range": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
+    "moe_combine_range": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _I, _P, _P, _P]),
     "moe_finalize": (_I, [_P, _I, _I, _I, _P, _P]),
     "moe_ep_partition_workspace_bytes": (_SZ, [_I, _I]),
     "moe_ep_owner": (_I, [_P, _I, _I, _I, _P, _P, _P]),
@@ -123,6 +125,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return MOE_BF16
     if t.dtype == torch.float32:
         return MOE_F32
+    if t.dtype == torch.float16:
+        return MOE_F16
     raise MoEError(MOE_ERR_INVALID_ARG, f"unsupported dtype {t.dtype}")
 
 
@@ -226,7 +230,7 @@ def moe_experts(x_packed, offsets, packed_w, w13, w2, h, y_packed, ws=None, stat
     I = w13.shape[1] // 2
     _check(load_library().moe_experts(
         _ptr(x_packed), _ptr(offsets), _ptr(packed_w), _ptr(w13), _ptr(w2), N, H, I, E,
-        _dtype_code(x_packed), _ptr(h), _ptr(y_packed), _ptr(ws),
+        _dtype_code(x_packed), _dtype_code(y_packed), _ptr(h), _ptr(y_packed), _ptr(ws),
         ws.numel() * ws.element_size() if ws is not None else 0, _ptr(status), _stream(stream)))
 
 
@@ -241,7 +245,8 @@ def moe_experts_shared(x_packed, offsets, packed_w, w13, w2, h, y_packed, x, w13
     I_s = w13s.shape[0] // 2
     _check(load_library().moe_experts_shared(
         _ptr(x_packed), _ptr(offsets), _ptr(packed_w), _ptr(w13), _ptr(w2), N, H, I, E,
-        _ptr(x), T, _ptr(w13s), _ptr(w2s), I_s, _dtype_code(x_packed), _ptr(h), _ptr(y_packed),
+        _ptr(x), T, _ptr(w13s), _ptr(w2s), I_s, _dtype_code(x_packed), _dtype_code(y_packed),
+        _ptr(h), _ptr(y_packed),
         _ptr(h_s), _ptr(y_s), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
         _ptr(status), _stream(stream)))
 
@@ -250,7 +255,8 @@ def moe_combine(y_packed, inv_perm, T: int, k: int, out, shared=None, shared_gat
                 status=None, stream=None):
     H = out.shape[1]
     _check(load_library().moe_combine(
-        _ptr(y_packed), _ptr(inv_perm), T, H, k, _ptr(shared), _ptr(shared_gate_logit),
+        _ptr(y_packed), _dtype_code(y_packed), _ptr(inv_perm), T, H, k, _ptr(shared),
+        _ptr(shared_gate_logit),
         _dtype_code(out), _ptr(out), _ptr(status), _stream(stream)))
 
 
@@ -271,7 +277,8 @@ def moe_combine_range(y_packed, inv_perm, offsets, expert_start: int, expert_end
     H = out.shape[1]
     E = offsets.shape[0] - 1
     _check(load_library().moe_combine_range(
-        _ptr(y_packed), _ptr(inv_perm), _ptr(offsets), E, expert_start, expert_end, T, H, k,
+        _ptr(y_packed), _dtype_code(y_packed), _ptr(inv_perm), _ptr(offsets), E, expert_start,
+        expert_end, T, H, k,
         _ptr(shared), _ptr(shared_gate_logit), _dtype_code(out), _ptr(out), _ptr(status),
         _stream(stream)))
 
@@ -332,10 +339,11 @@ class MoELayerDesc(ctypes.Structure):
     _fields_ = [("T", _I), ("H", _I), ("E", _I), ("k", _I), ("I", _I), ("dtype", _I),
                 ("renormalize", _I), ("n_groups", _I), ("topk_groups", _I), ("W_gate", _P),
                 ("bias", _P), ("w13", _P), ("w2", _P), ("I_s", _I), ("w13s", _P), ("w2s", _P),
-                ("w_sg", _P)]
+                ("w_sg", _P), ("y_f32", _I)]
 
 
-def _desc(params: dict, T: int, k: int, renormalize: bool, n_groups: int, topk_groups: int):
+def _desc(params: dict, T: int, k: int, renormalize: bool, n_groups: int, topk_groups: int,
+          y_f32: bool = False):
     W = params["W_gate"]
     E, H = W.shape
     I = params["w13"].shape[1] // 2
@@ -343,7 +351,8 @@ def _desc(params: dict, T: int, k: int, renormalize: bool, n_groups: int, topk_g
                      renormalize=int(bool(renormalize)), n_groups=n_groups,
                      topk_groups=topk_groups, W_gate=W.data_ptr(),
                      bias=params["bias"].data_ptr() if params.get("bias") is not None else None,
-                     w13=params["w13"].data_ptr(), w2=params["w2"].data_ptr())
+                     w13=params["w13"].data_ptr(), w2=params["w2"].data_ptr(),
+                     y_f32=int(bool(y_f32)))
     if params.get("w13s") is not None:
         d.I_s = params["w13s"].shape[0] // 2
         d.w13s = params["w13s"].data_ptr()
@@ -358,10 +367,10 @@ class MoELayer:
     tensors) must stay alive as long as the layer."""
 
     def __init__(self, params: dict, T: int, k: int, renormalize: bool, n_groups: int = 1,
-                 topk_groups: int = 1, stream=None):
+                 topk_groups: int = 1, stream=None, y_f32: bool = False):
         lib = load_library()
         self.params = params
-        self.desc = _desc(params, T, k, renormalize, n_groups, topk_groups)
+        self.desc = _desc(params, T, k, renormalize, n_groups, topk_groups, y_f32)
         nbytes = lib.moe_layer_workspace_bytes(ctypes.byref(self.desc))
         if nbytes == 0:
             raise MoEError(MOE_ERR_INVALID_ARG, "moe_layer_workspace_bytes: invalid layer")
@@ -422,10 +431,13 @@ class MoELayerBuffers:
 
     Shapes follow the ABI: T tokens, N = T*k assignments.  With a shared
     expert the buffers also hold its packed input/output and gate logit.
+    y_packed (and the shared expert's output) are fp16 for bf16 layers (half
+    the bytes of fp32; an element beyond the fp16 range sets MOE_ERR_OVERFLOW)
+    unless ``y_f32``, and fp32 for fp32 layers.
     """
 
     def __init__(self, T: int, H: int, E: int, k: int, I: int, dtype: torch.dtype,
-                 device="cuda", shared_I: Optional[int] = None):
+                 device="cuda", shared_I: Optional[int] = None, y_f32: bool = False):
         N = T * k
         dev = torch.device(device)
         i32 = dict(dtype=torch.int32, device=dev)
@@ -442,7 +454,8 @@ class MoELayerBuffers:
         self.packed_w = torch.empty(N, **f32)
         self.x_packed = torch.empty(N, H, dtype=dtype, device=dev)
         self.h = torch.empty(N, I, dtype=dtype, device=dev)
-        self.y_packed = torch.empty(N, H, **f32)        # packed expert outputs stay fp32
+        self.y_dtype = torch.float16 if dtype == torch.bfloat16 and not y_f32 else torch.float32
+        self.y_packed = torch.empty(N, H, dtype=self.y_dtype, device=dev)
         self.out = torch.empty(T, H, dtype=dtype, device=dev)
         self.ws = torch.empty(max(1, moe_dispatch_workspace_bytes(T, k, E)), dtype=torch.uint8,
                               device=dev)
@@ -461,7 +474,7 @@ class MoELayerBuffers:
             self.sg_logit = torch.empty(T, 1, **f32)
             self.sh_offsets = torch.tensor([0, T], **i32)
             self.sh_h = torch.empty(T, shared_I, dtype=dtype, device=dev)
-            self.sh_y = torch.empty(T, H, **f32)
+            self.sh_y = torch.empty(T, H, dtype=self.y_dtype, device=dev)
 
 
 def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,

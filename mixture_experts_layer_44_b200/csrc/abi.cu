@@ -43,6 +43,13 @@ int check_dtype(int dtype) {
   return MOE_OK;
 }
 
+// The type of y_packed and of a shared expert's output.
+int check_y_dtype(int y_dtype) {
+  if (y_dtype != MOE_F32 && y_dtype != MOE_F16)
+    return fail(MOE_ERR_INVALID_ARG, "y_dtype must be MOE_F32 (0) or MOE_F16 (2)");
+  return MOE_OK;
+}
+
 // Bounded-wait self-test: one thread waits on an mbarrier nothing arrives on.
 __global__ void probe_wait_kernel(int32_t* status, uint64_t budget_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -84,7 +91,7 @@ cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream
 
 extern "C" {
 
-int moe_abi_version(void) { return 3; }
+int moe_abi_version(void) { return 4; }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -237,10 +244,14 @@ namespace {
 // expert).
 int experts_impl(const char* fn, const void* x_packed, const int32_t* offsets,
                  const float* packed_w, const void* w13, const void* w2, int N, int H, int I,
-                 int E, int dtype, void* h, void* y_packed, const moe_host::SharedGroup* sh,
-                 void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+                 int E, int dtype, int y_dtype, void* h, void* y_packed,
+                 const moe_host::SharedGroup* sh, void* ws, size_t ws_bytes, int32_t* status,
+                 void* stream) {
   const std::string f = std::string(fn) + ": ";
   if (int r = check_dtype(dtype)) return r;
+  if (int r = check_y_dtype(y_dtype)) return r;
+  REQ(dtype == MOE_BF16 || y_dtype == MOE_F32, MOE_ERR_UNSUPPORTED,
+      f + "fp32 layers keep y_packed in fp32 (y_dtype must be MOE_F32)");
   REQ(N >= 0, MOE_ERR_INVALID_ARG, f + "N must be >= 0");
   if (N == 0 && sh == nullptr) return MOE_OK;
   REQ(x_packed && offsets && w13 && w2 && h && y_packed, MOE_ERR_INVALID_ARG,
@@ -262,7 +273,7 @@ int experts_impl(const char* fn, const void* x_packed, const int32_t* offsets,
         f + "the bf16 tensor-core path needs H % 256 == 0 and I % 64 == 0");
     const char* why = "";
     e = moe_host::launch_experts_tc(x_packed, offsets, packed_w, w13, w2, N, H, I, E, h, y_packed,
-                                    sh, ws, ws_bytes, status, s, &why);
+                                    y_dtype == MOE_F16, sh, ws, ws_bytes, status, s, &why);
     if (e != cudaSuccess && why[0]) return fail(MOE_ERR_CUDA, f + why);
   } else {
     REQ(sh == nullptr, MOE_ERR_UNSUPPORTED,
@@ -276,18 +287,19 @@ int experts_impl(const char* fn, const void* x_packed, const int32_t* offsets,
 }  // namespace
 
 int moe_experts(const void* x_packed, const int32_t* offsets, const float* packed_w,
-                const void* w13, const void* w2, int N, int H, int I, int E, int dtype, void* h,
-                void* y_packed, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+                const void* w13, const void* w2, int N, int H, int I, int E, int dtype,
+                int y_dtype, void* h, void* y_packed, void* ws, size_t ws_bytes,
+                int32_t* status, void* stream) {
   g_err.clear();
-  return experts_impl("moe_experts", x_packed, offsets, packed_w, w13, w2, N, H, I, E, dtype, h,
-                      y_packed, nullptr, ws, ws_bytes, status, stream);
+  return experts_impl("moe_experts", x_packed, offsets, packed_w, w13, w2, N, H, I, E, dtype,
+                      y_dtype, h, y_packed, nullptr, ws, ws_bytes, status, stream);
 }
 
 int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float* packed_w,
                        const void* w13, const void* w2, int N, int H, int I, int E,
                        const void* x, int T, const void* w13s, const void* w2s, int I_s,
-                       int dtype, void* h, void* y_packed, void* h_s, float* y_s, void* ws,
-                       size_t ws_bytes, int32_t* status, void* stream) {
+                       int dtype, int y_dtype, void* h, void* y_packed, void* h_s, void* y_s,
+                       void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   g_err.clear();
   REQ(x && w13s && w2s && h_s && y_s, MOE_ERR_INVALID_ARG,
       "moe_experts_shared: null shared-expert input or output");
@@ -299,14 +311,15 @@ int moe_experts_shared(const void* x_packed, const int32_t* offsets, const float
       MOE_ERR_INVALID_ARG, "moe_experts_shared: T too large");
   const moe_host::SharedGroup sh{x, T, w13s, w2s, I_s, h_s, y_s};
   return experts_impl("moe_experts_shared", x_packed, offsets, packed_w, w13, w2, N, H, I, E,
-                      dtype, h, y_packed, &sh, ws, ws_bytes, status, stream);
+                      dtype, y_dtype, h, y_packed, &sh, ws, ws_bytes, status, stream);
 }
 
-int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, int k,
-                const float* shared, const float* shared_gate_logit, int dtype, void* out,
+int moe_combine(const void* y_packed, int y_dtype, const int32_t* inv_perm, int T, int H, int k,
+                const void* shared, const float* shared_gate_logit, int dtype, void* out,
                 int32_t* status, void* stream) {
   g_err.clear();
   if (int r = check_dtype(dtype)) return r;
+  if (int r = check_y_dtype(y_dtype)) return r;
   REQ(y_packed && inv_perm && out, MOE_ERR_INVALID_ARG, "moe_combine: null y_packed, inv_perm or out");
   REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_combine: T and H must be >= 1");
   REQ(k >= 1 && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG, "moe_combine: k must be in [1, 8]");
@@ -316,17 +329,19 @@ int moe_combine(const float* y_packed, const int32_t* inv_perm, int T, int H, in
   REQ(aligned4(inv_perm) && aligned4(shared_gate_logit) && aligned4(status), MOE_ERR_INVALID_ARG,
       "moe_combine: inv_perm / gate / status must be 4-byte aligned");
   REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG, "moe_combine: T*k too large");
-  cudaError_t e = moe_host::launch_combine(y_packed, inv_perm, T, H, k, shared, shared_gate_logit,
-                                           dtype, out, status, static_cast<cudaStream_t>(stream));
+  cudaError_t e = moe_host::launch_combine(y_packed, y_dtype, inv_perm, T, H, k, shared,
+                                           shared_gate_logit, dtype, out, status,
+                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
 }
 
-int moe_combine_range(const float* y_packed, const int32_t* inv_perm, const int32_t* offsets,
-                      int E, int expert_start, int expert_end, int T, int H, int k,
-                      const float* shared, const float* shared_gate_logit, int dtype, void* out,
-                      int32_t* status, void* stream) {
+int moe_combine_range(const void* y_packed, int y_dtype, const int32_t* inv_perm,
+                      const int32_t* offsets, int E, int expert_start, int expert_end, int T,
+                      int H, int k, const void* shared, const float* shared_gate_logit,
+                      int dtype, void* out, int32_t* status, void* stream) {
   g_err.clear();
   if (int r = check_dtype(dtype)) return r;
+  if (int r = check_y_dtype(y_dtype)) return r;
   REQ(y_packed && inv_perm && offsets && out, MOE_ERR_INVALID_ARG,
       "moe_combine_range: null y_packed, inv_perm, offsets or out");
   REQ(T >= 1 && H >= 1, MOE_ERR_INVALID_ARG, "moe_combine_range: T and H must be >= 1");
@@ -341,9 +356,10 @@ int moe_combine_range(const float* y_packed, const int32_t* inv_perm, const int3
       MOE_ERR_INVALID_ARG, "moe_combine_range: index / gate / status arrays must be 4-byte aligned");
   REQ(static_cast<long long>(T) * k < (1ll << 30), MOE_ERR_INVALID_ARG,
       "moe_combine_range: T*k too large");
-  cudaError_t e = moe_host::launch_combine(y_packed, inv_perm, T, H, k, shared, shared_gate_logit,
-                                           dtype, out, status, static_cast<cudaStream_t>(stream),
-                                           offsets, expert_start, expert_end);
+  cudaError_t e = moe_host::launch_combine(y_packed, y_dtype, inv_perm, T, H, k, shared,
+                                           shared_gate_logit, dtype, out, status,
+                                           static_cast<cudaStream_t>(stream), offsets,
+                                           expert_start, expert_end);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine_range launch");
 }
 

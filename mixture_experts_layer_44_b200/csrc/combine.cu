@@ -7,9 +7,9 @@
 // sigmoid(gate_logit[t]) * shared[t] for the always-on shared expert
 // (diffulex.moe.layer, SharedExpertMLP).
 //
-// y_packed and the shared expert's output are fp32 (the executor keeps its
-// packed outputs in fp32), so the k terms and the shared term are added in
-// fp32 and rounded once, to the output type.
+// y_packed and the shared expert's output come in the executor's output type
+// (fp16 or fp32); the k terms and the shared term are added in fp32 and
+// rounded once, to the output type.
 //
 // One CTA per token at a time (grid-stride over tokens); each thread owns
 // 16-byte vectors of the hidden dimension, so every load and store is a
@@ -30,11 +30,38 @@ namespace {
 
 constexpr int CNT = 256;
 
-template <bool OUT_BF16, int KT>
-__global__ void __launch_bounds__(CNT) combine_kernel(const float* y,
+// Eight consecutive elements of an fp32 or fp16 row, as fp32 (read at L2:
+// the rows come from the kernels just before).
+template <bool BF>
+struct Vec8;
+template <>
+struct Vec8<false> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* base, size_t row, int H, int v) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + row * H) + 2 * v;
+    a = moe::ld_prod(p);
+    b = moe::ld_prod(p + 1);
+  }
+  __device__ __forceinline__ void get(float* f) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
+template <>
+struct Vec8<true> {
+  uint4 q;
+  __device__ __forceinline__ void load(const void* base, size_t row, int H, int v) {
+    q = moe::ld_prod(reinterpret_cast<const uint4*>(static_cast<const __half*>(base) + row * H) +
+                     v);
+  }
+  __device__ __forceinline__ void get(float* f) const { moe::unpack8_f16(q, f); }
+};
+
+template <bool Y_F16, bool OUT_BF16, int KT>
+__global__ void __launch_bounds__(CNT) combine_kernel(const void* y,
                                                       const int32_t* inv_perm,
                                                       int T, int H, int k, int N,
-                                                      const float* shared,
+                                                      const void* shared,
                                                       const float* sgate,
                                                       const int32_t* range_offs,
                                                       int lo_e, int hi_e,
@@ -68,31 +95,27 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const float* y,
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       // all k rows' loads first (in flight together), then the sums in j order
-      float4 a[KT], b[KT];
+      Vec8<Y_F16> yv[KT];
+#pragma unroll
+      for (int j = 0; j < KT; ++j)
+        if (rows[j] >= 0) yv[j].load(y, static_cast<size_t>(rows[j]), H, v);
 #pragma unroll
       for (int j = 0; j < KT; ++j) {
         if (rows[j] >= 0) {
-          const float4* src =
-              reinterpret_cast<const float4*>(y + static_cast<size_t>(rows[j]) * H) + 2 * v;
-          a[j] = moe::ld_prod(src);
-          b[j] = moe::ld_prod(src + 1);
-        }
-      }
+          float f[8];
+          yv[j].get(f);
 #pragma unroll
-      for (int j = 0; j < KT; ++j) {
-        if (rows[j] >= 0) {
-          acc[0] += a[j].x; acc[1] += a[j].y; acc[2] += a[j].z; acc[3] += a[j].w;
-          acc[4] += b[j].x; acc[5] += b[j].y; acc[6] += b[j].z; acc[7] += b[j].w;
+          for (int i = 0; i < 8; ++i) acc[i] += f[i];
         }
       }
       if (shared) {
         const float g = gate;
-        const float4* src = reinterpret_cast<const float4*>(shared + static_cast<size_t>(t) * H) + 2 * v;
-        const float4 a = moe::ld_prod(src), b = moe::ld_prod(src + 1);
-        acc[0] = fmaf(g, a.x, acc[0]); acc[1] = fmaf(g, a.y, acc[1]);
-        acc[2] = fmaf(g, a.z, acc[2]); acc[3] = fmaf(g, a.w, acc[3]);
-        acc[4] = fmaf(g, b.x, acc[4]); acc[5] = fmaf(g, b.y, acc[5]);
-        acc[6] = fmaf(g, b.z, acc[6]); acc[7] = fmaf(g, b.w, acc[7]);
+        Vec8<Y_F16> sv;
+        sv.load(shared, static_cast<size_t>(t), H, v);
+        float f[8];
+        sv.get(f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
       }
       if (OUT_BF16) {
         reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(outv) + static_cast<size_t>(t) * H)[v] =
@@ -144,20 +167,19 @@ cudaError_t launch_finalize(const float* acc, int T, int H, int dtype, void* out
              : launch_pdl(finalize_kernel<false>, dim3(grid), dim3(CNT), 0, s, 0, a, nvec8, out);
 }
 
-cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
-                           const float* shared, const float* shared_gate, int dtype, void* out,
-                           int32_t* status, cudaStream_t s, const int32_t* range_offs, int lo_e,
-                           int hi_e) {
+template <bool Y_F16, bool OUT_BF16>
+cudaError_t launch_combine_t(const void* y, const int32_t* inv_perm, int T, int H, int k,
+                             const void* shared, const float* shared_gate, void* out,
+                             int32_t* status, cudaStream_t s, const int32_t* range_offs,
+                             int lo_e, int hi_e) {
   const int grid = std::max(1, std::min(T, num_sms() * 8));
   const int N = T * k;
   // k is a template parameter so that exactly k rows are loaded, all in flight.
 #define MOE_COMBINE_K(KV)                                                                     \
   case KV:                                                                                    \
-    return dtype == MOE_BF16                                                                  \
-               ? launch_pdl(combine_kernel<true, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,       \
-                            inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out, status)           \
-               : launch_pdl(combine_kernel<false, KV>, dim3(grid), dim3(CNT), 0, s, 0, y,      \
-                            inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out, status);
+    return launch_pdl(combine_kernel<Y_F16, OUT_BF16, KV>, dim3(grid), dim3(CNT), 0, s, 0, y, \
+                      inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out,  \
+                      status);
   switch (k) {
     MOE_COMBINE_K(1)
     MOE_COMBINE_K(2)
@@ -171,6 +193,24 @@ cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H
       return cudaErrorInvalidValue;
   }
 #undef MOE_COMBINE_K
+}
+
+cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv_perm, int T, int H,
+                           int k, const void* shared, const float* shared_gate, int dtype,
+                           void* out, int32_t* status, cudaStream_t s,
+                           const int32_t* range_offs, int lo_e, int hi_e) {
+  const bool yb = y_dtype == MOE_F16, ob = dtype == MOE_BF16;
+  if (yb && ob)
+    return launch_combine_t<true, true>(y, inv_perm, T, H, k, shared, shared_gate, out, status,
+                                        s, range_offs, lo_e, hi_e);
+  if (yb)
+    return launch_combine_t<true, false>(y, inv_perm, T, H, k, shared, shared_gate, out, status,
+                                         s, range_offs, lo_e, hi_e);
+  if (ob)
+    return launch_combine_t<false, true>(y, inv_perm, T, H, k, shared, shared_gate, out, status,
+                                         s, range_offs, lo_e, hi_e);
+  return launch_combine_t<false, false>(y, inv_perm, T, H, k, shared, shared_gate, out, status,
+                                        s, range_offs, lo_e, hi_e);
 }
 
 }  // namespace moe_host

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <string>
@@ -85,6 +86,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
+// Two fp32 values rounded to fp16 (nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 t = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+// Eight fp16 values (one 16-byte word) as fp32.
+__device__ __forceinline__ void unpack8_f16(const uint4& v, float* f) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+    const float2 t = __half22float2(h);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Largest finite fp16 value: a larger fp32 value does not fit an fp16 output.
+constexpr float kF16Max = 65504.f;
+
 }  // namespace moe
 
 // Host-side internal launchers (one translation unit each).  They assume the
@@ -128,15 +150,17 @@ struct SharedGroup {
 };
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, const SharedGroup* sh,
+                              int H, int I, int E, void* h, void* y, bool y_f16,
+                              const SharedGroup* sh,
                               void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s,
                               const char** why);
 cudaError_t launch_experts_simt(const void* x_packed, const int32_t* offsets,
                                 const float* packed_w, const void* w13, const void* w2, int N,
                                 int H, int I, int E, void* h, void* y, cudaStream_t s);
 // range_offs != NULL: only packed rows [range_offs[lo_e], range_offs[hi_e]) are added.
-cudaError_t launch_combine(const float* y, const int32_t* inv_perm, int T, int H, int k,
-                           const float* shared, const float* shared_gate, int dtype, void* out,
+cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv_perm, int T, int H,
+                           int k, const void* shared, const float* shared_gate, int dtype,
+                           void* out,
                            int32_t* status, cudaStream_t s, const int32_t* range_offs = nullptr,
                            int lo_e = 0, int hi_e = 0);
 cudaError_t launch_finalize(const float* acc, int T, int H, int dtype, void* out,

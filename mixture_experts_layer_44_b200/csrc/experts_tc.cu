@@ -57,7 +57,8 @@
 // keep the full budget, so nothing is in flight when the CTA leaves.
 //
 // CTA = 6 warps, one CTA per SM, persistent over units:
-//   warp 0    TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle)
+//   warp 0    TMA producer   (4-stage ring, 48 KB per stage, 128B swizzle;
+//                             5 stages of 36 KB when no tile has over 32 rows)
 //   warp 1    MMA issuer     (tcgen05.mma kind::f16, M128 N256 K16; owns TMEM)
 //   warps 2-5 epilogue       (tcgen05.ld from the TMEM accumulator, math, store)
 // The two 256-column fp32 accumulators are double-buffered in TMEM, so the
@@ -77,19 +78,12 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int MAX_STAGES = 5;
 constexpr int NTHREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
 constexpr int MAX_SPLITS = 16;
-// Weights that one unit alone reads (an expert whose rows fit one token tile:
-// decode batches) stream from HBM exactly once, and the stage ring alone
-// keeps too few bytes in flight per SM to reach full bandwidth.  Such units
-// also ask L2 for the k-block L2_AHEAD ahead of each one they load.
-constexpr int L2_AHEAD = 4;
 constexpr int COUNTER_INTS = 4096;                        // per-tile arrival counters, then
 constexpr int SCHED_TICKET = COUNTER_INTS - 2;            // the unit ticket and the
 constexpr int SCHED_DONE = COUNTER_INTS - 1;              // CTA exit count of dynamic scheduling
@@ -99,8 +93,8 @@ constexpr size_t PARTIAL_BYTES = sizeof(float) * BM * BN;  // one unit's partial
 enum { EPI_SWIGLU = 0, EPI_SCALE = 1 };
 
 struct Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -124,14 +118,30 @@ constexpr int STAGE_OUT_BYTES = BM * 128;                  // epilogue staging: 
 // The staging buffer starts on a 1024-byte boundary: TMA stores read it with
 // the 128-byte swizzle, whose pattern is anchored there.
 constexpr size_t CTL_BYTES = (sizeof(Ctl) + 1023) / 1024 * 1024;
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTL_BYTES + STAGE_OUT_BYTES;
+// The stage ring.  A stage holds the A tile (AR rows of activations) and
+// then the B tile (256 weight rows), each 64 columns wide.  AR = 128 in
+// general; AR = 32 when no tile has more than 32 rows (decode batches): the
+// MMA still reads 128 rows of A, the 96 beyond the loaded ones falling inside
+// the same stage's B tile -- garbage in accumulator rows that are never
+// stored -- and the 12 KB saved per stage buy a fifth stage, 25 % more weight
+// bytes in flight per SM.
+template <int AR>
+struct Ring {
+  static constexpr int A_B = AR * BK * 2;
+  static constexpr int ST_B = A_B + B_BYTES;
+  static constexpr int N = AR == BM ? 4 : 5;
+  static constexpr size_t SMEM = 1024 + N * ST_B + CTL_BYTES + STAGE_OUT_BYTES;
+  static_assert(AR == BM || (AR >= 8 && AR % 8 == 0 && A_B + B_BYTES >= BM * BK * 2),
+                "a short A tile must be followed by at least 128 rows' worth of the stage");
+  static_assert(N <= MAX_STAGES && SMEM <= 227 * 1024, "stage ring exceeds shared memory");
+  static_assert(ST_B % 1024 == 0 && A_B % 1024 == 0, "tiles must stay 1024-byte aligned");
+};
 
 // A work unit: tile (group g, expert e, weight tile nt, token tile mt) and
 // its K-slice [kb0, kb1).  Group 1 is the optional shared expert (all rows of
 // its own input), group 0 the routed experts.  Its rows are [row0, rend).
 struct Unit {
   int tile, g, e, nt, mt, ks, S, kb0, kb1, row0, rend;
-  bool stream;   // the group's rows fit one token tile: no other unit reads these weights
 };
 
 template <bool SHARED>
@@ -160,7 +170,6 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     r.mt = r.tile - r.nt * c.mte2;
     r.row0 = r.mt * BM;
     r.rend = c.rows2;
-    r.stream = c.mte2 == 1;
     kb = kblocks2;
   } else {
     // largest e with tstart[e] <= tile (experts without tiles share their successor's start)
@@ -177,7 +186,6 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     r.mt = local - r.nt * mte;
     r.row0 = c.offs[r.e] + r.mt * BM;
     r.rend = c.offs[r.e + 1];
-    r.stream = mte == 1;
     kb = kblocks;
   }
   r.kb0 = (r.ks * kb) / r.S;
@@ -287,7 +295,46 @@ __device__ __forceinline__ void stage_f32x32(uint8_t* stg, int row, const uint32
                          __float_as_uint(__uint_as_float(b[4 * j + 3]) * sc)));
 }
 
-template <int EPI, bool SHARED>
+// 64 fp32 accumulator columns (four TMEM loads) scaled by sc and rounded to
+// fp16 -> 8 staged chunks (128 bytes of the row).  Returns the largest
+// magnitude stored (for the fp16 range check).
+__device__ __forceinline__ uint4 h16x8(const uint32_t* a, float sc, float& mx) {
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = __uint_as_float(a[i]) * sc;
+    mx = fmaxf(mx, fabsf(v[i]));
+  }
+  return make_uint4(moe::pack_f16x2(v[0], v[1]), moe::pack_f16x2(v[2], v[3]),
+                    moe::pack_f16x2(v[4], v[5]), moe::pack_f16x2(v[6], v[7]));
+}
+
+__device__ __forceinline__ float stage_h16x64(uint8_t* stg, int row, const uint32_t (&a)[4][16],
+                                              float sc) {
+  float mx = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) stage_put(stg, row, 2 * q + j, h16x8(&a[q][8 * j], sc, mx));
+  return mx;
+}
+
+// The same 64 columns stored directly to one fp16 row (dst: 16-byte aligned).
+__device__ __forceinline__ float store_h16x64(__half* dst, const uint32_t (&a)[4][16], float sc) {
+  float mx = 0.f;
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) d4[2 * q + j] = h16x8(&a[q][8 * j], sc, mx);
+  return mx;
+}
+
+// YH (pass 2 only): y_packed and the shared expert's y are fp16 -- each
+// element rounded once, after the fp32 accumulation and the routing-weight
+// scale -- instead of fp32.  A magnitude above the fp16 range is reported
+// (MOE_ERR_OVERFLOW); the element becomes inf.
+template <int EPI, bool SHARED, bool YH, int AR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -301,6 +348,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         void* __restrict__ out2, int ldo2, int* __restrict__ counters,
                         float* __restrict__ partials, int max_units, int32_t* status,
                         uint64_t wait_ns) {
+  using RG = Ring<AR>;
+  constexpr int STAGES = RG::N;
+  constexpr int A_BYTES = RG::A_B;
+  constexpr int STAGE_BYTES = RG::ST_B;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -530,7 +581,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
             load_b(un, kb, sa, fb);
             ++issued[stage];
-            if (L2_AHEAD > 0 && un.stream && kb + L2_AHEAD < un.kb1) prefetch_b(un, kb + L2_AHEAD);
           }
           if (++stage == STAGES) {
             stage = 0;
@@ -708,13 +758,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // global stores and no barrier spans the warps; a partly valid
           // quarter stores its valid rows directly.
           const float sc = live ? (upw ? moe::ld_prod(upw + grow) : 1.f) : 0.f;
-          uint8_t* gtile =
-              static_cast<uint8_t*>(uout) + (row0 * uldo + un.nt * BN) * sizeof(float);
           const int qrows = min(max(nvalid - q * 32, 0), 32);
           const CUtensorMap* ym = g1 ? &tmY2 : &tmY;
           const uint32_t wstg = moe::smem_addr(stg + q * 32 * 128);
+          if (YH) {
+            // fp16 output, 64 columns (one 128-byte staged row) per step
+            __half* yrow = static_cast<__half*>(uout) + grow * uldo + un.nt * BN;
+            float mx = 0.f;
 #pragma unroll 1
-          for (int cc = 0; cc < BN; cc += 32) {
+            for (int cc = 0; cc < BN; cc += 64) {
+              uint32_t a[4][16];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) moe::tmem_ld16(taddr + cc + 16 * j, a[j]);
+              moe::tmem_ld_wait();
+              if (qrows == 32) {
+                if (lane == 0) moe::bulk_wait_read_all();   // the last store has read the stage
+                __syncwarp();
+                mx = fmaxf(mx, stage_h16x64(stg, row, a, sc));
+                moe::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  moe::tma_store_2d(ym, wstg, un.nt * BN + cc, static_cast<int>(row0) + q * 32);
+                  moe::bulk_commit();
+                }
+              } else if (live) {
+                mx = fmaxf(mx, store_h16x64(yrow + cc, a, sc));
+              }
+            }
+            if (mx > moe::kF16Max) moe::report(status, MOE_ERR_OVERFLOW);
+          }
+          uint8_t* gtile =
+              static_cast<uint8_t*>(uout) + (row0 * uldo + un.nt * BN) * sizeof(float);
+#pragma unroll 1
+          for (int cc = 0; cc < (YH ? 0 : BN); cc += 32) {
             uint32_t a[16], b[16];
             moe::tmem_ld16(taddr + cc, a);
             moe::tmem_ld16(taddr + cc + 16, b);
@@ -820,9 +896,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
               }
               const float sc = upw ? moe::ld_prod(upw + row0 + r) : 1.f;
-              *reinterpret_cast<float4*>(static_cast<float*>(uout) + (row0 + r) * uldo +
-                                         un.nt * BN + cg * 4) =
-                  make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
+              if (YH) {
+                const float4 o = make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
+                if (fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))) >
+                    moe::kF16Max)
+                  moe::report(status, MOE_ERR_OVERFLOW);
+                uint2 pk;
+                pk.x = moe::pack_f16x2(o.x, o.y);
+                pk.y = moe::pack_f16x2(o.z, o.w);
+                *reinterpret_cast<uint2*>(static_cast<__half*>(uout) + (row0 + r) * uldo +
+                                          un.nt * BN + cg * 4) = pk;
+              } else {
+                *reinterpret_cast<float4*>(static_cast<float*>(uout) + (row0 + r) * uldo +
+                                           un.nt * BN + cg * 4) =
+                    make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
+              }
             }
           }
         }
@@ -847,11 +935,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// Activations [rows, K] bf16, box 64 x 128.
-bool map_rows(CUtensorMap* m, const void* p, int rows, int K) {
+// Activations [rows, K] bf16, box 64 x ar (the A tile of one stage).
+bool map_rows(CUtensorMap* m, const void* p, int rows, int K, int ar) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t box[2] = {BK, static_cast<cuuint32_t>(ar)};
   return moe_host::encode_bf16_sw128(m, p, 2, dims, str, box);
 }
 
@@ -864,6 +952,14 @@ bool map_out_f32(CUtensorMap* m, const void* p, int rows, int cols) {
   return moe_host::encode_f32_sw128(m, p, 2, dims, str, box);
 }
 
+// fp16 outputs [rows, cols]: box of 64 columns (128 bytes) x 32 rows.
+bool map_out_f16(CUtensorMap* m, const void* p, int rows, int cols) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t str[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, 32};
+  return moe_host::encode_f16_sw128(m, p, 2, dims, str, box);
+}
+
 }  // namespace
 
 namespace moe_host {
@@ -872,21 +968,48 @@ size_t experts_ws_bytes() {
   return sizeof(int) * COUNTER_INTS + PARTIAL_BYTES * 4 * static_cast<size_t>(num_sms());
 }
 
+namespace {
+
+// Every instance of the kernel has this signature.
+using GemmFn = decltype(&grouped_gemm_kernel<EPI_SWIGLU, false, false, BM>);
+
+// The kernels of both passes for one A-tile height (AR rows).
+template <int AR>
+void pick_kernels(bool shared, bool y_f16, GemmFn* k1, GemmFn* k2) {
+  *k1 = shared ? grouped_gemm_kernel<EPI_SWIGLU, true, false, AR>
+               : grouped_gemm_kernel<EPI_SWIGLU, false, false, AR>;
+  *k2 = y_f16 ? (shared ? grouped_gemm_kernel<EPI_SCALE, true, true, AR>
+                        : grouped_gemm_kernel<EPI_SCALE, false, true, AR>)
+              : (shared ? grouped_gemm_kernel<EPI_SCALE, true, false, AR>
+                        : grouped_gemm_kernel<EPI_SCALE, false, false, AR>);
+}
+
+}  // namespace
+
 cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                               const float* packed_w, const void* w13, const void* w2, int N,
-                              int H, int I, int E, void* h, void* y, const SharedGroup* sh,
-                              void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s,
-                              const char** why) {
+                              int H, int I, int E, void* h, void* y, bool y_f16,
+                              const SharedGroup* sh, void* ws, size_t ws_bytes, int32_t* status,
+                              cudaStream_t s, const char** why) {
+  // A tile of at most 32 rows needs only 32 rows of A per stage: every
+  // expert has at most N rows, the shared expert T2.
+  const int T2 = sh ? sh->T : 0, Is = sh ? sh->I : 0;
+  const bool short_a = N <= 32 && T2 <= 32;
+  const int ar = short_a ? 32 : BM;
   // The shared-expert group is compiled in only where it is used.
-  auto k1 = sh ? grouped_gemm_kernel<EPI_SWIGLU, true> : grouped_gemm_kernel<EPI_SWIGLU, false>;
-  auto k2 = sh ? grouped_gemm_kernel<EPI_SCALE, true> : grouped_gemm_kernel<EPI_SCALE, false>;
-  cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(k1), static_cast<int>(SMEM_BYTES));
+  GemmFn k1, k2;
+  if (short_a)
+    pick_kernels<32>(sh != nullptr, y_f16, &k1, &k2);
+  else
+    pick_kernels<BM>(sh != nullptr, y_f16, &k1, &k2);
+  const size_t smem = short_a ? Ring<32>::SMEM : Ring<BM>::SMEM;
+  cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(k1), static_cast<int>(smem));
   if (e1 != cudaSuccess) return e1;
-  e1 = ensure_smem(reinterpret_cast<const void*>(k2), static_cast<int>(SMEM_BYTES));
+  e1 = ensure_smem(reinterpret_cast<const void*>(k2), static_cast<int>(smem));
   if (e1 != cudaSuccess) return e1;
   const int nmap = N > 0 ? N : 1;           // a map needs one row; no tile reads it when N == 0
   CUtensorMap mA1, mB1, mA2, mB2;
-  bool ok = map_rows(&mA1, x_packed, nmap, H) && map_rows(&mA2, h, nmap, I);
+  bool ok = map_rows(&mA1, x_packed, nmap, H, ar) && map_rows(&mA2, h, nmap, I, ar);
   {
     // w13 as [2E][I][H]: one box = 128 gate rows + the matching 128 up rows.
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
@@ -906,9 +1029,8 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   // The shared expert's maps (x [T][H], w13s as [2][Is][H], h_s [T][Is], w2s [H][Is]);
   // without one the routed maps stand in, unread.
   CUtensorMap sA1 = mA1, sB1 = mB1, sA2 = mA2, sB2 = mB2;
-  const int T2 = sh ? sh->T : 0, Is = sh ? sh->I : 0;
   if (sh) {
-    ok = ok && map_rows(&sA1, sh->x, T2, H) && map_rows(&sA2, sh->h, T2, Is);
+    ok = ok && map_rows(&sA1, sh->x, T2, H, ar) && map_rows(&sA2, sh->h, T2, Is, ar);
     const cuuint64_t d1[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(Is), 2};
     const cuuint64_t s1[2] = {static_cast<cuuint64_t>(H) * 2,
                               static_cast<cuuint64_t>(Is) * H * 2};
@@ -919,11 +1041,12 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     const cuuint32_t b2[2] = {BK, BN};
     ok = ok && encode_bf16_sw128(&sB2, sh->w2, 2, d2, s2, b2);
   }
-  // the w2 pass's fp32 outputs (the shared expert's own, or the routed map standing in)
+  // the w2 pass's outputs (the shared expert's own, or the routed map standing in)
+  auto map_out = y_f16 ? map_out_f16 : map_out_f32;
   CUtensorMap mY, sY;
-  ok = ok && map_out_f32(&mY, y, nmap, H);
+  ok = ok && map_out(&mY, y, nmap, H);
   sY = mY;
-  if (sh) ok = ok && map_out_f32(&sY, sh->y, T2, H);
+  if (sh) ok = ok && map_out(&sY, sh->y, T2, H);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
     return cudaErrorInvalidValue;
@@ -950,15 +1073,15 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     g2 = std::max(1, std::min(sms, (mt_bound + mt2) * (H / BN)));
   }
   const float* no_w = nullptr;
-  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS),
-                               SMEM_BYTES, s, 0, mA1, mB1, sA1, sB1, mY, sY, offsets, E, H, ntw1,
-                               2 * I, no_w, h, I, T2, H, ntw1s, sh ? sh->h : nullptr, Is,
-                               counters, partials, max_units, status, main_wait_budget_ns());
+  const uint64_t wait_ns = main_wait_budget_ns();
+  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS), smem, s, 0, mA1, mB1, sA1, sB1,
+                               mY, sY, offsets, E, H, ntw1, 2 * I, no_w, h, I, T2, H, ntw1s,
+                               sh ? sh->h : nullptr, Is, counters, partials, max_units, status,
+                               wait_ns);
   if (err != cudaSuccess) return err;
-  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), SMEM_BYTES, s, 0,
-                    mA2, mB2, sA2, sB2, mY, sY, offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
-                    sh ? sh->y : nullptr, H, counters, partials, max_units, status,
-                    main_wait_budget_ns());
+  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), smem, s, 0, mA2, mB2, sA2, sB2, mY, sY,
+                    offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
+                    sh ? sh->y : nullptr, H, counters, partials, max_units, status, wait_ns);
 }
 
 }  // namespace moe_host

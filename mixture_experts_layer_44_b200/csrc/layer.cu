@@ -22,6 +22,8 @@ struct moe_layer {
   moe_layer_desc d;
   int N;
   int es;                        // activation bytes
+  int y_dtype;                   // y_packed and the shared expert's output
+  int ys;                        // their element bytes
   bool fuse_shared;
   // device buffers (carved from the caller's block)
   void* x[2];
@@ -37,7 +39,7 @@ struct moe_layer {
   float* packed_w;
   void* x_packed;
   void* h;
-  float* y_packed;
+  void* y_packed;
   void* dws;
   size_t dws_bytes;
   void* ews;
@@ -46,7 +48,7 @@ struct moe_layer {
   int32_t* counter;              // ticket of the fused small-batch route+dispatch
   float* sg_logit;
   void* sh_h;
-  float* sh_y;
+  void* sh_y;
   int32_t* sh_offsets;
   // host-buffer pipeline
   cudaStream_t s_in, s_comp, s_out;
@@ -88,7 +90,7 @@ size_t layout(moe_layer* L, uint8_t* base) {
   L->packed_w = static_cast<float*>(c.take(N * 4));
   L->x_packed = c.take(N * H * es);
   L->h = c.take(N * I * es);
-  L->y_packed = static_cast<float*>(c.take(N * H * 4));
+  L->y_packed = c.take(N * H * L->ys);
   L->dws_bytes = moe_host::dispatch_ws_bytes(d.T, d.k, d.E);
   L->dws = c.take(L->dws_bytes);
   L->ews_bytes = d.dtype == MOE_BF16 ? moe_host::experts_ws_bytes() : 0;
@@ -98,7 +100,7 @@ size_t layout(moe_layer* L, uint8_t* base) {
   if (d.w13s != nullptr) {
     L->sg_logit = static_cast<float*>(c.take(T * 4));
     L->sh_h = c.take(T * static_cast<size_t>(d.I_s) * es);
-    L->sh_y = static_cast<float*>(c.take(T * H * 4));
+    L->sh_y = c.take(T * H * L->ys);
     L->sh_offsets = static_cast<int32_t*>(c.take(8));
   } else {
     L->sg_logit = nullptr;
@@ -161,7 +163,8 @@ cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
   if (d.dtype == MOE_BF16) {
     moe_host::SharedGroup g{x, d.T, d.w13s, d.w2s, d.I_s, L->sh_h, L->sh_y};
     e = moe_host::launch_experts_tc(L->x_packed, L->offsets, L->packed_w, d.w13, d.w2, L->N, d.H,
-                                    d.I, d.E, L->h, L->y_packed, shared ? &g : nullptr, L->ews,
+                                    d.I, d.E, L->h, L->y_packed, L->y_dtype == MOE_F16,
+                                    shared ? &g : nullptr, L->ews,
                                     L->ews_bytes, L->status, s, &why);
   } else {
     e = moe_host::launch_experts_simt(L->x_packed, L->offsets, L->packed_w, d.w13, d.w2, L->N,
@@ -171,7 +174,7 @@ cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
                                         d.I_s, 1, L->sh_h, L->sh_y, s);
   }
   if (e != cudaSuccess) return e;
-  return moe_host::launch_combine(L->y_packed, L->inv_perm, d.T, d.H, d.k,
+  return moe_host::launch_combine(L->y_packed, L->y_dtype, L->inv_perm, d.T, d.H, d.k,
                                   shared ? L->sh_y : nullptr, shared ? L->sg_logit : nullptr,
                                   d.dtype, out, L->status, s);
 }
@@ -207,6 +210,8 @@ size_t moe_layer_workspace_bytes(const moe_layer_desc* d) {
   memset(&tmp, 0, sizeof(tmp));
   tmp.d = *d;
   tmp.es = d->dtype == MOE_BF16 ? 2 : 4;
+  tmp.y_dtype = d->dtype == MOE_BF16 && !d->y_f32 ? MOE_F16 : MOE_F32;
+  tmp.ys = tmp.y_dtype == MOE_F16 ? 2 : 4;
   return layout(&tmp, nullptr);
 }
 
@@ -228,6 +233,8 @@ int moe_layer_create(const moe_layer_desc* d, void* workspace, size_t workspace_
   L->d = *d;
   if (L->d.n_groups < 1) L->d.n_groups = 1;
   L->es = d->dtype == MOE_BF16 ? 2 : 4;
+  L->y_dtype = d->dtype == MOE_BF16 && !d->y_f32 ? MOE_F16 : MOE_F32;
+  L->ys = L->y_dtype == MOE_F16 ? 2 : 4;
   L->N = d->T * d->k;
   layout(L, static_cast<uint8_t*>(workspace));
   cudaStream_t s = static_cast<cudaStream_t>(stream);

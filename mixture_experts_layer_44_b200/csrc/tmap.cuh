@@ -14,6 +14,10 @@ namespace moe_host {
 bool encode_bf16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                        const cuuint64_t* strides_bytes, const cuuint32_t* box);
 
+// The same for an fp16 tensor (the target of TMA stores).
+bool encode_f16_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                      const cuuint64_t* strides_bytes, const cuuint32_t* box);
+
 // The same for an fp32 tensor (used as the target of TMA stores).
 bool encode_f32_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
                       const cuuint64_t* strides_bytes, const cuuint32_t* box);

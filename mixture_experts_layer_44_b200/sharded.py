@@ -228,8 +228,11 @@ class A2ABuffers:
         dev = torch.device(device)
         self.T, self.H, self.E, self.k, self.world = T, H, E, k, world
         self.dtype, self.device, self.shared_I = dtype, dev, shared_I
-        # routing and the by-owner dispatch of this rank's assignments
-        self.route = MoELayerBuffers(T, H, E, k, 8, dtype, device=dev, shared_I=shared_I)
+        # routing and the by-owner dispatch of this rank's assignments; the
+        # merge takes the returned rows as fp32, so the shared expert's output
+        # (merged beside them) is fp32 too
+        self.route = MoELayerBuffers(T, H, E, k, 8, dtype, device=dev, shared_I=shared_I,
+                                     y_f32=True)
         self.owner = torch.empty(T, k, dtype=torch.int32, device=dev)
         self.send = MoELayerBuffers(T, H, world, k, 8, dtype, device=dev)
         self.send_eid = torch.empty(T * k, dtype=torch.int32, device=dev)
@@ -259,7 +262,7 @@ def a2a_experts(x_recv, eid_recv, w_recv, params_local: dict, buf: A2ABuffers, s
     """Owner side: the rows this rank received (token rows, its own expert
     ids, routing weights) dispatched by local expert, run through its experts
     (weights applied there) and put back in the order they arrived.  Returns
-    y [n_recv, H] fp32."""
+    y [n_recv, H] fp32 (the executor's values exactly: k = 1 adds nothing)."""
     n_recv = x_recv.shape[0]
     y_recv = torch.empty(n_recv, buf.H, dtype=torch.float32, device=buf.device)
     if n_recv == 0:

@@ -78,3 +78,27 @@ def err_bf16_out(got, want) -> float:
     rms = float(np.sqrt(np.mean(w * w)))
     excess = np.maximum(np.abs(g - w) - bf16_half_ulp(np.maximum(np.abs(g), np.abs(w))), 0.0)
     return float(excess.max()) / rms if g.size else 0.0
+
+
+def f16_half_ulp(a: np.ndarray) -> np.ndarray:
+    """Half an fp16 ulp at |a| (11 significant bits; below 2^-14 the
+    subnormal spacing 2^-24): the most a correctly rounded fp16 store can
+    move a value inside the fp16 range."""
+    a = np.abs(a)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 11)
+
+
+def err_stored(got, want) -> float:
+    """Error of a STORED tensor against its fp64 reference, normalised by
+    rms(reference): beyond the store's own final rounding for bf16 and fp16
+    tensors (half an ulp of the larger magnitude), plain for fp32."""
+    if got.dtype == torch.bfloat16:
+        return err_bf16_out(got, want)
+    if got.dtype != torch.float16:
+        return rel(got, want)
+    g = O.to_f64(got)
+    w = O.to_f64(want)
+    rms = float(np.sqrt(np.mean(w * w)))
+    excess = np.maximum(np.abs(g - w) - f16_half_ulp(np.maximum(np.abs(g), np.abs(w))), 0.0)
+    return float(excess.max()) / rms if g.size else 0.0

@@ -52,7 +52,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_workspace_queries(lib):
-    assert M.moe_abi_version() == 3
+    assert M.moe_abi_version() == 4
     assert M.moe_launch_count() == 0     # nothing launched on a CPU-only host
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
@@ -122,7 +122,7 @@ def test_route_dispatch_rejects_bad_arguments_on_the_host(lib):
 
 
 def test_experts_rejects_bad_arguments_on_the_host(lib):
-    base = [P, P, P, P, P, 100, 256, 128, 4, M.MOE_BF16, P, P, NULL, 0, NULL, NULL]
+    base = [P, P, P, P, P, 100, 256, 128, 4, M.MOE_BF16, M.MOE_F16, P, P, NULL, 0, NULL, NULL]
     a = list(base); a[6] = 200            # H not a multiple of 256 on the bf16 path
     assert lib.moe_experts(*a) == M.MOE_ERR_UNSUPPORTED and "H % 256" in _err(lib)
     a = list(base); a[7] = 100            # I not a multiple of 8
@@ -133,28 +133,40 @@ def test_experts_rejects_bad_arguments_on_the_host(lib):
     assert lib.moe_experts(*a) == M.MOE_OK
     a = list(base); a[3] = NULL
     assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[9] = M.MOE_F32      # fp32 layers keep y_packed in fp32
+    assert lib.moe_experts(*a) == M.MOE_ERR_UNSUPPORTED and "y_dtype" in _err(lib)
+    a = list(base); a[10] = 5             # no such y type
+    assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(base); a[10] = M.MOE_BF16    # y_packed is fp16 or fp32 only
+    assert lib.moe_experts(*a) == M.MOE_ERR_INVALID_ARG and "y_dtype" in _err(lib)
 
 
 def test_experts_shared_rejects_bad_arguments_on_the_host(lib):
-    # routed part as above, then x, T, w13s, w2s, I_s, dtype, h, y, h_s, y_s, ws, bytes, status, stream
-    base = [P, P, P, P, P, 100, 256, 128, 4, P, 32, P, P, 512, M.MOE_BF16, P, P, P, P, NULL, 0,
-            NULL, NULL]
+    # routed part as above, then x, T, w13s, w2s, I_s, dtype, y_dtype, h, y, h_s, y_s, ws,
+    # bytes, status, stream
+    base = [P, P, P, P, P, 100, 256, 128, 4, P, 32, P, P, 512, M.MOE_BF16, M.MOE_F16, P, P, P,
+            P, NULL, 0, NULL, NULL]
     a = list(base); a[13] = 100           # I_s not a multiple of 128
     assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED and "I_s" in _err(lib)
     a = list(base); a[10] = 0             # T < 1
     assert lib.moe_experts_shared(*a) == M.MOE_ERR_INVALID_ARG
-    a = list(base); a[18] = NULL          # no y_s
+    a = list(base); a[19] = NULL          # no y_s
     assert lib.moe_experts_shared(*a) == M.MOE_ERR_INVALID_ARG
     a = list(base); a[14] = M.MOE_F32     # fp32 runs the two experts separately
+    a[15] = M.MOE_F32
     assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED
     a = list(base); a[6] = 200            # the routed rules still apply
     assert lib.moe_experts_shared(*a) == M.MOE_ERR_UNSUPPORTED and "H % 256" in _err(lib)
 
 
 def test_combine_and_status_reject_bad_arguments_on_the_host(lib):
-    assert lib.moe_combine(P, P, 4, 64, 0, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
-    assert lib.moe_combine(P, P, 4, 63, 2, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
-    assert lib.moe_combine(NULL, P, 4, 64, 2, NULL, NULL, M.MOE_BF16, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    B, F = M.MOE_BF16, M.MOE_F16
+    assert lib.moe_combine(P, F, P, 4, 64, 0, NULL, NULL, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(P, F, P, 4, 63, 2, NULL, NULL, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(NULL, F, P, 4, 64, 2, NULL, NULL, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(P, 3, P, 4, 64, 2, NULL, NULL, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(P, B, P, 4, 64, 2, NULL, NULL, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert "y_dtype" in _err(lib)
     v = ctypes.c_int32(0)
     assert lib.moe_read_status(NULL, NULL, ctypes.byref(v)) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_probe_wait_timeout(P, 0, NULL) == M.MOE_ERR_INVALID_ARG
@@ -172,8 +184,11 @@ def test_layer_descriptor_is_checked_on_the_host(lib):
     d = M.MoELayerDesc(T=64, H=256, E=8, k=2, I=128, dtype=M.MOE_BF16, renormalize=1,
                        n_groups=1, topk_groups=1, W_gate=256, bias=None, w13=512, w2=768)
     n = lib.moe_layer_workspace_bytes(ctypes.byref(d))
-    # two copies each of x and out, the packed buffers, fp32 y_packed, the workspaces
-    assert n >= 4 * 64 * 256 * 2 + 128 * 256 * 2 + 128 * 128 * 2 + 128 * 256 * 4
+    # two copies each of x and out, the packed buffers, fp16 y_packed, the workspaces
+    assert n >= 4 * 64 * 256 * 2 + 128 * 256 * 2 + 128 * 128 * 2 + 128 * 256 * 2
+    f = M.MoELayerDesc.from_buffer_copy(d)
+    f.y_f32 = 1                                 # fp32 y_packed: 2 more bytes per element
+    assert lib.moe_layer_workspace_bytes(ctypes.byref(f)) >= n + 128 * 256 * 2
     for field, bad in (("I", 100), ("k", 9), ("E", 0), ("dtype", 7), ("H", 200)):
         b = M.MoELayerDesc.from_buffer_copy(d)
         setattr(b, field, bad)
@@ -205,7 +220,7 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
     # range gather / merge: 0 <= start <= end <= E
     assert lib.moe_gather(P, P, P, 8, 3, 9, 16, 64, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_gather(P, P, P, 8, 5, 4, 16, 64, B, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
-    assert lib.moe_combine_range(P, P, P, 8, -1, 4, 4, 64, 2, NULL, NULL, M.MOE_F32, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_range(P, M.MOE_F16, P, P, 8, -1, 4, 4, 64, 2, NULL, NULL, M.MOE_F32, P, NULL, NULL) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_finalize(NULL, 4, 64, B, P, NULL) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_finalize(P, 4, 60, B, P, NULL) == M.MOE_ERR_INVALID_ARG
     # owner ids: at most one rank per expert

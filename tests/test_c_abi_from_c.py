@@ -18,7 +18,7 @@ PROGRAM = textwrap.dedent(r"""
 
     int main(void) {
       int fails = 0;
-      if (moe_abi_version() != 3) { puts("version"); ++fails; }
+      if (moe_abi_version() != 4) { puts("version"); ++fails; }
       if (moe_launch_count() != 0ull) { puts("launch count"); ++fails; }
       /* null x: rejected on the host before anything is enqueued */
       float logits[4];
@@ -30,7 +30,7 @@ PROGRAM = textwrap.dedent(r"""
       /* nothing to do: OK without touching the GPU */
       int dummy[4];
       r = moe_experts((void*)dummy, dummy, NULL, (void*)dummy, (void*)dummy, 0, 256, 128, 4,
-                      MOE_BF16, (void*)dummy, (void*)dummy, NULL, 0, NULL, NULL);
+                      MOE_BF16, MOE_F16, (void*)dummy, (void*)dummy, NULL, 0, NULL, NULL);
       if (r != MOE_OK) { puts("experts N=0"); ++fails; }
       if (moe_dispatch_workspace_bytes(16384, 8, 128) < (size_t)64 * 128 * 4) {
         puts("dispatch ws"); ++fails;

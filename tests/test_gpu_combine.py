@@ -1,9 +1,10 @@
 """Merger parity: GPU moe_combine against the oracle's combine().
 
-y_packed and the shared output are fp32; the only roundings on the GPU are
-the fp32 sum of k (+1) terms and one final rounding to the output type, so
-the bound is per element: |gpu - oracle| <= 2^-8 |oracle| + 1e-6 rms for a
-bf16 output, 1e-6 |oracle| + 1e-6 rms for an fp32 output.
+y_packed and the shared output come as fp16 or fp32 (the oracle reads the
+same values); the only roundings on the GPU are the fp32 sum of k (+1) terms
+and one final rounding to the output type, so the bound is per element:
+|gpu - oracle| <= 2^-8 |oracle| + 1e-6 rms for a bf16 output, 1e-6 |oracle| +
+1e-6 rms for an fp32 output.
 """
 import numpy as np
 import pytest
@@ -35,10 +36,11 @@ def _bound(got, want, dtype):
 @pytest.mark.parametrize("T,k,H", [(1, 1, 8), (64, 2, 128), (333, 8, 2048), (4096, 2, 4096),
                                    (32, 4, 2048), (7, 3, 72)])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_combine(T, k, H, dtype):
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.float16])
+def test_combine(T, k, H, dtype, y_dtype):
     rng = np.random.default_rng(T + k)
     N = T * k
-    y = torch.randn(N, H, generator=torch.Generator().manual_seed(N))
+    y = torch.randn(N, H, generator=torch.Generator().manual_seed(N)).to(y_dtype)
     inv = torch.tensor(rng.permutation(N), dtype=torch.int32)
     out, st = _run(y, inv, T, k, out_dtype=dtype)
     assert st == 0
@@ -46,12 +48,13 @@ def test_combine(T, k, H, dtype):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_combine_with_shared_expert_gate(dtype):
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.float16])
+def test_combine_with_shared_expert_gate(dtype, y_dtype):
     g = torch.Generator().manual_seed(9)
     T, k, H = 50, 4, 256
-    y = torch.randn(T * k, H, generator=g)
+    y = torch.randn(T * k, H, generator=g).to(y_dtype)
     inv = torch.randperm(T * k, generator=g).to(torch.int32)
-    sh = torch.randn(T, H, generator=g)
+    sh = torch.randn(T, H, generator=g).to(y_dtype)
     sg = torch.randn(T, generator=g) * 3
     out, st = _run(y, inv, T, k, sh, sg, out_dtype=dtype)
     assert st == 0
