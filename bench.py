@@ -648,14 +648,18 @@ def main():
     ap.add_argument("--profile-small", action="store_true",
                     help="the workload with E=16 experts and T=1024 tokens (weights 0.55 GB, "
                          "still above L2): the case detailed ncu captures run on")
+    ap.add_argument("--profile-shape", type=int, nargs=2, metavar=("E", "T"),
+                    help="the workload with at most E experts and T tokens (a mid-size case "
+                         "for detailed ncu captures: a few GB on the device)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     cfg = CONFIGS[args.workload]
-    if args.profile_small:
+    if args.profile_small or args.profile_shape:
         import dataclasses
-        cfg = dataclasses.replace(cfg, name=cfg.name + "_e16_t1024", E=min(cfg.E, 16),
-                                  T=min(cfg.T, 1024))
+        pe, pt = args.profile_shape or (16, 1024)
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_e{pe}_t{pt}", E=min(cfg.E, pe),
+                                  T=min(cfg.T, pt))
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_gpu(args, cfg)
