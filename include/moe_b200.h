@@ -547,18 +547,6 @@ int moe_probe_wait_timeout(int32_t* status, int budget_us, void* stream);
  */
 int moe_test_set_wait_budget_ns(unsigned long long ns);
 
-/*
- * Testing hook: how the grouped GEMM of moe_experts tiles its work.
- *   0  automatic (default): 128-row tiles on one CTA, or 256-row tiles on a
- *      pair of CTAs (a cluster of 2 sharing each tcgen05 MMA, cta_group::2)
- *      when the experts average at least 256 rows (N >= 8192, N >= 256 * E);
- *   1  always 128-row tiles;
- *   2  CTA pairs whenever a tile can hold more than 32 rows.
- * Results are the same up to the fp32 summation order (pairs never split K).
- * Process-wide; returns MOE_ERR_INVALID_ARG for other values.
- */
-int moe_test_set_gemm_mode(int mode);
-
 #ifdef __cplusplus
 }
 #endif

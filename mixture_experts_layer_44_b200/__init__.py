@@ -30,7 +30,7 @@ __all__ = [
     "moe_layer_forward", "moe_route_dispatch", "route_dispatch_fits", "route_and_dispatch",
     "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
     "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
-    "MoELayerDesc", "MoELayer", "moe_test_set_wait_budget_ns", "moe_test_set_gemm_mode",
+    "MoELayerDesc", "MoELayer", "moe_test_set_wait_budget_ns",
 ]
 
 (MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT,
@@ -76,7 +76,6 @@ _SIGS = {
                                 _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_layer_workspace_bytes": (_SZ, [_P]),
     "moe_test_set_wait_budget_ns": (_I, [ctypes.c_ulonglong]),
-    "moe_test_set_gemm_mode": (_I, [_I]),
     "moe_layer_create": (_I, [_P, _P, _SZ, _P, _P]),
     "moe_layer_destroy": (_I, [_P]),
     "moe_layer_forward": (_I, [_P, _P, _P, _P]),
@@ -329,11 +328,6 @@ def moe_read_status(status, stream=None) -> int:
 def moe_test_set_wait_budget_ns(ns: int):
     """Testing hook: budget of the tensor-core kernels' main-loop waits (0 = default)."""
     _check(load_library().moe_test_set_wait_budget_ns(ns))
-
-
-def moe_test_set_gemm_mode(mode: int):
-    """Testing hook: 0 automatic, 1 always 1-CTA tiles, 2 CTA pairs (M = 256)."""
-    _check(load_library().moe_test_set_gemm_mode(int(mode)))
 
 
 def moe_probe_wait_timeout(status, budget_us: int, stream=None):

@@ -67,9 +67,6 @@ void set_last_error(const std::string& msg) { g_err = msg; }
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 uint64_t main_wait_budget_ns() { return g_main_wait_ns.load(std::memory_order_relaxed); }
 
-std::atomic<int> g_gemm_mode{0};
-int gemm_mode() { return g_gemm_mode.load(std::memory_order_relaxed); }
-
 cudaError_t ensure_smem(const void* kernel, int bytes) {
   static std::mutex mu;
   static std::map<std::tuple<int, const void*>, int> done;
@@ -487,14 +484,6 @@ int moe_test_set_wait_budget_ns(unsigned long long ns) {
   REQ(ns >= 1000 && ns <= moe::kWaitBudgetNs, MOE_ERR_INVALID_ARG,
       "moe_test_set_wait_budget_ns: budget must be 0 (default) or in [1000, 2e9] ns");
   g_main_wait_ns.store(ns, std::memory_order_relaxed);
-  return MOE_OK;
-}
-
-int moe_test_set_gemm_mode(int mode) {
-  g_err.clear();
-  REQ(mode >= 0 && mode <= 2, MOE_ERR_INVALID_ARG,
-      "moe_test_set_gemm_mode: mode must be 0 (automatic), 1 (1-CTA tiles) or 2 (CTA pairs)");
-  moe_host::g_gemm_mode.store(mode, std::memory_order_relaxed);
   return MOE_OK;
 }
 

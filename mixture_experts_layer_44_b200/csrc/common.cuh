@@ -190,9 +190,6 @@ void note_launch();
 // Budget of the main-loop waits of the tensor-core kernels (nanoseconds):
 // kWaitBudgetNs unless moe_test_set_wait_budget_ns shortened it.
 uint64_t main_wait_budget_ns();
-// Testing hook: 0 = the grouped GEMM chooses 1-CTA or CTA-pair tiles itself,
-// 1 = always 1-CTA tiles, 2 = CTA pairs wherever a tile can have > 32 rows.
-int gemm_mode();
 
 // Launch with programmatic stream serialization (and a cluster of cluster_x
 // CTAs along x when cluster_x > 0).

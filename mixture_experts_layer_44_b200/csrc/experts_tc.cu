@@ -68,8 +68,6 @@
 #include <cuda.h>
 
 #include <algorithm>
-#include <map>
-#include <mutex>
 
 #include "common.cuh"
 #include "sm100_ptx.cuh"
@@ -81,7 +79,7 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
 constexpr int B_BYTES = BN * BK * 2;
-constexpr int MAX_STAGES = 6;
+constexpr int MAX_STAGES = 5;
 constexpr int NTHREADS = 192;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr uint32_t IDESC = moe::idesc_bf16_f32(BM, BN);
@@ -100,7 +98,6 @@ struct Ctl {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  uint64_t pexit;      // CTA pairs: the other CTA of the pair has finished
   uint64_t ufull[UNIT_RING];    // producer -> MMA + epilogue: unit id published
   uint64_t uempty[UNIT_RING];   // MMA + 4 epilogue warps -> producer: slot read
   int uid[UNIT_RING];
@@ -128,20 +125,13 @@ constexpr size_t CTL_BYTES = (sizeof(Ctl) + 1023) / 1024 * 1024;
 // the same stage's B tile -- garbage in accumulator rows that are never
 // stored -- and the 12 KB saved per stage buy a fifth stage, 25 % more weight
 // bytes in flight per SM.
-//
-// PAIR: a CTA pair (cluster of 2) runs M = 256 tiles; each CTA holds its 128
-// rows of A and half of the weight tile (128 rows), 32 KB per stage, so the
-// ring has 6 stages: half the operand bytes per MMA of the 1-CTA tile, and
-// 1.5x the MMA time covered by the loads in flight.
-template <int AR, bool PAIR = false>
+template <int AR>
 struct Ring {
   static constexpr int A_B = AR * BK * 2;
-  static constexpr int B_B = PAIR ? B_BYTES / 2 : B_BYTES;   // this CTA's part of the weights
-  static constexpr int ST_B = A_B + B_B;
-  static constexpr int N = PAIR ? 6 : (AR == BM ? 4 : 5);
+  static constexpr int ST_B = A_B + B_BYTES;
+  static constexpr int N = AR == BM ? 4 : 5;
   static constexpr size_t SMEM = 1024 + N * ST_B + CTL_BYTES + STAGE_OUT_BYTES;
-  static_assert(!PAIR || AR == BM, "CTA pairs load whole 128-row A tiles");
-  static_assert(AR == BM || (AR >= 8 && AR % 8 == 0 && A_B + B_B >= BM * BK * 2),
+  static_assert(AR == BM || (AR >= 8 && AR % 8 == 0 && A_B + B_BYTES >= BM * BK * 2),
                 "a short A tile must be followed by at least 128 rows' worth of the stage");
   static_assert(N <= MAX_STAGES && SMEM <= 227 * 1024, "stage ring exceeds shared memory");
   static_assert(ST_B % 1024 == 0 && A_B % 1024 == 0, "tiles must stay 1024-byte aligned");
@@ -154,8 +144,7 @@ struct Unit {
   int tile, g, e, nt, mt, ks, S, kb0, kb1, row0, rend;
 };
 
-// TM: rows of a token tile (128; 256 for a CTA pair).
-template <bool SHARED, int TM = BM>
+template <bool SHARED>
 __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, int kblocks2,
                                             int u) {
   // Units: the shared tiles' slices first (splits2 each), then the routed
@@ -179,7 +168,7 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     r.e = 0;
     r.nt = r.tile / c.mte2;
     r.mt = r.tile - r.nt * c.mte2;
-    r.row0 = r.mt * TM;
+    r.row0 = r.mt * BM;
     r.rend = c.rows2;
     kb = kblocks2;
   } else {
@@ -191,11 +180,11 @@ __device__ __forceinline__ Unit decode_unit(const Ctl& c, int E, int kblocks, in
     }
     r.g = 0;
     r.e = lo;
-    const int mte = (c.offs[r.e + 1] - c.offs[r.e] + TM - 1) / TM;
+    const int mte = (c.offs[r.e + 1] - c.offs[r.e] + BM - 1) / BM;
     const int local = r.tile - c.tstart[r.e];
     r.nt = local / mte;
     r.mt = local - r.nt * mte;
-    r.row0 = c.offs[r.e] + r.mt * TM;
+    r.row0 = c.offs[r.e] + r.mt * BM;
     r.rend = c.offs[r.e + 1];
     kb = kblocks;
   }
@@ -345,7 +334,7 @@ __device__ __forceinline__ float store_h16x64(__half* dst, const uint32_t (&a)[4
 // element rounded once, after the fp32 accumulation and the routing-weight
 // scale -- instead of fp32.  A magnitude above the fp16 range is reported
 // (MOE_ERR_OVERFLOW); the element becomes inf.
-template <int EPI, bool SHARED, bool YH, int AR, bool PAIR>
+template <int EPI, bool SHARED, bool YH, int AR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
@@ -359,13 +348,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         void* __restrict__ out2, int ldo2, int* __restrict__ counters,
                         float* __restrict__ partials, int max_units, int32_t* status,
                         uint64_t wait_ns) {
-  using RG = Ring<AR, PAIR>;
+  using RG = Ring<AR>;
   constexpr int STAGES = RG::N;
   constexpr int A_BYTES = RG::A_B;
   constexpr int STAGE_BYTES = RG::ST_B;
-  constexpr int TM = PAIR ? 2 * BM : BM;                    // rows of a token tile
-  // The MMA of a pair covers 256 rows: both CTAs' A tiles and weight halves.
-  constexpr uint32_t MMA_IDESC = PAIR ? moe::idesc_bf16_f32(2 * BM, BN) : IDESC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -376,20 +362,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int kblocks = K / BK;
   const int kblocks2 = K2 / BK;
   rows2 = SHARED ? rows2 : 0;
-  // A CTA pair is one worker: rank 0 (the leader) issues the MMAs, both
-  // load and store their own 128 rows.  Workers take units statically.
-  const uint32_t rank = PAIR ? moe::cluster_ctarank() : 0u;
-  const int worker = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int nworkers = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  // cluster addresses of the leader's / the other CTA's variables
-  auto at_leader = [&](const void* p) {
-    return PAIR ? moe::mapa_shared(moe::smem_addr(p), 0u) : moe::smem_addr(p);
-  };
-  auto at_other = [&](const void* p) { return moe::mapa_shared(moe::smem_addr(p), rank ^ 1u); };
-  auto abort_now = [&]() {
-    set_abort(c, status);
-    if (PAIR) moe::st_cluster_u32(at_other(&c.abort), 1u);   // the pair stops together
-  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -398,18 +370,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       moe::mbar_init(moe::smem_addr(&c.tfull[b]), 1);
-      // a pair's accumulator is free once both CTAs' epilogue warps read it
-      moe::mbar_init(moe::smem_addr(&c.tempty[b]), PAIR ? 8 : 4);
+      moe::mbar_init(moe::smem_addr(&c.tempty[b]), 4);
     }
     moe::mbar_init(moe::smem_addr(&c.drain), 1);
-    moe::mbar_init(moe::smem_addr(&c.pexit), 1);
     for (int r = 0; r < UNIT_RING; ++r) {
       moe::mbar_init(moe::smem_addr(&c.ufull[r]), 1);
-      // A pair's ring is the leader's: its producer takes the units and writes
-      // them into both CTAs' slots; a slot is free again once the leader's MMA
-      // and epilogue warps and the other CTA's producer and epilogue warps
-      // have read it.
-      moe::mbar_init(moe::smem_addr(&c.uempty[r]), PAIR ? 10 : 5);
+      moe::mbar_init(moe::smem_addr(&c.uempty[r]), 5);
     }
     c.abort = 0;
     moe::fence_barrier_init();
@@ -421,17 +387,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   }
   if (warp == 1) {
-    if (PAIR) {
-      moe::tmem_alloc_pair(moe::smem_addr(&c.tmem_base), TMEM_COLS);
-      moe::tmem_relinquish_pair();
-    } else {
-      moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
-      moe::tmem_relinquish();
-    }
+    moe::tmem_alloc(moe::smem_addr(&c.tmem_base), TMEM_COLS);
+    moe::tmem_relinquish();
   }
-  // Both CTAs of a pair have initialised their barriers before either
-  // signals the other's.
-  if (PAIR) moe::cluster_sync_all();
   // Pass 1 reads offsets and x_packed, both written by the kernels just before
   // it, so it waits for them first.  Pass 2's inputs other than h are older:
   // its offsets were final before pass 1 could start (pass 1 waited for them,
@@ -456,14 +414,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int o0 = __ldcg(offsets + e), o1 = __ldcg(offsets + e + 1);
         c.offs[e] = o0;
         const int rows = o1 - o0;
-        m = (rows + TM - 1) / TM;
+        m = (rows + BM - 1) / BM;
         rmax = max(rmax, min(rows, BM));
       }
       cnt[j] = m;
       local += m;
     }
     rmax = static_cast<int>(__reduce_max_sync(0xffffffffu, static_cast<unsigned>(rmax)));
-    const int mte2 = (rows2 + TM - 1) / TM;      // the shared group's tiles come first
+    const int mte2 = (rows2 + BM - 1) / BM;      // the shared group's tiles come first
     const int n2 = mte2 * ntw2;
     int incl = local;
 #pragma unroll
@@ -493,7 +451,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int units_cap = static_cast<int>(
           min(static_cast<long long>(max_units) * BM / slot_rows, 1ll << 30));
       int sp = 1, sp2 = 1;
-      if (!PAIR && counters != nullptr && partials != nullptr && tiles <= SCHED_TICKET) {
+      if (counters != nullptr && partials != nullptr && tiles <= SCHED_TICKET) {
         if (rt == 0) {
           sp2 = choose_splits(n2, gridDim.x, kblocks2, units_cap, min(rows2, BM));
         } else {
@@ -522,26 +480,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = c.tmem_base;
 
   // The B operand (weights) of k-block kb of unit un into stage buffer sa,
-  // completing on barrier fb.  A pair splits the weight tile: in pass 1 the
-  // leader loads the 128 gate rows and the other CTA the 128 up rows (the w13
-  // map's box is one expert half deep), in pass 2 rows [0,128) and [128,256)
-  // of the tile; fb is then the leader's barrier (a cluster address).
+  // completing on barrier fb.
   auto load_b = [&](const Unit& un, int kb, uint32_t sa, uint32_t fb) {
-    if (PAIR) {
-      const int h = static_cast<int>(rank);
-      if (SHARED && un.g) {
-        if (EPI == EPI_SWIGLU)
-          moe::tma_load_3d_pair(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), h);
-        else
-          moe::tma_load_2d_pair(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * BN + h * (BN / 2));
-      } else if (EPI == EPI_SWIGLU) {
-        moe::tma_load_3d_pair(sa + A_BYTES, &tmB, fb, kb * BK, un.nt * (BN / 2), 2 * un.e + h);
-      } else {
-        moe::tma_load_2d_pair(sa + A_BYTES, &tmB, fb, kb * BK,
-                              un.e * rows_per_expert + un.nt * BN + h * (BN / 2));
-      }
-      return;
-    }
     if (SHARED && un.g) {
       if (EPI == EPI_SWIGLU)
         moe::tma_load_3d(sa + A_BYTES, &tmB2, fb, kb * BK, un.nt * (BN / 2), 0);
@@ -554,26 +494,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   };
 
-  // The A operand: this CTA's rows of the token tile.
-  auto load_a = [&](const CUtensorMap* ma, int kb, int arow, uint32_t sa, uint32_t fb) {
-    if (PAIR)
-      moe::tma_load_2d_pair(sa, ma, fb, kb * BK, arow + static_cast<int>(rank) * BM);
-    else
-      moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
-  };
-
   // The same k-block of the B operand, requested into L2 only.
   auto prefetch_b = [&](const Unit& un, int kb) {
     if (SHARED && un.g) {
       if (EPI == EPI_SWIGLU)
-        moe::tma_prefetch_3d(&tmB2, kb * BK, un.nt * (BN / 2), PAIR ? rank : 0);
+        moe::tma_prefetch_3d(&tmB2, kb * BK, un.nt * (BN / 2), 0);
       else
-        moe::tma_prefetch_2d(&tmB2, kb * BK, un.nt * BN + (PAIR ? rank * (BN / 2) : 0));
+        moe::tma_prefetch_2d(&tmB2, kb * BK, un.nt * BN);
     } else if (EPI == EPI_SWIGLU) {
-      moe::tma_prefetch_3d(&tmB, kb * BK, un.nt * (BN / 2), 2 * un.e + (PAIR ? rank : 0));
+      moe::tma_prefetch_3d(&tmB, kb * BK, un.nt * (BN / 2), 2 * un.e);
     } else {
-      moe::tma_prefetch_2d(&tmB, kb * BK,
-                           un.e * rows_per_expert + un.nt * BN + (PAIR ? rank * (BN / 2) : 0));
+      moe::tma_prefetch_2d(&tmB, kb * BK, un.e * rows_per_expert + un.nt * BN);
     }
   };
 
@@ -583,14 +514,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // follows after the wait.
   int pre = 0;                                   // stages whose B half is on its way
   int pre_issued[STAGES] = {};
-  if (EARLY && warp == 0 && lane == 0 && worker < total) {
-    const Unit un = decode_unit<SHARED, TM>(c, E, kblocks, kblocks2, worker);
+  if (EARLY && warp == 0 && lane == 0 && static_cast<int>(blockIdx.x) < total) {
+    const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, blockIdx.x);
     pre = min(STAGES, un.kb1 - un.kb0);
     for (int s = 0; s < pre; ++s) {
-      // a pair's stage holds both CTAs' bytes, counted on the leader's barrier
-      if (rank == 0) moe::mbar_arrive_expect_tx(moe::smem_addr(&c.full[s]),
-                                                PAIR ? 2 * STAGE_BYTES : STAGE_BYTES);
-      load_b(un, un.kb0 + s, moe::smem_addr(smem + s * STAGE_BYTES), at_leader(&c.full[s]));
+      const uint32_t fb = moe::smem_addr(&c.full[s]);
+      moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+      load_b(un, un.kb0 + s, moe::smem_addr(smem + s * STAGE_BYTES), fb);
       pre_issued[s] = 1;
     }
     const int l2_end = min(un.kb1, un.kb0 + pre + 8);
@@ -607,64 +537,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int s = 0; s < STAGES; ++s) issued[s] = pre_issued[s];
       int uslot = 0;
       uint32_t uphase = 0;
-      int next_static = worker;
+      int next_static = blockIdx.x;
       int npre = pre;                              // the first unit's prefetched k-blocks
       for (;;) {
-        int u;
-        if (PAIR && rank != 0) {
-          // the leader took the unit and wrote its id into this CTA's slot
-          if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns, true)) {
-            abort_now();
-            break;
-          }
-          u = c.uid[uslot];
-          moe::mbar_arrive_cluster(at_leader(&c.uempty[uslot]));
-        } else {
-          // Take the next unit and publish its id (-1: no more work) to the consumers.
-          if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1, wait_ns, PAIR)) {
-            abort_now();
-            break;
-          }
-          if (next_static == worker || counters == nullptr) {
-            u = next_static;                    // the first unit of every worker is static
-            next_static += nworkers;
-          } else {
-            u = nworkers + atomicAdd(&counters[SCHED_TICKET], 1);
-          }
-          if (u >= total || aborted(c)) u = -1;
-          c.uid[uslot] = u;
-          if (PAIR) {
-            moe::st_cluster_u32(at_other(&c.uid[uslot]), static_cast<uint32_t>(u));
-            moe::mbar_arrive_cluster(at_other(&c.ufull[uslot]));
-          }
-          moe::mbar_arrive(moe::smem_addr(&c.ufull[uslot]));
+        // Take the next unit and publish its id (-1: no more work) to the consumers.
+        if (!moe::mbar_wait(moe::smem_addr(&c.uempty[uslot]), uphase ^ 1, wait_ns)) {
+          set_abort(c, status);
+          break;
         }
+        int u;
+        if (next_static == static_cast<int>(blockIdx.x) || counters == nullptr) {
+          u = next_static;                    // the first unit of every CTA is static
+          next_static += gridDim.x;
+        } else {
+          u = gridDim.x + atomicAdd(&counters[SCHED_TICKET], 1);
+        }
+        if (u >= total || aborted(c)) u = -1;
+        c.uid[uslot] = u;
+        moe::mbar_arrive(moe::smem_addr(&c.ufull[uslot]));
         if (++uslot == UNIT_RING) {
           uslot = 0;
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit<SHARED, TM>(c, E, kblocks, kblocks2, u);
+        const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int arow = un.row0;
         const bool g1 = SHARED && un.g;
         const CUtensorMap* ma = g1 ? &tmA2 : &tmA;
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
-          const uint32_t fb = at_leader(&c.full[stage]);
+          const uint32_t fb = moe::smem_addr(&c.full[stage]);
           const uint32_t sa = moe::smem_addr(smem + stage * STAGE_BYTES);
           if (kb - un.kb0 < npre) {
             // B already requested before the wait (fresh stage, nothing to wait for)
-            load_a(ma, kb, arow, sa, fb);
+            moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
           } else {
             if (!moe::mbar_wait(moe::smem_addr(&c.empty[stage]), phase ^ 1, wait_ns)) {
-              abort_now();
+              set_abort(c, status);
               ok = false;
               break;
             }
-            if (rank == 0)
-              moe::mbar_arrive_expect_tx(moe::smem_addr(&c.full[stage]),
-                                         PAIR ? 2 * STAGE_BYTES : STAGE_BYTES);
-            load_a(ma, kb, arow, sa, fb);
+            moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
             load_b(un, kb, sa, fb);
             ++issued[stage];
           }
@@ -676,19 +590,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         npre = 0;
         if (!ok) break;
       }
-      // Drain: every load issued has landed before the CTA can leave.  A
-      // pair's loads complete on the leader's barriers, which count both
-      // CTAs' bytes; the other CTA leaves only after the leader (pexit).
-      if (rank == 0)
-        for (int s = 0; s < STAGES; ++s)
-          if (issued[s] > 0) moe::mbar_wait(moe::smem_addr(&c.full[s]), (issued[s] - 1) & 1);
+      // Drain: every load issued has landed before the CTA can leave.
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] > 0) moe::mbar_wait(moe::smem_addr(&c.full[s]), (issued[s] - 1) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0 && PAIR && rank != 0) {
-      // The other CTA of a pair issues no MMAs: the leader's final commit
-      // tells it that none still reads its shared memory or writes its TMEM.
-      moe::mbar_wait(moe::smem_addr(&c.drain), 0, moe::kWaitBudgetNs, true);
-    } else if (lane == 0) {
+    if (lane == 0) {
       // ----------------------------------------------------------- MMA ---
       int stage = 0;
       uint32_t phase = 0;
@@ -697,7 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t uphase = 0;
       for (;; ++i) {
         if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns)) {
-          abort_now();
+          set_abort(c, status);
           break;
         }
         const int u = c.uid[uslot];
@@ -707,10 +614,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           uphase ^= 1;
         }
         if (u < 0) break;
-        const Unit un = decode_unit<SHARED, TM>(c, E, kblocks, kblocks2, u);
+        const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int buf = i & 1;
-        if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1, wait_ns, PAIR)) {
-          abort_now();
+        if (!moe::mbar_wait(moe::smem_addr(&c.tempty[buf]), ((i >> 1) & 1) ^ 1, wait_ns)) {
+          set_abort(c, status);
           break;
         }
         moe::tc_fence_after();
@@ -718,7 +625,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
           if (!moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase, wait_ns)) {
-            abort_now();
+            set_abort(c, status);
             ok = false;
             break;
           }
@@ -728,82 +635,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = moe::sw128_kmajor_desc(sa + kk * 32);
             const uint64_t bd = moe::sw128_kmajor_desc(sa + A_BYTES + kk * 32);
-            const uint32_t acc = (kb > un.kb0 || kk > 0) ? 1u : 0u;
-            if (PAIR)
-              moe::tc_mma_f16_pair(d, ad, bd, MMA_IDESC, acc);
-            else
-              moe::tc_mma_f16(d, ad, bd, MMA_IDESC, acc);
+            moe::tc_mma_f16(d, ad, bd, IDESC, (kb > un.kb0 || kk > 0) ? 1u : 0u);
           }
-          if (PAIR) {
-            // both CTAs' stage buffers are free once these MMAs complete
-            moe::tc_commit_pair(moe::smem_addr(&c.empty[stage]));
-            moe::tc_commit_pair(at_other(&c.empty[stage]));
-          } else {
-            moe::tc_commit(moe::smem_addr(&c.empty[stage]));
-          }
+          moe::tc_commit(moe::smem_addr(&c.empty[stage]));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        if (PAIR) {
-          moe::tc_commit_pair(moe::smem_addr(&c.tfull[buf]));
-          moe::tc_commit_pair(at_other(&c.tfull[buf]));
-        } else {
-          moe::tc_commit(moe::smem_addr(&c.tfull[buf]));
-        }
+        moe::tc_commit(moe::smem_addr(&c.tfull[buf]));
       }
-      // Drain: all MMAs this thread issued have completed (for a pair, the
-      // other CTA learns it from the same commit).
-      if (PAIR) {
-        moe::tc_commit_pair(moe::smem_addr(&c.drain));
-        moe::tc_commit_pair(at_other(&c.drain));
-      } else {
-        moe::tc_commit(moe::smem_addr(&c.drain));
-      }
+      // Drain: all MMAs this thread issued have completed.
+      moe::tc_commit(moe::smem_addr(&c.drain));
       moe::mbar_wait(moe::smem_addr(&c.drain), 0);
     }
   } else {
     // ------------------------------------------------------- epilogue ---
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;          // row of the tile owned by this thread
-    // this warp has read accumulator buffer b (a pair's: the leader's barrier)
-    auto release_tmem = [&](int b) {
-      if (PAIR)
-        moe::mbar_arrive_cluster(at_leader(&c.tempty[b]));
-      else
-        moe::mbar_arrive(moe::smem_addr(&c.tempty[b]));
-    };
     int i = 0;
     int uslot = 0;
     uint32_t uphase = 0;
     for (;; ++i) {
-      if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns, PAIR)) {
-        abort_now();
+      if (!moe::mbar_wait(moe::smem_addr(&c.ufull[uslot]), uphase, wait_ns)) {
+        set_abort(c, status);
         break;
       }
       const int u = c.uid[uslot];
       __syncwarp();
-      if (lane == 0) {
-        if (PAIR)
-          moe::mbar_arrive_cluster(at_leader(&c.uempty[uslot]));
-        else
-          moe::mbar_arrive(moe::smem_addr(&c.uempty[uslot]));
-      }
+      if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.uempty[uslot]));
       if (++uslot == UNIT_RING) {
         uslot = 0;
         uphase ^= 1;
       }
       if (u < 0) break;
       const int buf = i & 1;
-      if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1, wait_ns, PAIR)) {
-        abort_now();
+      if (!moe::mbar_wait(moe::smem_addr(&c.tfull[buf]), (i >> 1) & 1, wait_ns)) {
+        set_abort(c, status);
         break;
       }
       moe::tc_fence_after();
-      Unit un = decode_unit<SHARED, TM>(c, E, kblocks, kblocks2, u);
-      if (PAIR) un.row0 += static_cast<int>(rank) * BM;   // this CTA's half of the pair tile
+      const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
       const int rows_valid = un.rend - un.row0;
       const bool live = row < rows_valid;
       const size_t grow = static_cast<size_t>(un.row0 + row);
@@ -940,7 +813,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         moe::tc_fence_before();
         __syncwarp();
-        if (lane == 0) release_tmem(buf);
+        if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));
       } else {
         // Partial of one K-slice: valid rows to this unit's workspace slot.
         // (In the w2 pass a TMA store of an earlier unit may still be reading
@@ -969,7 +842,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         moe::tc_fence_before();
         __syncwarp();
-        if (lane == 0) release_tmem(buf);   // TMEM free
+        if (lane == 0) moe::mbar_arrive(moe::smem_addr(&c.tempty[buf]));   // TMEM free
         __threadfence();
         epi_bar();
         if (warp == 2 && lane == 0) {
@@ -1051,30 +924,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   moe::tc_fence_before();
   __syncthreads();
   moe::tc_fence_after();
-  if (PAIR) {
-    // Neither CTA of a pair leaves (or frees the pair's TMEM) before the
-    // other is done: the leader's MMAs read the other CTA's shared memory and
-    // write its TMEM, and the other CTA's copies and epilogue signal the
-    // leader's barriers.  After an abort the other CTA first gives the copies
-    // it may still have in flight time to land (it cannot observe them: they
-    // complete on the leader's barriers).
-    if (threadIdx.x == 0) {
-      if (rank != 0 && aborted(c)) {
-        const uint64_t t0 = moe::globaltimer_ns();
-        while (moe::globaltimer_ns() - t0 < 200000ull) {
-        }
-      }
-      moe::mbar_arrive_cluster(at_other(&c.pexit));
-      if (!moe::mbar_wait(moe::smem_addr(&c.pexit), 0, moe::kWaitBudgetNs, true))
-        moe::report(status, MOE_ERR_TIMEOUT);
-    }
-    moe::tc_fence_before();
-    __syncthreads();
-    moe::tc_fence_after();
-    if (warp == 1) moe::tmem_dealloc_pair(tmem, TMEM_COLS);
-  } else if (warp == 1) {
-    moe::tmem_dealloc(tmem, TMEM_COLS);
-  }
+  if (warp == 1) moe::tmem_dealloc(tmem, TMEM_COLS);
   if (threadIdx.x == 0 && counters != nullptr) {
     // The last CTA to leave returns the ticket (and the exit count) to zero.
     __threadfence();
@@ -1121,50 +971,17 @@ size_t experts_ws_bytes() {
 namespace {
 
 // Every instance of the kernel has this signature.
-using GemmFn = decltype(&grouped_gemm_kernel<EPI_SWIGLU, false, false, BM, false>);
+using GemmFn = decltype(&grouped_gemm_kernel<EPI_SWIGLU, false, false, BM>);
 
-// The kernels of both passes for one A-tile height (AR rows) and mode.
-template <int AR, bool PAIR>
+// The kernels of both passes for one A-tile height (AR rows).
+template <int AR>
 void pick_kernels(bool shared, bool y_f16, GemmFn* k1, GemmFn* k2) {
-  *k1 = shared ? grouped_gemm_kernel<EPI_SWIGLU, true, false, AR, PAIR>
-               : grouped_gemm_kernel<EPI_SWIGLU, false, false, AR, PAIR>;
-  *k2 = y_f16 ? (shared ? grouped_gemm_kernel<EPI_SCALE, true, true, AR, PAIR>
-                        : grouped_gemm_kernel<EPI_SCALE, false, true, AR, PAIR>)
-              : (shared ? grouped_gemm_kernel<EPI_SCALE, true, false, AR, PAIR>
-                        : grouped_gemm_kernel<EPI_SCALE, false, false, AR, PAIR>);
-}
-
-// CTA pairs that can be resident at once (one pair per two SMs at most);
-// the persistent grid is twice that, so no pair waits for another to leave.
-int resident_pairs(GemmFn k, size_t smem) {
-  static std::mutex mu;
-  static std::map<std::pair<int, const void*>, int> cache;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(mu);
-  auto key = std::make_pair(dev, reinterpret_cast<const void*>(k));
-  auto it = cache.find(key);
-  if (it != cache.end()) return it->second;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * (num_sms() / 2));
-  cfg.blockDim = dim3(NTHREADS);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 2;
-  attr.val.clusterDim.y = 1;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(k), &cfg) != cudaSuccess ||
-      n <= 0) {
-    cudaGetLastError();
-    n = num_sms() / 2;
-  }
-  n = std::max(1, std::min(n, num_sms() / 2));
-  cache[key] = n;
-  return n;
+  *k1 = shared ? grouped_gemm_kernel<EPI_SWIGLU, true, false, AR>
+               : grouped_gemm_kernel<EPI_SWIGLU, false, false, AR>;
+  *k2 = y_f16 ? (shared ? grouped_gemm_kernel<EPI_SCALE, true, true, AR>
+                        : grouped_gemm_kernel<EPI_SCALE, false, true, AR>)
+              : (shared ? grouped_gemm_kernel<EPI_SCALE, true, false, AR>
+                        : grouped_gemm_kernel<EPI_SCALE, false, false, AR>);
 }
 
 }  // namespace
@@ -1179,28 +996,17 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   const int T2 = sh ? sh->T : 0, Is = sh ? sh->I : 0;
   const bool short_a = N <= 32 && T2 <= 32;
   const int ar = short_a ? 32 : BM;
-  // CTA pairs (256-row tiles) when the experts average at least 256 rows:
-  // the operand feed, not the weight stream, bounds such batches.
-  const int mode = gemm_mode();
-  const bool pairs = !short_a && (mode == 2 || (mode == 0 && N >= 8192 && N >= 256 * E));
   // The shared-expert group is compiled in only where it is used.
   GemmFn k1, k2;
   if (short_a)
-    pick_kernels<32, false>(sh != nullptr, y_f16, &k1, &k2);
-  else if (pairs)
-    pick_kernels<BM, true>(sh != nullptr, y_f16, &k1, &k2);
+    pick_kernels<32>(sh != nullptr, y_f16, &k1, &k2);
   else
-    pick_kernels<BM, false>(sh != nullptr, y_f16, &k1, &k2);
-  const size_t smem =
-      short_a ? Ring<32>::SMEM : (pairs ? Ring<BM, true>::SMEM : Ring<BM>::SMEM);
+    pick_kernels<BM>(sh != nullptr, y_f16, &k1, &k2);
+  const size_t smem = short_a ? Ring<32>::SMEM : Ring<BM>::SMEM;
   cudaError_t e1 = ensure_smem(reinterpret_cast<const void*>(k1), static_cast<int>(smem));
   if (e1 != cudaSuccess) return e1;
   e1 = ensure_smem(reinterpret_cast<const void*>(k2), static_cast<int>(smem));
   if (e1 != cudaSuccess) return e1;
-  // A pair's CTA loads half of each weight tile: 128 gate or up rows (pass 1),
-  // 128 of the 256 rows (pass 2).
-  const cuuint32_t b_rows = pairs ? BN / 2 : BN;
-  const cuuint32_t b_halves = pairs ? 1 : 2;
   const int nmap = N > 0 ? N : 1;           // a map needs one row; no tile reads it when N == 0
   CUtensorMap mA1, mB1, mA2, mB2;
   bool ok = map_rows(&mA1, x_packed, nmap, H, ar) && map_rows(&mA2, h, nmap, I, ar);
@@ -1210,14 +1016,14 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
                                 static_cast<cuuint64_t>(2) * E};
     const cuuint64_t str[2] = {static_cast<cuuint64_t>(H) * 2,
                                static_cast<cuuint64_t>(I) * H * 2};
-    const cuuint32_t box[3] = {BK, BN / 2, b_halves};
+    const cuuint32_t box[3] = {BK, BN / 2, 2};
     ok = ok && encode_bf16_sw128(&mB1, w13, 3, dims, str, box);
   }
   {
     // w2 as [E*H][I]
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(E) * H};
     const cuuint64_t str[1] = {static_cast<cuuint64_t>(I) * 2};
-    const cuuint32_t box[2] = {BK, b_rows};
+    const cuuint32_t box[2] = {BK, BN};
     ok = ok && encode_bf16_sw128(&mB2, w2, 2, dims, str, box);
   }
   // The shared expert's maps (x [T][H], w13s as [2][Is][H], h_s [T][Is], w2s [H][Is]);
@@ -1228,11 +1034,11 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
     const cuuint64_t d1[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(Is), 2};
     const cuuint64_t s1[2] = {static_cast<cuuint64_t>(H) * 2,
                               static_cast<cuuint64_t>(Is) * H * 2};
-    const cuuint32_t b1[3] = {BK, BN / 2, b_halves};
+    const cuuint32_t b1[3] = {BK, BN / 2, 2};
     ok = ok && encode_bf16_sw128(&sB1, sh->w13, 3, d1, s1, b1);
     const cuuint64_t d2[2] = {static_cast<cuuint64_t>(Is), static_cast<cuuint64_t>(H)};
     const cuuint64_t s2[1] = {static_cast<cuuint64_t>(Is) * 2};
-    const cuuint32_t b2[2] = {BK, b_rows};
+    const cuuint32_t b2[2] = {BK, BN};
     ok = ok && encode_bf16_sw128(&sB2, sh->w2, 2, d2, s2, b2);
   }
   // the w2 pass's outputs (the shared expert's own, or the routed map standing in)
@@ -1260,29 +1066,20 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   const int ntw1 = (I + BN / 2 - 1) / (BN / 2);
   const int ntw1s = (Is + BN / 2 - 1) / (BN / 2);
   int g1 = sms, g2 = sms;
-  const int tm = pairs ? 2 * BM : BM;
-  const int workers = pairs ? 2 : 1;          // CTAs per worker
-  if (pairs) {
-    g1 = 2 * resident_pairs(k1, smem);
-    g2 = 2 * resident_pairs(k2, smem);
-  }
-  if (counters == nullptr) {   // no split possible: never more workers than tiles
-    const int mt_bound = (N + tm - 1) / tm + E;
-    const int mt2 = (T2 + tm - 1) / tm;
-    g1 = workers * std::max(1, std::min(g1 / workers, mt_bound * ntw1 + mt2 * ntw1s));
-    g2 = workers * std::max(1, std::min(g2 / workers, (mt_bound + mt2) * (H / BN)));
+  if (counters == nullptr) {   // no split possible: never more CTAs than tiles
+    const int mt_bound = (N + BM - 1) / BM + E;
+    const int mt2 = (T2 + BM - 1) / BM;
+    g1 = std::max(1, std::min(sms, mt_bound * ntw1 + mt2 * ntw1s));
+    g2 = std::max(1, std::min(sms, (mt_bound + mt2) * (H / BN)));
   }
   const float* no_w = nullptr;
-  // Pairs keep the full wait budget: the testing hook that shortens it drives
-  // the abort path of the 1-CTA kernels.
-  const uint64_t wait_ns = pairs ? moe::kWaitBudgetNs : main_wait_budget_ns();
-  const int cluster = pairs ? 2 : 0;
-  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS), smem, s, cluster, mA1, mB1, sA1,
-                               sB1, mY, sY, offsets, E, H, ntw1, 2 * I, no_w, h, I, T2, H, ntw1s,
+  const uint64_t wait_ns = main_wait_budget_ns();
+  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS), smem, s, 0, mA1, mB1, sA1, sB1,
+                               mY, sY, offsets, E, H, ntw1, 2 * I, no_w, h, I, T2, H, ntw1s,
                                sh ? sh->h : nullptr, Is, counters, partials, max_units, status,
                                wait_ns);
   if (err != cudaSuccess) return err;
-  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), smem, s, cluster, mA2, mB2, sA2, sB2, mY, sY,
+  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), smem, s, 0, mA2, mB2, sA2, sB2, mY, sY,
                     offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
                     sh ? sh->y : nullptr, H, counters, partials, max_units, status, wait_ns);
 }

@@ -237,85 +237,3 @@ def test_experts_fp16_y_overflow_is_reported_not_faulted():
             assert err_stored(yc[ok], ys[ok.numpy()]) <= 1e-3
         else:
             assert rel(yc, ys) <= 1e-3
-
-
-# ------------------------------------------------ CTA pairs (M = 256) ---
-
-@pytest.fixture
-def pair_tiles():
-    """Force CTA-pair tiles (tcgen05 cta_group::2) for the test's calls."""
-    M.moe_test_set_gemm_mode(2)
-    try:
-        yield
-    finally:
-        M.moe_test_set_gemm_mode(0)
-
-
-@pytest.mark.parametrize("counts,H,I", [
-    ([0, 1, 127, 300], 256, 128),            # tiles of 1, 127 and 300 rows: one or both CTAs idle
-    ([200], 512, 256),                       # the other CTA of the pair has no rows
-    ([256, 512, 0, 257], 768, 384),          # exact pair tiles, then one row over
-    ([900, 0, 37, 260, 1, 0, 0, 130], 2048, 768),   # the Qwen3 expert shape, skewed
-    ([130, 70], 256, 192),                   # I % 128 == 64: a half feature tile in pass 1
-])
-@pytest.mark.parametrize("y_dtype", [torch.float16, torch.float32])
-def test_experts_pairs(pair_tiles, counts, H, I, y_dtype):
-    _check(*_make(counts, H, I, torch.bfloat16, seed=3 * sum(counts) + H), tol=TOL["bf16"],
-           y_dtype=y_dtype)
-
-
-def test_experts_pairs_many_tiles_and_repeatable(pair_tiles):
-    rng = np.random.default_rng(4)
-    counts = list(rng.multinomial(20000, rng.dirichlet(np.ones(8))))
-    args = _make(counts, 512, 512, torch.bfloat16, seed=9)
-    h1, y1 = _check(*args, tol=TOL["bf16"])
-    h2, y2 = _run(*args)
-    assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
-    assert torch.equal(_bits(y1), _bits(y2))
-
-
-def test_experts_pairs_agree_with_single_cta_tiles():
-    args = _make([700, 0, 300, 1100, 45], 1024, 512, torch.bfloat16, seed=10)
-    hn = int(args[1][-1])
-    M.moe_test_set_gemm_mode(1)
-    try:
-        h1, y1 = _run(*args, y_dtype=torch.float32)
-    finally:
-        M.moe_test_set_gemm_mode(0)
-    M.moe_test_set_gemm_mode(2)
-    try:
-        h2, y2 = _run(*args, y_dtype=torch.float32)
-    finally:
-        M.moe_test_set_gemm_mode(0)
-    # the same products in the same K order: at most a summation-order difference
-    assert err_bf16_out(h2[:hn], O.to_f64(h1[:hn])) <= 1e-2
-    assert rel(y2[:hn], O.to_f64(y1[:hn])) <= 1e-4
-
-
-@pytest.mark.parametrize("counts,H,I,T,Is", [
-    ([300, 0, 129, 40], 256, 128, 200, 384),          # prefill-like
-    ([600, 300], 512, 256, 520, 256),                 # shared rows span three pair tiles
-])
-def test_experts_shared_pairs(pair_tiles, counts, H, I, T, Is):
-    x_packed, offs, pw, w13, w2 = _make(counts, H, I, torch.bfloat16, seed=T + Is + 1)
-    g = torch.Generator().manual_seed(T + 1)
-    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
-    w13s = (torch.randn(2 * Is, H, generator=g) / H ** 0.5).to(torch.bfloat16)
-    w2s = (torch.randn(H, Is, generator=g) / Is ** 0.5).to(torch.bfloat16)
-    N = x_packed.shape[0]
-    h = torch.full((N, I), 1536.0, dtype=torch.bfloat16, device=DEV)
-    y = torch.full((N, H), 1536.0, dtype=torch.float16, device=DEV)
-    hs = torch.full((T, Is), 1536.0, dtype=torch.bfloat16, device=DEV)
-    ys = torch.full((T, H), 1536.0, dtype=torch.float16, device=DEV)
-    status = torch.zeros(1, dtype=torch.int32, device=DEV)
-    M.moe_experts_shared(dev(x_packed), dev(offs), dev(pw), dev(w13), dev(w2), h, y, dev(x),
-                         dev(w13s), dev(w2s), hs, ys, ws=_ws(x_packed, w13), status=status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
-    ho, yo = O.experts(x_packed, offs.numpy(), pw, w13, w2)
-    assert err_bf16_out(h.cpu(), ho) <= TOL["bf16"] and _staged(y.cpu(), yo) <= TOL["bf16"]
-    assert _staged(y.cpu(), O.experts_down(h.cpu(), offs.numpy(), pw, w2)) <= 1e-3
-    one = np.array([0, T])
-    hso, yso = O.experts(x, one, None, w13s.unsqueeze(0), w2s.unsqueeze(0))
-    assert err_bf16_out(hs.cpu(), hso) <= TOL["bf16"] and _staged(ys.cpu(), yso) <= TOL["bf16"]
-    assert _staged(ys.cpu(), O.experts_down(hs.cpu(), one, None, w2s.unsqueeze(0))) <= 1e-3
