@@ -237,3 +237,14 @@ def test_experts_fp16_y_overflow_is_reported_not_faulted():
             assert err_stored(yc[ok], ys[ok.numpy()]) <= 1e-3
         else:
             assert rel(yc, ys) <= 1e-3
+
+
+# Experts with several token tiles beside single-tile and empty ones, K not
+# split: without a workspace (static units) and with one when there are enough
+# tiles (dynamic units).
+@pytest.mark.parametrize("counts,H,I,ws", [
+    ([300, 5, 0, 700, 60, 1, 200, 40], 512, 512, None),
+    ([2000, 5, 3000, 1, 90, 0, 700, 33], 512, 1024, "zeros"),
+])
+def test_experts_mixed_sizes_unsplit(counts, H, I, ws):
+    _check(*_make(counts, H, I, torch.bfloat16, seed=sum(counts) + I), tol=TOL["bf16"], ws=ws)
