@@ -497,7 +497,8 @@ def workload_summary(cfg, counts, ms, per_stage, launches, steps, peaks):
     return {"ms_per_step": ms, "tokens_per_s": cfg.T / (ms / 1e3), "T": cfg.T,
             "stage_ms": stage_dict(per_stage, route_dispatch_fits(cfg)),
             "layer_roofline": layer_roofline(cfg, counts, ms, peaks),
-            "gemm_roofline": gemm_roofline(cfg, counts, per_stage[2], peaks),
+            "gemm_roofline": dict(gemm_roofline(cfg, counts, per_stage[2], peaks),
+                                  traffic=ncu_traffic(cfg.name)),
             "active_experts": sum(1 for c in counts if c > 0), "max_expert_rows": max(counts),
             "zipf_slope_realised": zipf_slope(counts) if cfg.zipf_s is not None else None,
             "gpu_launches_per_step": launches / steps}
