@@ -515,8 +515,9 @@ int moe_layer_join(moe_layer* L, void* stream);
 int moe_layer_status(moe_layer* L, void* stream, int32_t* host_status);
 
 /* Device address of one of L's intermediate buffers, for inspection:
- * "logits", "ids", "w", "counts", "offsets", "inv_perm", "status"; NULL for
- * any other name. */
+ * "logits", "ids", "w", "counts", "offsets", "perm", "inv_perm",
+ * "packed_tok", "packed_w", "x_packed", "h", "y_packed" (fp16, or fp32 with
+ * y_f32), "status"; NULL for any other name. */
 void* moe_layer_buffer(moe_layer* L, const char* name);
 
 /* Copy the device status word to *host_status after the stream's prior work

@@ -346,6 +346,12 @@ void* moe_layer_buffer(moe_layer* L, const char* name) {
   if (!strcmp(name, "counts")) return L->counts;
   if (!strcmp(name, "offsets")) return L->offsets;
   if (!strcmp(name, "inv_perm")) return L->inv_perm;
+  if (!strcmp(name, "perm")) return L->perm;
+  if (!strcmp(name, "packed_tok")) return L->packed_tok;
+  if (!strcmp(name, "packed_w")) return L->packed_w;
+  if (!strcmp(name, "x_packed")) return L->x_packed;
+  if (!strcmp(name, "h")) return L->h;
+  if (!strcmp(name, "y_packed")) return L->y_packed;
   if (!strcmp(name, "status")) return L->status;
   return nullptr;
 }

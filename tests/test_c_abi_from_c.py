@@ -1,6 +1,7 @@
 """The boundary from plain C: include/moe_b200.h compiles as C99 with
 -Wall -Werror, and a C program linked against libmoe_b200.so gets the ABI
 version, the launch count and the host-side argument checks (no GPU call)."""
+import ctypes
 import os
 import subprocess
 import textwrap
@@ -83,3 +84,26 @@ def test_header_is_c99_and_the_library_links_from_c(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip().endswith("OK"), r.stdout + r.stderr
+
+
+def test_layer_descriptor_layout_matches_the_binding(tmp_path):
+    # the ctypes mirror of moe_layer_desc must have the C struct's size and offsets
+    fields = [f for f, _ in M.MoELayerDesc._fields_]
+    body = "\n".join(f'  printf("{f} %zu\\n", offsetof(moe_layer_desc, {f}));' for f in fields)
+    src = tmp_path / "desc_layout.c"
+    src.write_text(textwrap.dedent("""\
+        #include <stddef.h>
+        #include <stdio.h>
+        #include "moe_b200.h"
+        int main(void) {
+          printf("sizeof %zu\\n", sizeof(moe_layer_desc));
+        """) + body + "\n  return 0;\n}\n")
+    exe = tmp_path / "desc_layout"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                 timeout=60).stdout.splitlines())
+    assert int(out["sizeof"]) == ctypes.sizeof(M.MoELayerDesc)
+    for f in fields:
+        assert int(out[f]) == getattr(M.MoELayerDesc, f).offset, f

@@ -76,3 +76,25 @@ def test_layer_handle_against_the_oracle_on_host_buffers():
     want = O.moe_forward_tokens(p, np.arange(cfg.T), ids, O.routing_weights(l64, ids, True))
     from tests.gpu_util import err_bf16_out
     assert err_bf16_out(oh, want) <= 2e-2
+
+
+@pytest.mark.parametrize("name", ["qwen15_t32", "decode_t1"])
+def test_layer_handle_with_fp32_packed_outputs(name):
+    # y_f32: y_packed (and the shared expert's output) kept in fp32, as the
+    # Python chain does with MoELayerBuffers(y_f32=True): the same bits
+    cfg = CONFIGS[name]
+    p = make_layer(cfg, seed=3)
+    dp = params_to(p)
+    buf = M.MoELayerBuffers(cfg.T, cfg.H, cfg.E, cfg.k, cfg.I, cfg.torch_dtype,
+                            shared_I=cfg.shared_I, y_f32=True)
+    assert buf.y_packed.dtype == torch.float32
+    ref = M.moe_layer_forward(dp["x"], dp, cfg.k, cfg.renormalize, buf).clone()
+    L = M.MoELayer(dp, cfg.T, cfg.k, cfg.renormalize, y_f32=True)
+    out = torch.empty_like(ref)
+    L.forward(dp["x"], out)
+    torch.cuda.synchronize()
+    assert L.status() == 0
+    assert torch.equal(_bits(out), _bits(ref))
+    y = L.buffer("y_packed", (cfg.T * cfg.k, cfg.H), torch.float32)
+    assert torch.equal(y, buf.y_packed)
+    L.close()
