@@ -42,25 +42,32 @@ constexpr int DNT = 256;           // threads per CTA
 constexpr int DWARPS = DNT / 32;
 constexpr int PER_WARP = CHUNK / DWARPS;
 
-// Per-warp per-expert counts of this CTA's slice.  Invalid ids (outside
-// [0,E)) are reported and skipped.  wc: [DWARPS][E] in shared memory.
-__device__ __forceinline__ void warp_counts(const int32_t* ids, int N, int E,
-                                            int base, int* wc, int32_t* status) {
+constexpr int ROUNDS = PER_WARP / 32;
+
+// Per-warp per-expert counts of this CTA's slice.  The warp's ids are read
+// once, all loads in flight together, into eid (-1: no assignment, or an id
+// outside [0,E), which is reported and skipped).  wc: [DWARPS][E] in shared
+// memory.
+__device__ __forceinline__ void warp_counts(const int32_t* ids, int N, int E, int base,
+                                            int (&eid)[ROUNDS], int* wc, int32_t* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < DWARPS * E; i += DNT) wc[i] = 0;
   moe::grid_dep_wait();
-  __syncthreads();
   const int w0 = base + warp * PER_WARP;
-  for (int r = 0; r < PER_WARP; r += 32) {
-    const int f = w0 + r + lane;
-    int e = -1;
-    if (f < N) {
-      e = moe::ld_prod(ids + f);
-      if (e < 0 || e >= E) {
-        moe::report(status, MOE_ERR_BAD_INDEX);
-        e = -1;
-      }
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    const int f = w0 + 32 * i + lane;
+    eid[i] = f < N ? moe::ld_prod(ids + f) : -1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    int e = eid[i];
+    if (w0 + 32 * i + lane < N && (e < 0 || e >= E)) {
+      if (status) moe::report(status, MOE_ERR_BAD_INDEX);
+      e = -1;
     }
+    eid[i] = e;
     const unsigned valid = __ballot_sync(0xffffffffu, e >= 0);
     // Lanes without a valid id get a unique key so they never match.
     const int key = e >= 0 ? e : -1 - lane;
@@ -75,7 +82,8 @@ __global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* ids,
                                                              int32_t* __restrict__ bc,
                                                              int32_t* status) {
   extern __shared__ int wc[];
-  warp_counts(ids, N, E, blockIdx.x * CHUNK, wc, status);
+  int eid[ROUNDS];
+  warp_counts(ids, N, E, blockIdx.x * CHUNK, eid, wc, status);
   for (int e = threadIdx.x; e < E; e += DNT) {
     int s = 0;
 #pragma unroll
@@ -92,9 +100,18 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
   __shared__ int s_scan[256];
   const int e = threadIdx.x;
   moe::grid_dep_wait();
+  // The column of CTA counts is read in batches of 16 loads in flight.
+  constexpr int BATCH = 16;
   int total = 0;
   if (e < E)
-    for (int b = 0; b < B; ++b) total += moe::ld_prod(bc + static_cast<size_t>(b) * E + e);
+    for (int b0 = 0; b0 < B; b0 += BATCH) {
+      int c[BATCH];
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j)
+        c[j] = b0 + j < B ? moe::ld_prod(bc + static_cast<size_t>(b0 + j) * E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j) total += c[j];
+    }
   // Exclusive scan over experts (Hillis-Steele on 256 entries).
   s_scan[e] = total;
   __syncthreads();
@@ -109,11 +126,17 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict_
     counts[e] = total;
     offsets[e] = excl;
     int run = excl;
-    for (int b = 0; b < B; ++b) {
-      const size_t i = static_cast<size_t>(b) * E + e;
-      const int c = moe::ld_prod(bc + i);
-      bc[i] = run;
-      run += c;
+    for (int b0 = 0; b0 < B; b0 += BATCH) {
+      int c[BATCH];
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j)
+        c[j] = b0 + j < B ? moe::ld_prod(bc + static_cast<size_t>(b0 + j) * E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j)
+        if (b0 + j < B) {
+          bc[static_cast<size_t>(b0 + j) * E + e] = run;
+          run += c[j];
+        }
     }
   }
   if (e == 255) offsets[E] = s_scan[255];
@@ -125,43 +148,77 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     const int32_t* bc, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
     int32_t* __restrict__ packed_tok, float* __restrict__ packed_w, int32_t* status) {
   extern __shared__ int wc[];  // [DWARPS][E] counts, then bases
+  // The CTA's assignments in local expert-major order (position, f, weight),
+  // copied out after the scatter: consecutive local entries of one expert go
+  // to consecutive positions, so the stores come in runs instead of one
+  // L2 write per assignment.
+  __shared__ int s_pos[CHUNK], s_f[CHUNK];
+  __shared__ float s_w[CHUNK];
+  __shared__ int s_shift[moe::kMaxExperts];   // local index - position, per expert
+  __shared__ int s_scan[DNT];
   const int base = blockIdx.x * CHUNK;
-  warp_counts(ids, N, E, base, wc, nullptr);
-  for (int e = threadIdx.x; e < E; e += DNT) {
-    int run = moe::ld_prod(bc + static_cast<size_t>(blockIdx.x) * E + e);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w0 = base + warp * PER_WARP;
+  int eid[ROUNDS];
+  warp_counts(ids, N, E, base, eid, wc, nullptr);
+  float wv[ROUNDS];
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    const int f = w0 + 32 * i + lane;
+    wv[i] = packed_w != nullptr && f < N ? moe::ld_prod(w + f) : 0.f;
+  }
+  // Per-warp global bases, and the CTA's total per expert (E <= DNT).
+  int total = 0, gbase = 0;
+  const int e = threadIdx.x;
+  if (e < E) {
+    gbase = moe::ld_prod(bc + static_cast<size_t>(blockIdx.x) * E + e);
+    int run = gbase;
 #pragma unroll
     for (int ww = 0; ww < DWARPS; ++ww) {
       const int c = wc[ww * E + e];
       wc[ww * E + e] = run;
       run += c;
     }
+    total = run - gbase;
+  }
+  // Local exclusive scan of the totals over the experts.
+  s_scan[e] = total;
+  __syncthreads();
+  for (int o = 1; o < DNT; o <<= 1) {
+    const int v = e >= o ? s_scan[e - o] : 0;
+    __syncthreads();
+    s_scan[e] += v;
+    __syncthreads();
+  }
+  if (e < E) s_shift[e] = s_scan[e] - total - gbase;
+  const int nvalid = s_scan[DNT - 1];
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int i = 0; i < ROUNDS; ++i) {
+    const int f = w0 + 32 * i + lane;
+    const int ex = eid[i];
+    if (f < N && ex < 0) inv_perm[f] = -1;
+    const int key = ex >= 0 ? ex : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    if (ex >= 0) {
+      const int p = wc[warp * E + ex] + __popc(peers & lt);
+      inv_perm[f] = p;
+      const int q = p + s_shift[ex];
+      s_pos[q] = p;
+      s_f[q] = f;
+      s_w[q] = wv[i];
+    }
+    __syncwarp();
+    if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
+    __syncwarp();
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  const int w0 = base + warp * PER_WARP;
-  for (int r = 0; r < PER_WARP; r += 32) {
-    const int f = w0 + r + lane;
-    int e = -1;
-    if (f < N) {
-      e = moe::ld_prod(ids + f);
-      if (e < 0 || e >= E) {
-        e = -1;
-        inv_perm[f] = -1;
-      }
-    }
-    const int key = e >= 0 ? e : -1 - lane;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    if (e >= 0) {
-      const int p = wc[warp * E + e] + __popc(peers & lt);
-      perm[p] = f;
-      inv_perm[f] = p;
-      packed_tok[p] = f / k;
-      if (packed_w) packed_w[p] = moe::ld_prod(w + f);
-    }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
-    __syncwarp();
+  for (int q = threadIdx.x; q < nvalid; q += DNT) {
+    const int p = s_pos[q], f = s_f[q];
+    perm[p] = f;
+    packed_tok[p] = f / k;
+    if (packed_w) packed_w[p] = s_w[q];
   }
   moe::grid_dep_launch();
 }
@@ -178,14 +235,15 @@ __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
     int32_t* __restrict__ inv_perm, int32_t* __restrict__ packed_tok,
     float* __restrict__ packed_w, const uint4* x, int row_vecs,
     uint4* __restrict__ xp, int32_t* status) {
-  extern __shared__ int wc[];                  // [SMALL_WARPS][E]
+  extern __shared__ int wc[];                  // [SMALL_WARPS][E], then the staging arrays
   __shared__ int s_scan[moe::kMaxExperts];
   for (int i = threadIdx.x; i < SMALL_WARPS * E; i += blockDim.x) wc[i] = 0;
   moe::grid_dep_wait();
   __syncthreads();
   moe::dispatch_cta<SMALL_WARPS, SMALL_PER_WARP / 32>(ids, w, N, E, k, counts, offsets, perm,
                                                       inv_perm, packed_tok, packed_w, x,
-                                                      row_vecs, xp, status, wc, s_scan);
+                                                      row_vecs, xp, status, wc, s_scan,
+                                                      wc + SMALL_WARPS * E);
 }
 
 // ------------------------------------------------------------- gather ---
@@ -304,8 +362,13 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
     // One CTA copies at most 128 KiB of rows; more goes to the multi-CTA gather.
     const bool fuse_gather =
         x != nullptr && static_cast<size_t>(N) * row_bytes <= (static_cast<size_t>(128) << 10);
-    cudaError_t err = launch_pdl(
-        dispatch_small_kernel, dim3(1), dim3(SMALL_WARPS * 32), sizeof(int) * SMALL_WARPS * E, s,
+    // per-warp counts, then perm, packed_tok and packed_w staged (at most 128 KiB)
+    const size_t sm = sizeof(int) * (static_cast<size_t>(SMALL_WARPS) * E + 3 * SMALL_N);
+    cudaError_t err =
+        ensure_smem(reinterpret_cast<const void*>(dispatch_small_kernel), static_cast<int>(sm));
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(
+        dispatch_small_kernel, dim3(1), dim3(SMALL_WARPS * 32), sm, s,
         0, ids, w, N, E, k, counts, offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,
         fuse_gather ? static_cast<const uint4*>(x) : nullptr, row_bytes / 16,
         static_cast<uint4*>(x_packed), status);

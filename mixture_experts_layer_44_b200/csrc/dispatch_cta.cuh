@@ -18,23 +18,33 @@ namespace moe {
 // by the caller before a __syncthreads; s_scan: shared [kMaxExperts].  Every
 // thread of the CTA calls this (it synchronises the CTA).  Ids outside [0,E)
 // are reported (MOE_ERR_BAD_INDEX), given inv_perm -1 and left out.
+//
+// With stage (shared, 3 * NW * 32 * ROUNDS ints) the scatter writes perm,
+// packed_tok and packed_w into shared memory, and the CTA then copies the
+// three arrays out in position order: a scattered 4-byte store from one SM
+// costs a separate L2 write per distinct sector, a copied-out row of 32
+// positions costs four.
 template <int NW, int ROUNDS>
 __device__ __forceinline__ void dispatch_cta(
     const int32_t* ids, const float* w, int N, int E, int k, int32_t* counts, int32_t* offsets,
     int32_t* perm, int32_t* inv_perm, int32_t* packed_tok, float* packed_w, const uint4* x,
-    int row_vecs, uint4* xp, int32_t* status, int* wc, int* s_scan) {
+    int row_vecs, uint4* xp, int32_t* status, int* wc, int* s_scan, int* stage = nullptr) {
+  constexpr int NMAX = NW * 32 * ROUNDS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   const int per = (N + NW - 1) / NW;
   const int w0 = warp * per, w1 = min(N, w0 + per);
-  // The warp's slice of ids, read once (all loads in flight together) and
-  // kept in registers for both passes; -1 marks no assignment / a bad id.
+  // The warp's slice of ids and weights, read once (all loads in flight
+  // together) and kept in registers for both passes; -1 marks no assignment
+  // or a bad id.
   const int nr = w1 > w0 ? (w1 - w0 + 31) / 32 : 0;   // rounds this warp needs
   int eid[ROUNDS];
+  float wv[ROUNDS];
 #pragma unroll
   for (int i = 0; i < ROUNDS; ++i) {
     const int f = w0 + 32 * i + lane;
     eid[i] = f < w1 ? ld_prod(ids + f) : -1;
+    wv[i] = packed_w != nullptr && f < w1 ? ld_prod(w + f) : 0.f;
   }
   // 1. per-warp counts over this warp's contiguous slice
 #pragma unroll
@@ -88,21 +98,35 @@ __device__ __forceinline__ void dispatch_cta(
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     if (ex >= 0) {
       const int p = wc[warp * E + ex] + __popc(peers & lt);
-      perm[p] = f;
       inv_perm[f] = p;
-      packed_tok[p] = f / k;
-      if (packed_w) packed_w[p] = ld_prod(w + f);
+      if (stage != nullptr) {
+        stage[p] = f;
+        stage[NMAX + p] = f / k;
+        stage[2 * NMAX + p] = __float_as_int(wv[i]);
+      } else {
+        perm[p] = f;
+        packed_tok[p] = f / k;
+        if (packed_w) packed_w[p] = wv[i];
+      }
     }
     __syncwarp();
     if (ex >= 0 && lane == __ffs(peers) - 1) wc[warp * E + ex] += __popc(peers);
     __syncwarp();
+  }
+  const int nrows = s_scan[kMaxExperts - 1];
+  if (stage != nullptr) {
+    __syncthreads();
+    for (int p = threadIdx.x; p < nrows; p += NW * 32) {
+      perm[p] = stage[p];
+      packed_tok[p] = stage[NMAX + p];
+      if (packed_w) packed_w[p] = __int_as_float(stage[2 * NMAX + p]);
+    }
   }
   grid_dep_launch();
   if (x == nullptr) return;
   __syncthreads();
   // 4. gather (small total): one warp per row, 16-byte vectors, 8 loads in
   //    flight per lane before the stores
-  const int nrows = s_scan[kMaxExperts - 1];
   for (int p = warp; p < nrows; p += NW) {
     const uint4* src = x + static_cast<size_t>(ld_prod(packed_tok + p)) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
