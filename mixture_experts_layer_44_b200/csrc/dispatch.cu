@@ -6,7 +6,7 @@
 // activations for the expert ranges.  Assignment f = t*k + j (row-major
 // [T, k], the flat order of metrale's ep_dispatch.rs).
 //
-// Small batches (N <= 8192 assignments) take one CTA of 32 warps through
+// Small batches (N <= 2048 assignments) take one CTA of 32 warps through
 // count, scan and scatter in a single launch (the same warp-slice algorithm
 // as below), and also gather the rows when they total at most 128 KiB
 // (decode); larger gathers use the bulk-copy kernel.  Larger N takes four launches:
@@ -22,6 +22,8 @@
 //              round a lane's rank among equal experts is the popcount of
 //              the lower lanes in its match mask.  Positions therefore grow
 //              with f inside an expert: the order is stable (bit-exact).
+//              The CTA's entries are staged in shared memory in expert
+//              order and stored in runs of consecutive positions.
 //   gather  -- x_packed[p] = x[packed_tok[p]] with bulk asynchronous copies
 //              (global -> shared -> global on the TMA engine), one issuing
 //              lane per warp, a 4-row ring per warp.
@@ -225,9 +227,12 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
 
 // ------------------------------------------------- single-CTA variant ---
 
+// Up to 2048 assignments.  Above that the multi-CTA kernels are faster even
+// with their two extra launches: one SM's match / scatter rounds over 8192
+// assignments took 18 us, four CTAs of 2048 take 11 us.
 constexpr int SMALL_WARPS = 32;
-constexpr int SMALL_PER_WARP = 256;
-constexpr int SMALL_N = SMALL_WARPS * SMALL_PER_WARP;   // 8192 assignments
+constexpr int SMALL_PER_WARP = 64;
+constexpr int SMALL_N = SMALL_WARPS * SMALL_PER_WARP;   // 2048 assignments
 
 __global__ void __launch_bounds__(SMALL_WARPS * 32) dispatch_small_kernel(
     const int32_t* ids, const float* w, int N, int E, int k,

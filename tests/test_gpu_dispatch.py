@@ -53,7 +53,8 @@ def _check(ids, w, x, E):
 
 @pytest.mark.parametrize("T,k,E", [(1, 1, 1), (1, 2, 8), (5, 3, 4), (64, 2, 8), (300, 4, 60),
                                    (1000, 8, 128), (4096, 2, 64), (2049, 1, 3), (700, 8, 256),
-                                   (2000, 8, 256), (10000, 1, 1), (4097, 2, 64)])
+                                   (2000, 8, 256), (10000, 1, 1), (4097, 2, 64), (1024, 2, 16),
+                                   (256, 8, 256)])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_dispatch_random(T, k, E, dtype):
     rng = np.random.default_rng(T * 31 + k * 7 + E)
