@@ -125,6 +125,15 @@ constexpr size_t CTL_BYTES = (sizeof(Ctl) + 1023) / 1024 * 1024;
 // the same stage's B tile -- garbage in accumulator rows that are never
 // stored -- and the 12 KB saved per stage buy a fifth stage, 25 % more weight
 // bytes in flight per SM.
+//
+// A routed tile with at most 32 (64) valid rows loads only 32 (64) rows of
+// A, in one box; the rows not loaded hold stale data of an earlier stage and
+// likewise only reach accumulator rows that are never stored.  A-tile
+// reads, although they hit L2, slow the weight stream from DRAM (a TMA-only
+// probe of the builder's w13 shape: 6.38 TB/s of weights alone, 5.07 with a
+// 16 KB A box per 32 KB weight box, 5.97 with a 4 KB one).  One box per
+// stage matters as much: four 32-row boxes instead of one 128-row box made
+// the prefill GEMMs 10-15 % slower.
 template <int AR>
 struct Ring {
   static constexpr int A_B = AR * BK * 2;
@@ -337,6 +346,8 @@ __device__ __forceinline__ float store_h16x64(__half* dst, const uint32_t (&a)[4
 template <int EPI, bool SHARED, bool YH, int AR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmA64,
+                        const __grid_constant__ CUtensorMap tmA32,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmB2,
@@ -380,6 +391,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     c.abort = 0;
     moe::fence_barrier_init();
     moe::prefetch_tmap(&tmA);
+    if (AR == BM) {
+      moe::prefetch_tmap(&tmA64);
+      moe::prefetch_tmap(&tmA32);
+    }
     moe::prefetch_tmap(&tmB);
     if (rows2 > 0) {
       moe::prefetch_tmap(&tmA2);
@@ -481,6 +496,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   // The B operand (weights) of k-block kb of unit un into stage buffer sa,
   // completing on barrier fb.
+  // The A box of a unit (its map and rows): 32 or 64 rows for a routed
+  // tile with at most that many valid rows, else the full AR rows.
+  auto a_rows = [&](const Unit& un) {
+    if (AR != BM || (SHARED && un.g)) return AR;
+    const int rows = un.rend - un.row0;
+    return rows <= 32 ? 32 : (rows <= 64 ? 64 : BM);
+  };
+  auto a_map = [&](const Unit& un, int ar) -> const CUtensorMap* {
+    if (SHARED && un.g) return &tmA2;
+    return ar == 32 && AR == BM ? &tmA32 : (ar == 64 ? &tmA64 : &tmA);
+  };
+  auto stage_tx = [&](int ar) {
+    return static_cast<uint32_t>(STAGE_BYTES - A_BYTES + ar * BK * 2);
+  };
+
   auto load_b = [&](const Unit& un, int kb, uint32_t sa, uint32_t fb) {
     if (SHARED && un.g) {
       if (EPI == EPI_SWIGLU)
@@ -517,9 +547,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (EARLY && warp == 0 && lane == 0 && static_cast<int>(blockIdx.x) < total) {
     const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, blockIdx.x);
     pre = min(STAGES, un.kb1 - un.kb0);
+    const uint32_t tx = stage_tx(a_rows(un));
     for (int s = 0; s < pre; ++s) {
       const uint32_t fb = moe::smem_addr(&c.full[s]);
-      moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+      moe::mbar_arrive_expect_tx(fb, tx);
       load_b(un, un.kb0 + s, moe::smem_addr(smem + s * STAGE_BYTES), fb);
       pre_issued[s] = 1;
     }
@@ -563,7 +594,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const Unit un = decode_unit<SHARED>(c, E, kblocks, kblocks2, u);
         const int arow = un.row0;
         const bool g1 = SHARED && un.g;
-        const CUtensorMap* ma = g1 ? &tmA2 : &tmA;
+        const int ar = a_rows(un);
+        const CUtensorMap* ma = a_map(un, ar);
+        const uint32_t tx = stage_tx(ar);
         bool ok = true;
         for (int kb = un.kb0; kb < un.kb1; ++kb) {
           const uint32_t fb = moe::smem_addr(&c.full[stage]);
@@ -577,7 +610,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               ok = false;
               break;
             }
-            moe::mbar_arrive_expect_tx(fb, STAGE_BYTES);
+            moe::mbar_arrive_expect_tx(fb, tx);
             moe::tma_load_2d(sa, ma, fb, kb * BK, arow);
             load_b(un, kb, sa, fb);
             ++issued[stage];
@@ -935,7 +968,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// Activations [rows, K] bf16, box 64 x ar (the A tile of one stage).
+// Activations [rows, K] bf16, box 64 x ar (a stage's A tile).
 bool map_rows(CUtensorMap* m, const void* p, int rows, int K, int ar) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t str[1] = {static_cast<cuuint64_t>(K) * 2};
@@ -1008,8 +1041,10 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   e1 = ensure_smem(reinterpret_cast<const void*>(k2), static_cast<int>(smem));
   if (e1 != cudaSuccess) return e1;
   const int nmap = N > 0 ? N : 1;           // a map needs one row; no tile reads it when N == 0
-  CUtensorMap mA1, mB1, mA2, mB2;
-  bool ok = map_rows(&mA1, x_packed, nmap, H, ar) && map_rows(&mA2, h, nmap, I, ar);
+  CUtensorMap mA1, mB1, mA2, mB2, mA1_64, mA1_32, mA2_64, mA2_32;
+  bool ok = map_rows(&mA1, x_packed, nmap, H, ar) && map_rows(&mA2, h, nmap, I, ar) &&
+            map_rows(&mA1_64, x_packed, nmap, H, 64) && map_rows(&mA1_32, x_packed, nmap, H, 32) &&
+            map_rows(&mA2_64, h, nmap, I, 64) && map_rows(&mA2_32, h, nmap, I, 32);
   {
     // w13 as [2E][I][H]: one box = 128 gate rows + the matching 128 up rows.
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(I),
@@ -1074,12 +1109,14 @@ cudaError_t launch_experts_tc(const void* x_packed, const int32_t* offsets,
   }
   const float* no_w = nullptr;
   const uint64_t wait_ns = main_wait_budget_ns();
-  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS), smem, s, 0, mA1, mB1, sA1, sB1,
+  cudaError_t err = launch_pdl(k1, dim3(g1), dim3(NTHREADS), smem, s, 0, mA1, mA1_64, mA1_32,
+                               mB1, sA1, sB1,
                                mY, sY, offsets, E, H, ntw1, 2 * I, no_w, h, I, T2, H, ntw1s,
                                sh ? sh->h : nullptr, Is, counters, partials, max_units, status,
                                wait_ns);
   if (err != cudaSuccess) return err;
-  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), smem, s, 0, mA2, mB2, sA2, sB2, mY, sY,
+  return launch_pdl(k2, dim3(g2), dim3(NTHREADS), smem, s, 0, mA2, mA2_64, mA2_32, mB2, sA2,
+                    sB2, mY, sY,
                     offsets, E, I, H / BN, H, packed_w, y, H, T2, Is, H / BN,
                     sh ? sh->y : nullptr, H, counters, partials, max_units, status, wait_ns);
 }
