@@ -28,7 +28,7 @@
 
 namespace {
 
-constexpr int CNT = 256;
+constexpr int CNT = 256;   // threads per CTA of the finalize kernel
 
 // Eight consecutive elements of an fp32 or fp16 row, as fp32 (read at L2:
 // the rows come from the kernels just before).
@@ -57,8 +57,11 @@ struct Vec8<true> {
   __device__ __forceinline__ void get(float* f) const { moe::unpack8_f16(q, f); }
 };
 
-template <bool Y_F16, bool OUT_BF16, int KT>
-__global__ void __launch_bounds__(CNT) combine_kernel(const void* y,
+// NT threads per CTA (one token at a time): 256 while the tokens fit one
+// wave of 8 CTAs per SM (decode: the shortest chain per token), 128 above it
+// (16 tokens in flight per SM: Qwen1.5 T = 8192 merger 51 -> 44 us).
+template <bool Y_F16, bool OUT_BF16, int KT, int NT>
+__global__ void __launch_bounds__(NT) combine_kernel(const void* y,
                                                       const int32_t* inv_perm,
                                                       int T, int H, int k, int N,
                                                       const void* shared,
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(CNT) combine_kernel(const void* y,
     if (threadIdx.x == 0)
       gate = shared ? (sgate ? 1.f / (1.f + expf(-moe::ld_prod(sgate + t))) : 1.f) : 0.f;
     __syncthreads();
-    for (int v = threadIdx.x; v < nvec; v += CNT) {
+    for (int v = threadIdx.x; v < nvec; v += NT) {
       float acc[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -172,14 +175,18 @@ cudaError_t launch_combine_t(const void* y, const int32_t* inv_perm, int T, int 
                              const void* shared, const float* shared_gate, void* out,
                              int32_t* status, cudaStream_t s, const int32_t* range_offs,
                              int lo_e, int hi_e) {
-  const int grid = std::max(1, std::min(T, num_sms() * 8));
+  const bool narrow = T > num_sms() * 8;
+  const int grid = std::max(1, std::min(T, num_sms() * (narrow ? 16 : 8)));
   const int N = T * k;
   // k is a template parameter so that exactly k rows are loaded, all in flight.
-#define MOE_COMBINE_K(KV)                                                                     \
-  case KV:                                                                                    \
-    return launch_pdl(combine_kernel<Y_F16, OUT_BF16, KV>, dim3(grid), dim3(CNT), 0, s, 0, y, \
-                      inv_perm, T, H, k, N, shared, shared_gate, range_offs, lo_e, hi_e, out,  \
-                      status);
+#define MOE_COMBINE_K(KV)                                                                      \
+  case KV:                                                                                     \
+    return narrow ? launch_pdl(combine_kernel<Y_F16, OUT_BF16, KV, 128>, dim3(grid), dim3(128), \
+                               0, s, 0, y, inv_perm, T, H, k, N, shared, shared_gate,          \
+                               range_offs, lo_e, hi_e, out, status)                            \
+                  : launch_pdl(combine_kernel<Y_F16, OUT_BF16, KV, 256>, dim3(grid), dim3(256), \
+                               0, s, 0, y, inv_perm, T, H, k, N, shared, shared_gate,          \
+                               range_offs, lo_e, hi_e, out, status);
   switch (k) {
     MOE_COMBINE_K(1)
     MOE_COMBINE_K(2)
