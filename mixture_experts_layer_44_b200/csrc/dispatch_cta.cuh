@@ -62,19 +62,27 @@ __device__ __forceinline__ void dispatch_cta(
     if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * E + e] += __popc(peers);
   }
   __syncthreads();
-  // 2. counts, exclusive scan over experts, per-warp bases (blockDim >= 256)
+  // 2. counts, inclusive scan over experts into s_scan (a shuffle scan in
+  //    each warp of 32 experts, then the warp totals), per-warp bases
+  //    (blockDim >= 256)
   const int e = threadIdx.x;
   int total = 0;
   if (e < E)
     for (int ww = 0; ww < NW; ++ww) total += wc[ww * E + e];
-  if (e < kMaxExperts) s_scan[e] = total;
-  __syncthreads();
-  for (int o = 1; o < kMaxExperts; o <<= 1) {
-    const int v = (e < kMaxExperts && e >= o) ? s_scan[e - o] : 0;
-    __syncthreads();
-    if (e < kMaxExperts) s_scan[e] += v;
-    __syncthreads();
+  __shared__ int s_wsum[kMaxExperts / 32];
+  int incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
+  if (e < kMaxExperts && lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  if (e < kMaxExperts) {
+    for (int ww = 0; ww < warp; ++ww) incl += s_wsum[ww];
+    s_scan[e] = incl;
+  }
+  __syncthreads();
   if (e < E) {
     const int excl = s_scan[e] - total;
     counts[e] = total;
@@ -128,7 +136,8 @@ __device__ __forceinline__ void dispatch_cta(
   // 4. gather (small total): one warp per row, 16-byte vectors, 8 loads in
   //    flight per lane before the stores
   for (int p = warp; p < nrows; p += NW) {
-    const uint4* src = x + static_cast<size_t>(ld_prod(packed_tok + p)) * row_vecs;
+    const int tok = stage != nullptr ? stage[NMAX + p] : ld_prod(packed_tok + p);
+    const uint4* src = x + static_cast<size_t>(tok) * row_vecs;
     uint4* dst = xp + static_cast<size_t>(p) * row_vecs;
     for (int v0 = lane; v0 < row_vecs; v0 += 32 * 8) {
       uint4 q[8];

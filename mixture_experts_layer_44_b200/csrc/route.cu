@@ -113,25 +113,15 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nvec = H / 8;
-  moe::grid_dep_wait();
-  for (int v = threadIdx.x; v < nvec; v += NS) {
-    float f[8];
-    load8<BF16>(xv, static_cast<size_t>(t) * H + v * 8, true, f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) xs[v * 8 + j] = f[j];
-  }
-  __syncthreads();
   const int slice = warp % WPE;
   const int group = warp / WPE;
   const int vs = slice * nvec / WPE, ve = (slice + 1) * nvec / WPE;
   const uint4* wb = reinterpret_cast<const uint4*>(wv);
-  float acc[EPW];
-#pragma unroll
-  for (int i = 0; i < EPW; ++i) acc[i] = 0.f;
-  for (int vb = vs + lane; vb < ve; vb += 32 * BATCH) {
-    // loads are unconditional (clamped to the slice's last vector) so that a
-    // whole batch is in flight before the first FMA
-    uint4 wq[EPW][BATCH][Q];
+  // One batch of W_gate vectors per lane; the loads are unconditional
+  // (clamped to the slice's last vector) so that a whole batch is in flight
+  // before the first FMA.
+  uint4 wq[EPW][BATCH][Q];
+  auto load_w = [&](int vb) {
 #pragma unroll
     for (int i = 0; i < EPW; ++i) {
       const int e = min(group + GROUPS * i, E - 1);
@@ -143,6 +133,24 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
           wq[i][j][q] = moe::ld_nc_v4(wb + (static_cast<size_t>(e) * nvec + vc) * Q + q);
       }
     }
+  };
+  // W_gate is a weight, never written by the kernel just before this one
+  // (only this library's kernels let a successor start early, and none
+  // writes it): the first batch is requested before waiting for that kernel.
+  if (vs + lane < ve) load_w(vs + lane);
+  moe::grid_dep_wait();
+  for (int v = threadIdx.x; v < nvec; v += NS) {
+    float f[8];
+    load8<BF16>(xv, static_cast<size_t>(t) * H + v * 8, true, f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xs[v * 8 + j] = f[j];
+  }
+  __syncthreads();
+  float acc[EPW];
+#pragma unroll
+  for (int i = 0; i < EPW; ++i) acc[i] = 0.f;
+  for (int vb = vs + lane; vb < ve; vb += 32 * BATCH) {
+    if (vb != vs + lane) load_w(vb);
 #pragma unroll
     for (int j = 0; j < BATCH; ++j) {
       const int v = vb + 32 * j;
@@ -207,20 +215,27 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
     __shared__ int s_last;
     __shared__ int s_scan[moe::kMaxExperts];
     __syncthreads();                           // this token's ids and weights are written
+    const bool one = gridDim.x == 1;           // a single token: no other CTA to wait for
     if (threadIdx.x == 0) {
-      __threadfence();
-      s_last = atomicAdd(dd.counter, 1) == static_cast<int>(gridDim.x) - 1;
+      if (one) {
+        s_last = 1;
+      } else {
+        __threadfence();
+        s_last = atomicAdd(dd.counter, 1) == static_cast<int>(gridDim.x) - 1;
+      }
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();                           // every other token's writes are now visible
-    int* wc = reinterpret_cast<int*>(xs);      // [NWARP][E]: x is no longer needed
+    if (!one) __threadfence();                 // every other token's writes are now visible
+    // x is no longer needed: its shared memory holds the [NWARP][E] counts,
+    // then the staged perm, packed_tok and packed_w
+    int* wc = reinterpret_cast<int*>(xs);
     for (int i = threadIdx.x; i < NWARP * E; i += NS) wc[i] = 0;
     __syncthreads();
     moe::dispatch_cta<NWARP, kFusedRounds>(ids, wout, static_cast<int>(gridDim.x) * k, E, k,
                                            dd.counts, dd.offsets, dd.perm, dd.inv_perm,
                                            dd.packed_tok, dd.packed_w, dd.x, dd.row_vecs,
-                                           dd.x_packed, dd.status, wc, s_scan);
+                                           dd.x_packed, dd.status, wc, s_scan, wc + NWARP * E);
     if (threadIdx.x == 0) *dd.counter = 0;
   }
 }
@@ -424,8 +439,9 @@ template <int EP, bool FUSED>
 cudaError_t launch_small_ep(const void* x, const void* W, const float* b, int T, int H, int E,
                             int k, int renorm, bool bf, float* logits, int32_t* ids, float* w,
                             moe::GroupLimit gl, const SmallDispatch& dd, cudaStream_t s) {
-  // The fused dispatch reuses the x row's shared memory for its [16][E] counts.
-  const int smem = std::max(H, FUSED ? (NS / 32) * E : 0) * 4;
+  // The fused dispatch reuses the x row's shared memory for its [16][E]
+  // counts and its three staged [512] arrays.
+  const int smem = std::max(H, FUSED ? (NS / 32) * E + 3 * NS * kFusedRounds : 0) * 4;
   auto fn = bf ? route_small_kernel<EP, true, FUSED> : route_small_kernel<EP, false, FUSED>;
   cudaError_t e = moe_host::ensure_smem(reinterpret_cast<const void*>(fn), smem);
   if (e != cudaSuccess) return e;
