@@ -178,9 +178,10 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x,
  * array of the library (a file-scope __device__ array of 128 KiB that every
  * GPU which loads the library holds until the process exits).  The call
  * allocates nothing.
- *   - Limit: ceil(T*k / 2048) * E <= 32768 (e.g. T*k <= 524288 at E = 128);
- *     larger problems return MOE_ERR_INVALID_ARG with a message naming the
- *     limit.  Use moe_dispatch with a workspace for them.
+ *   - Limit: ceil(T*k / 2048) * E <= 32768 (e.g. T*k <= 524288 at E = 128;
+ *     up to T*k = 65536 the table always fits); larger problems return
+ *     MOE_ERR_INVALID_ARG with a message naming the limit.  Use moe_dispatch
+ *     with a workspace for them.
  *   - The first call on a device looks up the array's device address on that
  *     device (cudaGetSymbolAddress), so make that first call before any
  *     stream capture.  The address is cached per device and CUDA context and
