@@ -57,6 +57,11 @@ def test_abi_version_and_workspace_queries(lib):
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
     assert M.moe_dispatch_workspace_bytes(0, 2, 8) == 0
+    # up to T*k = 65536 the count and scatter CTAs take 1024 assignments each:
+    # one count row per 1024, and at most 64 * E entries (inside the 128 KiB
+    # of the allocation-free entry point even at E = 256)
+    assert M.moe_dispatch_workspace_bytes(4096, 2, 64) >= 8 * 64 * 4
+    assert M.moe_dispatch_workspace_bytes(65536, 1, 256) <= 128 * 1024
     assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_BF16) >= 4096 * 4 + 128 * 1024
     assert M.moe_experts_workspace_bytes(100, 256, 128, 4, M.MOE_F32) == 0
 
