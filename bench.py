@@ -377,9 +377,11 @@ class Layer:
         shared = cfg.shared_I is not None
         if ev:
             ev[0].record(stream)
+        gate_done = False
         if buf.route_dispatch:
-            # decode batches: router and dispatcher are one launch (timed as "route")
-            M.route_and_dispatch(x, dp, cfg.k, cfg.renormalize, buf, stream)
+            # decode batches: router (with a shared expert's gate) and dispatcher are one
+            # launch (timed as "route")
+            gate_done = M.route_and_dispatch(x, dp, cfg.k, cfg.renormalize, buf, stream)
             if ev:
                 ev[1].record(stream)
         else:
@@ -396,8 +398,9 @@ class Layer:
             M.moe_experts(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"], dp["w2"], buf.h,
                           buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
         else:
-            M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
-                        status=buf.status, stream=stream)
+            if not gate_done:
+                M.moe_route(x, dp["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
+                            status=buf.status, stream=stream)
             if buf.fuse_shared:
                 M.moe_experts_shared(buf.x_packed, buf.offsets, buf.packed_w, dp["w13"],
                                      dp["w2"], buf.h, buf.y_packed, x, dp["w13s"], dp["w2s"],

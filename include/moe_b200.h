@@ -218,13 +218,28 @@ int moe_dispatch_noalloc(const int32_t* topk_ids, const float* topk_w, const voi
  *   counter   device int32, zero before the first call; every call leaves it
  *             at zero again.  Calls that may overlap on the GPU (different
  *             streams) need different counters.
- *   Needs 1 <= T <= 64, 1 <= E <= 64, H <= 32768 and 1 <= k <= min(E, 8):
- *   other shapes return MOE_ERR_INVALID_ARG (use the two separate calls).
+ *   w_gate_shared      device [H] (dtype): the always-on shared expert's gate
+ *                      row (diffulex.moe.layer, SharedExpertMLP), or NULL;
+ *   shared_gate_logit  device [T] f32: x[t] . w_gate_shared (no bias), the
+ *                      logit moe_combine's sigmoid gate takes; NULL exactly
+ *                      when w_gate_shared is.  The gate is contracted as one
+ *                      more row beside the E experts, in the same launch, and
+ *                      takes no part in the selection; it equals moe_route
+ *                      with E = 1, k = 0 on that row up to fp32 summation
+ *                      order.  When E + 1 passes a power of two, the routed
+ *                      rows are contracted in a larger block too, and their
+ *                      logits can then differ from the call without the gate
+ *                      in fp32 summation order (the bit-for-bit identity with
+ *                      the two separate calls holds without a gate).
+ *   Needs 1 <= T <= 64, 1 <= E <= 64 (E <= 63 with a shared gate),
+ *   H <= 32768 and 1 <= k <= min(E, 8): other shapes return
+ *   MOE_ERR_INVALID_ARG (use the two separate calls).
  *   No workspace.
  */
-int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
-                       int k, int renormalize, int n_groups, int topk_groups, int dtype,
-                       float* logits, int32_t* topk_ids, float* topk_w,
+int moe_route_dispatch(const void* x, const void* W_gate, const float* bias,
+                       const void* w_gate_shared, int T, int H, int E, int k, int renormalize,
+                       int n_groups, int topk_groups, int dtype, float* logits,
+                       int32_t* topk_ids, float* topk_w, float* shared_gate_logit,
                        int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv_perm,
                        int32_t* packed_tok, float* packed_w, void* x_packed,
                        int32_t* counter, int32_t* status, void* stream);

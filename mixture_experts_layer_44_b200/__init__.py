@@ -72,8 +72,8 @@ _SIGS = {
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
-    "moe_route_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
-                                _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+                                _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_layer_workspace_bytes": (_SZ, [_P]),
     "moe_test_set_wait_budget_ns": (_I, [ctypes.c_ulonglong]),
     "moe_layer_create": (_I, [_P, _P, _SZ, _P, _P]),
@@ -170,23 +170,28 @@ def moe_route_grouped(x, W_gate, bias, k: int, renormalize: bool, n_groups: int,
         _stream(stream)))
 
 
-def route_dispatch_fits(T: int, H: int, E: int, k: int) -> bool:
-    """Shapes moe_route_dispatch takes (one launch for router + dispatcher)."""
-    return 1 <= T <= 64 and 1 <= E <= 64 and H <= 32768 and 1 <= k <= min(E, 8)
+def route_dispatch_fits(T: int, H: int, E: int, k: int, gate: bool = False) -> bool:
+    """Shapes moe_route_dispatch takes (one launch for router + dispatcher;
+    with a shared expert's gate row, E + 1 rows)."""
+    return 1 <= T <= 64 and 1 <= E and E + int(gate) <= 64 and H <= 32768 and 1 <= k <= min(E, 8)
 
 
 def moe_route_dispatch(x, W_gate, bias, k: int, renormalize: bool, logits, topk_ids, topk_w,
                        counts, offsets, perm, inv_perm, packed_tok, packed_w, x_packed, counter,
-                       status=None, stream=None, n_groups: int = 1, topk_groups: int = 1):
+                       status=None, stream=None, n_groups: int = 1, topk_groups: int = 1,
+                       w_gate_shared=None, shared_gate_logit=None):
     """moe_route_grouped then moe_dispatch in one launch (T <= 64, E <= 64).
-    ``counter``: one int32 on the device, zero before the first call."""
+    ``counter``: one int32 on the device, zero before the first call.  With
+    ``w_gate_shared`` [H] (a shared expert's gate row; E <= 63) the same launch
+    also writes x . w_gate_shared into ``shared_gate_logit`` [T] f32."""
     T, H = x.shape
     E = W_gate.shape[0]
     _check(load_library().moe_route_dispatch(
-        _ptr(x), _ptr(W_gate), _ptr(bias), T, H, E, k, int(bool(renormalize)), n_groups,
-        topk_groups, _dtype_code(x), _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _ptr(counts),
-        _ptr(offsets), _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w),
-        _ptr(x_packed), _ptr(counter), _ptr(status), _stream(stream)))
+        _ptr(x), _ptr(W_gate), _ptr(bias), _ptr(w_gate_shared), T, H, E, k,
+        int(bool(renormalize)), n_groups, topk_groups, _dtype_code(x), _ptr(logits),
+        _ptr(topk_ids), _ptr(topk_w), _ptr(shared_gate_logit), _ptr(counts), _ptr(offsets),
+        _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w), _ptr(x_packed),
+        _ptr(counter), _ptr(status), _stream(stream)))
 
 
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
@@ -465,7 +470,7 @@ class MoELayerBuffers:
                                                 else MOE_F32)), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, **i32)
         self.rd_counter = torch.zeros(1, **i32)    # ticket of moe_route_dispatch
-        self.route_dispatch = route_dispatch_fits(T, H, E, k)
+        self.route_dispatch = route_dispatch_fits(T, H, E, k, gate=shared_I is not None)
         self.shared_I = shared_I
         # bf16 tensor-core layers run the shared expert inside the routed launches
         self.fuse_shared = bool(shared_I) and dtype == torch.bfloat16 and H % 256 == 0 and \
@@ -478,17 +483,21 @@ class MoELayerBuffers:
 
 
 def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
-                       stream=None, n_groups: int = 1, topk_groups: int = 1):
+                       stream=None, n_groups: int = 1, topk_groups: int = 1) -> bool:
     """Router then dispatcher into ``buf``: one launch for decode batches
-    (moe_route_dispatch), else moe_route[_grouped] and moe_dispatch."""
+    (moe_route_dispatch, which then also writes a shared expert's gate logit
+    into ``buf.sg_logit``), else moe_route[_grouped] and moe_dispatch.
+    Returns whether the shared gate logit was written."""
     E = params["W_gate"].shape[0]
     if buf.route_dispatch:
+        w_sg = params.get("w_sg") if params.get("w13s") is not None else None
         moe_route_dispatch(x, params["W_gate"], params.get("bias"), k, renormalize, buf.logits,
                            buf.ids, buf.w, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                            buf.packed_tok, buf.packed_w, buf.x_packed, buf.rd_counter,
                            status=buf.status, stream=stream, n_groups=n_groups,
-                           topk_groups=topk_groups)
-        return
+                           topk_groups=topk_groups, w_gate_shared=w_sg,
+                           shared_gate_logit=buf.sg_logit if w_sg is not None else None)
+        return w_sg is not None
     if n_groups > 1:
         moe_route_grouped(x, params["W_gate"], params.get("bias"), k, renormalize, n_groups,
                           topk_groups, buf.logits, buf.ids, buf.w, status=buf.status,
@@ -498,6 +507,7 @@ def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayer
                   buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
+    return False
 
 
 def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
@@ -508,15 +518,15 @@ def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerB
     for a shared expert, w13s [2I_s,H], w2s [H,I_s], w_sg [H].  n_groups > 1
     routes group-limited (moe_route_grouped).
     """
-    E = params["W_gate"].shape[0]
-    route_and_dispatch(x, params, k, renormalize, buf, stream, n_groups, topk_groups)
+    gate_done = route_and_dispatch(x, params, k, renormalize, buf, stream, n_groups, topk_groups)
     shared = sg = None
     if params.get("w13s") is None:
         moe_experts(buf.x_packed, buf.offsets, buf.packed_w, params["w13"], params["w2"], buf.h,
                     buf.y_packed, ws=buf.ws_experts, status=buf.status, stream=stream)
     else:
-        moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
-                  status=buf.status, stream=stream)
+        if not gate_done:
+            moe_route(x, params["w_sg"].view(1, -1), None, 0, False, buf.sg_logit,
+                      status=buf.status, stream=stream)
         if buf.fuse_shared:
             moe_experts_shared(buf.x_packed, buf.offsets, buf.packed_w, params["w13"],
                                params["w2"], buf.h, buf.y_packed, x, params["w13s"],

@@ -91,7 +91,7 @@ cudaError_t launch_probe_wait_timeout(int32_t* status, int budget_us, cudaStream
 
 extern "C" {
 
-int moe_abi_version(void) { return 4; }
+int moe_abi_version(void) { return 5; }
 
 unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -192,9 +192,10 @@ int moe_dispatch(const int32_t* topk_ids, const float* topk_w, const void* x, in
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_dispatch launch");
 }
 
-int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int T, int H, int E,
-                       int k, int renormalize, int n_groups, int topk_groups, int dtype,
-                       float* logits, int32_t* topk_ids, float* topk_w, int32_t* counts,
+int moe_route_dispatch(const void* x, const void* W_gate, const float* bias,
+                       const void* w_gate_shared, int T, int H, int E, int k, int renormalize,
+                       int n_groups, int topk_groups, int dtype, float* logits,
+                       int32_t* topk_ids, float* topk_w, float* shared_gate_logit, int32_t* counts,
                        int32_t* offsets, int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
                        float* packed_w, void* x_packed, int32_t* counter, int32_t* status,
                        void* stream) {
@@ -205,8 +206,12 @@ int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int
       f + "null x, W_gate, logits, topk_ids or topk_w");
   REQ(counts && offsets && perm && inv_perm && packed_tok && packed_w && counter,
       MOE_ERR_INVALID_ARG, f + "null dispatch output or counter");
+  REQ((w_gate_shared == nullptr) == (shared_gate_logit == nullptr), MOE_ERR_INVALID_ARG,
+      f + "w_gate_shared and shared_gate_logit come together");
+  const int gate = w_gate_shared != nullptr ? 1 : 0;
   REQ(T >= 1 && T <= 64, MOE_ERR_INVALID_ARG, f + "T must be in [1, 64]");
-  REQ(E >= 1 && E <= 64, MOE_ERR_INVALID_ARG, f + "E must be in [1, 64]");
+  REQ(E >= 1 && E + gate <= 64, MOE_ERR_INVALID_ARG,
+      f + (gate ? "E must be in [1, 63] with a shared gate" : "E must be in [1, 64]"));
   REQ(H >= 8 && H % 8 == 0 && H <= 32768, MOE_ERR_INVALID_ARG,
       f + "H must be a multiple of 8 in [8, 32768]");
   REQ(k >= 1 && k <= E && k <= moe::kMaxTopK, MOE_ERR_INVALID_ARG,
@@ -220,16 +225,18 @@ int moe_route_dispatch(const void* x, const void* W_gate, const float* bias, int
     REQ(k <= topk_groups * (E / n_groups), MOE_ERR_INVALID_ARG,
         f + "k must be in [1, topk_groups * E / n_groups]");
   }
-  REQ(aligned16(x) && aligned16(W_gate) && aligned16(x_packed), MOE_ERR_INVALID_ARG,
-      f + "x, W_gate and x_packed must be 16-byte aligned");
+  REQ(aligned16(x) && aligned16(W_gate) && aligned16(x_packed) && aligned16(w_gate_shared),
+      MOE_ERR_INVALID_ARG, f + "x, W_gate, w_gate_shared and x_packed must be 16-byte aligned");
   REQ(aligned4(logits) && aligned4(topk_ids) && aligned4(topk_w) && aligned4(bias) &&
+          aligned4(shared_gate_logit) &&
           aligned4(counts) && aligned4(offsets) && aligned4(perm) && aligned4(inv_perm) &&
           aligned4(packed_tok) && aligned4(packed_w) && aligned4(counter) && aligned4(status),
       MOE_ERR_INVALID_ARG, f + "index arrays, bias, counter and status must be 4-byte aligned");
   cudaError_t e = moe_host::launch_route_dispatch(
       x, W_gate, bias, T, H, E, k, renormalize != 0, dtype, logits, topk_ids, topk_w, counts,
       offsets, perm, inv_perm, packed_tok, packed_w, x_packed, counter, status,
-      static_cast<cudaStream_t>(stream), n_groups, n_groups > 1 ? topk_groups : 1);
+      static_cast<cudaStream_t>(stream), n_groups, n_groups > 1 ? topk_groups : 1, w_gate_shared,
+      shared_gate_logit);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route_dispatch launch");
 }
 

@@ -118,15 +118,18 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
                          int32_t* ids, float* w, int32_t* status, cudaStream_t s,
                          int n_groups = 1, int topk_groups = 1);
 // Router and dispatcher in one launch (T <= 64, E <= 64, H <= 32768,
-// 1 <= k <= 8): route_dispatch_fits says whether a shape qualifies.
-bool route_dispatch_fits(int T, int H, int E, int k);
+// 1 <= k <= 8; with a shared expert's gate row wsg, E + 1 <= 64, and its
+// logit per token goes to sg): route_dispatch_fits says whether a shape
+// qualifies.
+bool route_dispatch_fits(int T, int H, int E, int k, bool gate = false);
 cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float* bias, int T,
                                   int H, int E, int k, int renormalize, int dtype, float* logits,
                                   int32_t* ids, float* w, int32_t* counts, int32_t* offsets,
                                   int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
                                   float* packed_w, void* x_packed, int32_t* counter,
                                   int32_t* status, cudaStream_t s, int n_groups = 1,
-                                  int topk_groups = 1);
+                                  int topk_groups = 1, const void* wsg = nullptr,
+                                  float* sg = nullptr);
 cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
                             int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
                             int32_t* status, cudaStream_t s, int n_groups, int topk_groups);

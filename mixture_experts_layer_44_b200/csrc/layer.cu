@@ -118,6 +118,12 @@ const char* check_desc(const moe_layer_desc* d) {
   if (d->E < 1 || d->E > moe::kMaxExperts) return "E must be in [1, 256]";
   if (d->k < 1 || d->k > d->E || d->k > moe::kMaxTopK) return "k must be in [1, min(E, 8)]";
   if (!d->W_gate || !d->w13 || !d->w2) return "null W_gate, w13 or w2";
+  {
+    auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    if (mis(d->W_gate) || mis(d->w13) || mis(d->w2) || mis(d->w13s) || mis(d->w2s) ||
+        mis(d->w_sg))
+      return "weights must be 16-byte aligned";
+  }
   if (d->dtype == MOE_BF16 && (d->H % 256 || d->I % 64))
     return "bf16 layers need H % 256 == 0 and I % 64 == 0";
   if (d->w13s != nullptr) {
@@ -136,13 +142,18 @@ cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
   const moe_layer_desc& d = L->d;
   const int ng = d.n_groups > 1 ? d.n_groups : 1;
   cudaError_t e;
-  if (moe_host::route_dispatch_fits(d.T, d.H, d.E, d.k)) {
-    // decode batches: router and dispatcher in one launch
+  const bool shared = d.w13s != nullptr;
+  bool gate_done = false;       // the shared expert's gate logit is written
+  if (moe_host::route_dispatch_fits(d.T, d.H, d.E, d.k, shared)) {
+    // decode batches: router (and the shared expert's gate) and dispatcher in one launch
     e = moe_host::launch_route_dispatch(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k,
                                         d.renormalize != 0, d.dtype, L->logits, L->ids, L->w,
                                         L->counts, L->offsets, L->perm, L->inv_perm,
                                         L->packed_tok, L->packed_w, L->x_packed, L->counter,
-                                        L->status, s, ng, d.topk_groups);
+                                        L->status, s, ng, d.topk_groups,
+                                        shared ? d.w_sg : nullptr,
+                                        shared ? L->sg_logit : nullptr);
+    gate_done = shared;
   } else {
     e = moe_host::launch_route(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k, d.renormalize != 0,
                                d.dtype, L->logits, L->ids, L->w, L->status, s, ng,
@@ -154,8 +165,7 @@ cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
   }
   if (e != cudaSuccess) return e;
   const char* why = "";
-  const bool shared = d.w13s != nullptr;
-  if (shared) {
+  if (shared && !gate_done) {
     e = moe_host::launch_route(x, d.w_sg, nullptr, d.T, d.H, 1, 0, 0, d.dtype, L->sg_logit,
                                nullptr, nullptr, L->status, s);
     if (e != cudaSuccess) return e;

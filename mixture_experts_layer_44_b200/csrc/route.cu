@@ -78,6 +78,9 @@ constexpr int NS = 512;   // threads per CTA of the small-batch router
 // dispatch (per-warp counts, scan, stable scatter, and the gather of the rows
 // when they total at most 128 KiB), then puts the counter back to zero for
 // the next launch.
+// With wsg (any launch of the small router), the shared expert's gate row is
+// contracted with x as one more expert, E: its logit goes to sg[t] (no bias)
+// and it takes no part in the top-k (diffulex.moe.layer, SharedExpertMLP).
 struct SmallDispatch {
   int32_t* counter;            // zero before the launch; zero again after it
   int32_t* counts;
@@ -90,6 +93,8 @@ struct SmallDispatch {
   int row_vecs;
   uint4* x_packed;
   int32_t* status;
+  const void* wsg;             // shared expert's gate row [H], or null
+  float* sg;                   // its logit per token [T]
 };
 
 constexpr int kFusedRounds = 1;                       // N <= 16 warps x 32 = 512
@@ -121,16 +126,19 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
   // (clamped to the slice's last vector) so that a whole batch is in flight
   // before the first FMA.
   uint4 wq[EPW][BATCH][Q];
+  const int Etot = E + (dd.wsg != nullptr ? 1 : 0);       // rows: experts, then the gate
   auto load_w = [&](int vb) {
 #pragma unroll
     for (int i = 0; i < EPW; ++i) {
-      const int e = min(group + GROUPS * i, E - 1);
+      const int e = min(group + GROUPS * i, Etot - 1);
+      const uint4* row = e < E ? wb + static_cast<size_t>(e) * nvec * Q
+                               : static_cast<const uint4*>(dd.wsg);
 #pragma unroll
       for (int j = 0; j < BATCH; ++j) {
         const int vc = min(vb + 32 * j, ve - 1);
 #pragma unroll
         for (int q = 0; q < Q; ++q)
-          wq[i][j][q] = moe::ld_nc_v4(wb + (static_cast<size_t>(e) * nvec + vc) * Q + q);
+          wq[i][j][q] = moe::ld_nc_v4(row + static_cast<size_t>(vc) * Q + q);
       }
     }
   };
@@ -204,6 +212,10 @@ __global__ void __launch_bounds__(NS) route_small_kernel(const void* xv,
         for (int sl = 0; sl < WPE; ++sl) s += part[ex][sl];
         s += bias ? bias[ex] : 0.f;
         logits[static_cast<size_t>(t) * E + ex] = s;
+      } else if (ex == E && dd.wsg != nullptr) {
+#pragma unroll
+        for (int sl = 0; sl < WPE; ++sl) s += part[ex][sl];
+        dd.sg[t] = s;
       }
       v[j] = live[j] ? s : -FLT_MAX;
     }
@@ -453,12 +465,13 @@ template <bool FUSED>
 cudaError_t launch_small(const void* x, const void* W, const float* b, int T, int H, int E, int k,
                          int renorm, bool bf, float* logits, int32_t* ids, float* w,
                          moe::GroupLimit gl, const SmallDispatch& dd, cudaStream_t s) {
-  if (E <= 1) return launch_small_ep<1, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
-  if (E <= 2) return launch_small_ep<2, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
-  if (E <= 4) return launch_small_ep<4, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
-  if (E <= 8) return launch_small_ep<8, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
-  if (E <= 16) return launch_small_ep<16, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
-  if (E <= 32) return launch_small_ep<32, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  const int Er = E + (dd.wsg != nullptr ? 1 : 0);      // rows contracted (experts, gate)
+  if (Er <= 1) return launch_small_ep<1, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (Er <= 2) return launch_small_ep<2, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (Er <= 4) return launch_small_ep<4, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (Er <= 8) return launch_small_ep<8, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (Er <= 16) return launch_small_ep<16, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
+  if (Er <= 32) return launch_small_ep<32, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
   return launch_small_ep<64, FUSED>(x, W, b, T, H, E, k, renorm, bf, logits, ids, w, gl, dd, s);
 }
 
@@ -485,9 +498,9 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
   return cudaErrorInvalidValue;
 }
 
-bool route_dispatch_fits(int T, int H, int E, int k) {
-  return T >= 1 && T <= 64 && E >= 1 && E <= 64 && H <= 32768 && k >= 1 && k <= moe::kMaxTopK &&
-         T * k <= (NS / 32) * 32 * kFusedRounds;
+bool route_dispatch_fits(int T, int H, int E, int k, bool gate) {
+  return T >= 1 && T <= 64 && E >= 1 && E + (gate ? 1 : 0) <= 64 && H <= 32768 && k >= 1 &&
+         k <= moe::kMaxTopK && T * k <= (NS / 32) * 32 * kFusedRounds;
 }
 
 cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float* bias, int T,
@@ -496,7 +509,7 @@ cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float
                                   int32_t* perm, int32_t* inv_perm, int32_t* packed_tok,
                                   float* packed_w, void* x_packed, int32_t* counter,
                                   int32_t* status, cudaStream_t s, int n_groups,
-                                  int topk_groups) {
+                                  int topk_groups, const void* wsg, float* sg) {
   const bool bf = dtype == MOE_BF16;
   const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
                            n_groups > 1 ? topk_groups : 1};
@@ -505,7 +518,7 @@ cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float
                            static_cast<size_t>(T) * k * row_bytes <= (static_cast<size_t>(128) << 10);
   const SmallDispatch dd{counter, counts, offsets, perm, inv_perm, packed_tok, packed_w,
                          fuse_gather ? static_cast<const uint4*>(x) : nullptr, row_bytes / 16,
-                         static_cast<uint4*>(x_packed), status};
+                         static_cast<uint4*>(x_packed), status, wsg, sg};
   cudaError_t e = launch_small<true>(x, W_gate, bias, T, H, E, k, renormalize, bf, logits, ids, w,
                                      gl, dd, s);
   if (e != cudaSuccess || x_packed == nullptr || fuse_gather) return e;

@@ -52,7 +52,7 @@ def test_library_is_built_for_sm100a_only():
 
 
 def test_abi_version_and_workspace_queries(lib):
-    assert M.moe_abi_version() == 4
+    assert M.moe_abi_version() == 5
     assert M.moe_launch_count() == 0     # nothing launched on a CPU-only host
     ws = M.moe_dispatch_workspace_bytes(16384, 8, 128)
     assert ws >= (16384 * 8 + 2047) // 2048 * 128 * 4
@@ -106,24 +106,28 @@ def test_dispatch_rejects_bad_arguments_on_the_host(lib):
 
 
 def test_route_dispatch_rejects_bad_arguments_on_the_host(lib):
-    # x, W, bias, T, H, E, k, renorm, G, Mg, dtype, logits, ids, w, counts, offsets, perm,
-    # inv_perm, packed_tok, packed_w, x_packed, counter, status, stream
-    args = [P, P, NULL, 4, 64, 8, 2, 1, 1, 1, M.MOE_BF16, P, P, P, P, P, P, P, P, P, P, P, NULL,
-            NULL]
-    a = list(args); a[3] = 65             # more tokens than the one-launch path takes
+    # x, W, bias, w_sg, T, H, E, k, renorm, G, Mg, dtype, logits, ids, w, sg_logit, counts,
+    # offsets, perm, inv_perm, packed_tok, packed_w, x_packed, counter, status, stream
+    args = [P, P, NULL, NULL, 4, 64, 8, 2, 1, 1, 1, M.MOE_BF16, P, P, P, NULL, P, P, P, P, P, P,
+            P, P, NULL, NULL]
+    a = list(args); a[4] = 65             # more tokens than the one-launch path takes
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "T must be" in _err(lib)
-    a = list(args); a[5] = 65; a[6] = 2   # more experts than it takes
+    a = list(args); a[6] = 65; a[7] = 2   # more experts than it takes
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "E must be" in _err(lib)
-    a = list(args); a[6] = 0              # it always dispatches: k >= 1
+    a = list(args); a[7] = 0              # it always dispatches: k >= 1
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "k must be" in _err(lib)
-    a = list(args); a[21] = NULL          # no ticket word
+    a = list(args); a[23] = NULL          # no ticket word
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "counter" in _err(lib)
-    a = list(args); a[8] = 3              # 3 groups do not divide 8 experts
+    a = list(args); a[9] = 3              # 3 groups do not divide 8 experts
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "n_groups" in _err(lib)
-    a = list(args); a[4] = 32776          # H above 32768
+    a = list(args); a[5] = 32776          # H above 32768
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "H must be" in _err(lib)
-    a = list(args); a[10] = 7
+    a = list(args); a[11] = 7
     assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG
+    a = list(args); a[3] = P              # a gate row without its logit output
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "shared_gate_logit" in _err(lib)
+    a = list(args); a[3] = P; a[15] = P; a[6] = 64   # 64 experts leave no row for the gate
+    assert lib.moe_route_dispatch(*a) == M.MOE_ERR_INVALID_ARG and "E must be" in _err(lib)
 
 
 def test_experts_rejects_bad_arguments_on_the_host(lib):

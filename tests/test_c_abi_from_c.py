@@ -19,7 +19,7 @@ PROGRAM = textwrap.dedent(r"""
 
     int main(void) {
       int fails = 0;
-      if (moe_abi_version() != 4) { puts("version"); ++fails; }
+      if (moe_abi_version() != 5) { puts("version"); ++fails; }
       if (moe_launch_count() != 0ull) { puts("launch count"); ++fails; }
       /* null x: rejected on the host before anything is enqueued */
       float logits[4];

@@ -74,7 +74,12 @@ def _check(cfg, seed, G=1, Mg=1, bias=True):
     assert int(g["status"][0]) == 0 and int(s["status"][0]) == 0
     for key in KEYS:
         assert _same_bits(g[key], s[key]), f"{key} differs from the two-call chain"
-    # and the oracle: routing from the GPU's logits, then its counting sort
+    _against_oracle(g, p, cfg, G, Mg, bias)
+    return g
+
+
+def _against_oracle(g, p, cfg, G=1, Mg=1, bias=True):
+    # routing from the GPU's logits, then the oracle's counting sort
     assert rel(g["logits"], O.router_logits(p["x"], p["W_gate"], p["bias"] if bias else None)) \
         <= 1e-5
     ids_o, w_o = O.route_from_logits(g["logits"], cfg.k, cfg.renormalize, G, Mg)
@@ -85,7 +90,6 @@ def _check(cfg, seed, G=1, Mg=1, bias=True):
         np.testing.assert_array_equal(g[key].numpy(), o[key], err_msg=key)
     np.testing.assert_array_equal(g["packed_w"].numpy(), g["w"].numpy().reshape(-1)[o["perm"]])
     assert _same_bits(g["x_packed"], p["x"][torch.as_tensor(o["packed_tok"])])
-    return g
 
 
 @pytest.mark.parametrize("T,H,E,k", [(1, 4096, 8, 2), (8, 4096, 8, 2), (3, 96, 1, 1),
@@ -128,3 +132,50 @@ def test_route_dispatch_rejects_large_shapes():
         M.moe_route_dispatch(x, W, None, 2, True, o["logits"], o["ids"], o["w"], o["counts"],
                              o["offsets"], o["perm"], o["inv_perm"], o["packed_tok"],
                              o["packed_w"], o["x_packed"], counter)
+
+
+@pytest.mark.parametrize("T,H,E,k,dtype", [(32, 2048, 60, 4, "bf16"), (1, 4096, 8, 2, "bf16"),
+                                           (5, 72, 3, 2, "f32"), (64, 256, 63, 8, "bf16"),
+                                           (17, 512, 15, 4, "f32")])
+def test_route_dispatch_with_the_shared_gate(T, H, E, k, dtype):
+    # the shared expert's gate row rides along as row E: the routed outputs
+    # match the oracle as without it (and are bit-identical to the launch
+    # without it when E + 1 rows keep the same power-of-two row block, so
+    # that every dot product is split into the same slices), and the gate
+    # logit is x . w_sg
+    cfg = LayerConfig("rdsg", T=T, H=H, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 2 == 0))
+    p = make_layer(cfg, seed=T + E)
+    x, W, b = dev(p["x"]), dev(p["W_gate"]), dev(p["bias"])
+    g = torch.Generator().manual_seed(E)
+    w_sg = (torch.randn(H, generator=g) / H ** 0.5).to(p["x"].dtype)
+    plain = _fused(x, W, b, k, cfg.renormalize)
+    o = _bufs(T, H, E, k, x.dtype)
+    sg = torch.full((T,), -7.0, device=DEV)
+    counter = torch.zeros(1, dtype=torch.int32, device=DEV)
+    M.moe_route_dispatch(x, W, b, k, cfg.renormalize, o["logits"], o["ids"], o["w"], o["counts"],
+                         o["offsets"], o["perm"], o["inv_perm"], o["packed_tok"], o["packed_w"],
+                         o["x_packed"], counter, status=o["status"], w_gate_shared=dev(w_sg),
+                         shared_gate_logit=sg)
+    torch.cuda.synchronize()
+    assert int(counter[0]) == 0 and int(o["status"][0]) == 0
+    gated = {key: v.cpu() for key, v in o.items()}
+    _against_oracle(gated, p, cfg)
+    pow2 = lambda n: 1 << max(0, (n - 1).bit_length())
+    if pow2(E + 1) == pow2(E):
+        for key in KEYS:
+            assert _same_bits(gated[key], plain[key]), f"{key} changed with the gate row"
+    ref = p["x"].double() @ w_sg.double()
+    assert rel(sg.cpu(), ref) <= 1e-5
+
+
+def test_route_dispatch_gate_needs_a_free_row():
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device=DEV)
+    W = torch.zeros(64, 64, dtype=torch.bfloat16, device=DEV)
+    o = _bufs(4, 64, 64, 2, torch.bfloat16)
+    counter = torch.zeros(1, dtype=torch.int32, device=DEV)
+    with pytest.raises(M.MoEError, match="E must be"):
+        M.moe_route_dispatch(x, W, None, 2, True, o["logits"], o["ids"], o["w"], o["counts"],
+                             o["offsets"], o["perm"], o["inv_perm"], o["packed_tok"],
+                             o["packed_w"], o["x_packed"], counter,
+                             w_gate_shared=torch.zeros(64, dtype=torch.bfloat16, device=DEV),
+                             shared_gate_logit=torch.zeros(4, device=DEV))
