@@ -384,6 +384,17 @@ class Layer:
             gate_done = M.route_and_dispatch(x, dp, cfg.k, cfg.renormalize, buf, stream)
             if ev:
                 ev[1].record(stream)
+        elif shared:
+            # the shared expert's gate logit comes out of the router's launch
+            M.moe_route_gated(x, dp["W_gate"], dp["bias"], dp["w_sg"], cfg.k, cfg.renormalize,
+                              buf.logits, buf.ids, buf.w, buf.sg_logit, status=buf.status,
+                              stream=stream)
+            gate_done = True
+            if ev:
+                ev[1].record(stream)
+            M.moe_dispatch(buf.ids, buf.w, x, cfg.E, buf.counts, buf.offsets, buf.perm,
+                           buf.inv_perm, buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws,
+                           buf.status, stream=stream)
         else:
             M.moe_route(x, dp["W_gate"], dp["bias"], cfg.k, cfg.renormalize, buf.logits,
                         buf.ids, buf.w, status=buf.status, stream=stream)

@@ -129,6 +129,29 @@ int moe_route_grouped(const void* x, const void* W_gate, const float* bias, int 
                       float* logits, int32_t* topk_ids, float* topk_w, int32_t* status,
                       void* stream);
 
+/*
+ * moe_route_gated -- moe_route_grouped plus the always-on shared expert's
+ * gate logit (diffulex.moe.layer, SharedExpertMLP: the sigmoid gate that
+ * scales the shared expert's output; moe_combine applies the sigmoid):
+ *   shared_gate_logit[t] = x[t] . w_gate_shared      (fp32 accumulate, no bias)
+ * The gate row is contracted in the router's own launch where the router has
+ * room for it -- small batches (T <= 64, E + 1 <= 64, H <= 32768) as row E,
+ * the bf16 tensor-core router (T > 64) by the warps that are otherwise idle
+ * during its main loop, from the x tiles already in shared memory -- else in
+ * a second launch (moe_route with E = 1, k = 0 on that row).  Either way x is
+ * read from HBM once per launch.  The routed outputs are those of
+ * moe_route_grouped; where the gate changes the router's row block (E + 1
+ * passing a power of two) their logits can differ from it in fp32 summation
+ * order.
+ *   w_gate_shared      device [H] (dtype), 16-byte aligned
+ *   shared_gate_logit  device [T] f32
+ *   All other arguments as moe_route_grouped (n_groups = 1: plain top-k).
+ */
+int moe_route_gated(const void* x, const void* W_gate, const float* bias,
+                    const void* w_gate_shared, int T, int H, int E, int k, int renormalize,
+                    int n_groups, int topk_groups, int dtype, float* logits, int32_t* topk_ids,
+                    float* topk_w, float* shared_gate_logit, int32_t* status, void* stream);
+
 /* Bytes of device scratch moe_dispatch needs for (T, k, E). */
 size_t moe_dispatch_workspace_bytes(int T, int k, int E);
 

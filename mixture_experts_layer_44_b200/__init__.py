@@ -27,7 +27,7 @@ __all__ = [
     "moe_experts", "moe_experts_shared", "moe_combine", "moe_read_status", "moe_probe_wait_timeout",
     "MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_UNSUPPORTED", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
     "MOE_ERR_BAD_INDEX", "MOE_ERR_OVERFLOW", "MOE_F32", "MOE_BF16", "MOE_F16", "MoELayerBuffers",
-    "moe_layer_forward", "moe_route_dispatch", "route_dispatch_fits", "route_and_dispatch",
+    "moe_layer_forward", "moe_route_dispatch", "moe_route_gated", "route_dispatch_fits", "route_and_dispatch",
     "moe_layer_forward_host", "moe_gather", "moe_combine_range", "moe_finalize",
     "moe_ep_partition_workspace_bytes", "moe_ep_partition", "moe_ep_owner", "moe_ep_pack_ids",
     "MoELayerDesc", "MoELayer", "moe_test_set_wait_budget_ns",
@@ -72,6 +72,8 @@ _SIGS = {
     "moe_probe_wait_timeout": (_I, [_P, _I, _P]),
     "moe_gather": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "moe_route_grouped": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "moe_route_gated": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                             _P]),
     "moe_route_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
                                 _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_layer_workspace_bytes": (_SZ, [_P]),
@@ -192,6 +194,20 @@ def moe_route_dispatch(x, W_gate, bias, k: int, renormalize: bool, logits, topk_
         _ptr(topk_ids), _ptr(topk_w), _ptr(shared_gate_logit), _ptr(counts), _ptr(offsets),
         _ptr(perm), _ptr(inv_perm), _ptr(packed_tok), _ptr(packed_w), _ptr(x_packed),
         _ptr(counter), _ptr(status), _stream(stream)))
+
+
+def moe_route_gated(x, W_gate, bias, w_gate_shared, k: int, renormalize: bool, logits,
+                    topk_ids, topk_w, shared_gate_logit, status=None, stream=None,
+                    n_groups: int = 1, topk_groups: int = 1):
+    """moe_route_grouped plus a shared expert's gate logit x . w_gate_shared
+    into ``shared_gate_logit`` [T] f32, in the router's own launch where it
+    has room for it."""
+    T, H = x.shape
+    E = W_gate.shape[0]
+    _check(load_library().moe_route_gated(
+        _ptr(x), _ptr(W_gate), _ptr(bias), _ptr(w_gate_shared), T, H, E, k,
+        int(bool(renormalize)), n_groups, topk_groups, _dtype_code(x), _ptr(logits),
+        _ptr(topk_ids), _ptr(topk_w), _ptr(shared_gate_logit), _ptr(status), _stream(stream)))
 
 
 def moe_dispatch_workspace_bytes(T: int, k: int, E: int) -> int:
@@ -485,9 +501,10 @@ class MoELayerBuffers:
 def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,
                        stream=None, n_groups: int = 1, topk_groups: int = 1) -> bool:
     """Router then dispatcher into ``buf``: one launch for decode batches
-    (moe_route_dispatch, which then also writes a shared expert's gate logit
-    into ``buf.sg_logit``), else moe_route[_grouped] and moe_dispatch.
-    Returns whether the shared gate logit was written."""
+    (moe_route_dispatch), else moe_route_gated / moe_route[_grouped] and
+    moe_dispatch.  With a shared expert (``params["w13s"]``) its gate logit
+    goes to ``buf.sg_logit`` in the router's launch.  Returns whether the
+    shared gate logit was written."""
     E = params["W_gate"].shape[0]
     if buf.route_dispatch:
         w_sg = params.get("w_sg") if params.get("w13s") is not None else None
@@ -498,7 +515,12 @@ def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayer
                            topk_groups=topk_groups, w_gate_shared=w_sg,
                            shared_gate_logit=buf.sg_logit if w_sg is not None else None)
         return w_sg is not None
-    if n_groups > 1:
+    gated = params.get("w13s") is not None
+    if gated:
+        moe_route_gated(x, params["W_gate"], params.get("bias"), params["w_sg"], k, renormalize,
+                        buf.logits, buf.ids, buf.w, buf.sg_logit, status=buf.status,
+                        stream=stream, n_groups=n_groups, topk_groups=topk_groups)
+    elif n_groups > 1:
         moe_route_grouped(x, params["W_gate"], params.get("bias"), k, renormalize, n_groups,
                           topk_groups, buf.logits, buf.ids, buf.w, status=buf.status,
                           stream=stream)
@@ -507,7 +529,7 @@ def route_and_dispatch(x, params: dict, k: int, renormalize: bool, buf: MoELayer
                   buf.w, status=buf.status, stream=stream)
     moe_dispatch(buf.ids, buf.w, x, E, buf.counts, buf.offsets, buf.perm, buf.inv_perm,
                  buf.packed_tok, buf.packed_w, buf.x_packed, buf.ws, buf.status, stream=stream)
-    return False
+    return gated
 
 
 def moe_layer_forward(x, params: dict, k: int, renormalize: bool, buf: MoELayerBuffers,

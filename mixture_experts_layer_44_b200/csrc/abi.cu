@@ -101,7 +101,8 @@ namespace {
 
 int route_impl(const char* fn, const void* x, const void* W_gate, const float* bias, int T,
                int H, int E, int k, int renormalize, int n_groups, int topk_groups, int dtype,
-               float* logits, int32_t* topk_ids, float* topk_w, int32_t* status, void* stream) {
+               float* logits, int32_t* topk_ids, float* topk_w, int32_t* status, void* stream,
+               const void* wsg = nullptr, float* sg = nullptr) {
   const std::string f = std::string(fn) + ": ";
   if (int r = check_dtype(dtype)) return r;
   REQ(x && W_gate && logits, MOE_ERR_INVALID_ARG, f + "null x, W_gate or logits");
@@ -126,10 +127,15 @@ int route_impl(const char* fn, const void* x, const void* W_gate, const float* b
     REQ(k >= 1 && k <= topk_groups * (E / n_groups), MOE_ERR_INVALID_ARG,
         f + "k must be in [1, topk_groups * E / n_groups]");
   }
-  cudaError_t e = moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
-                                         logits, topk_ids, topk_w, status,
+  cudaError_t e =
+      wsg != nullptr
+          ? moe_host::launch_route_gated(x, W_gate, bias, wsg, T, H, E, k, renormalize != 0,
+                                         dtype, logits, topk_ids, topk_w, sg, status,
                                          static_cast<cudaStream_t>(stream), n_groups,
-                                         topk_groups);
+                                         topk_groups)
+          : moe_host::launch_route(x, W_gate, bias, T, H, E, k, renormalize != 0, dtype,
+                                   logits, topk_ids, topk_w, status,
+                                   static_cast<cudaStream_t>(stream), n_groups, topk_groups);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, (f + "launch").c_str());
 }
 
@@ -151,6 +157,21 @@ int moe_route_grouped(const void* x, const void* W_gate, const float* bias, int 
   REQ(n_groups >= 1, MOE_ERR_INVALID_ARG, "moe_route_grouped: n_groups must be >= 1");
   return route_impl("moe_route_grouped", x, W_gate, bias, T, H, E, k, renormalize, n_groups,
                     topk_groups, dtype, logits, topk_ids, topk_w, status, stream);
+}
+
+int moe_route_gated(const void* x, const void* W_gate, const float* bias,
+                    const void* w_gate_shared, int T, int H, int E, int k, int renormalize,
+                    int n_groups, int topk_groups, int dtype, float* logits, int32_t* topk_ids,
+                    float* topk_w, float* shared_gate_logit, int32_t* status, void* stream) {
+  g_err.clear();
+  REQ(n_groups >= 1, MOE_ERR_INVALID_ARG, "moe_route_gated: n_groups must be >= 1");
+  REQ(w_gate_shared && shared_gate_logit, MOE_ERR_INVALID_ARG,
+      "moe_route_gated: null w_gate_shared or shared_gate_logit");
+  REQ(aligned16(w_gate_shared) && aligned4(shared_gate_logit), MOE_ERR_INVALID_ARG,
+      "moe_route_gated: w_gate_shared must be 16-byte and shared_gate_logit 4-byte aligned");
+  return route_impl("moe_route_gated", x, W_gate, bias, T, H, E, k, renormalize, n_groups,
+                    topk_groups, dtype, logits, topk_ids, topk_w, status, stream, w_gate_shared,
+                    shared_gate_logit);
 }
 
 size_t moe_dispatch_workspace_bytes(int T, int k, int E) {

@@ -117,6 +117,13 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
                          int E, int k, int renormalize, int dtype, float* logits,
                          int32_t* ids, float* w, int32_t* status, cudaStream_t s,
                          int n_groups = 1, int topk_groups = 1);
+// launch_route plus the shared expert's gate logit sg[t] = x[t] . wsg: in the
+// same launch where the router has room for it (small batches with E + 1 <=
+// 64; the bf16 tensor-core router), else a second launch.
+cudaError_t launch_route_gated(const void* x, const void* W_gate, const float* bias,
+                               const void* wsg, int T, int H, int E, int k, int renormalize,
+                               int dtype, float* logits, int32_t* ids, float* w, float* sg,
+                               int32_t* status, cudaStream_t s, int n_groups, int topk_groups);
 // Router and dispatcher in one launch (T <= 64, E <= 64, H <= 32768,
 // 1 <= k <= 8; with a shared expert's gate row wsg, E + 1 <= 64, and its
 // logit per token goes to sg): route_dispatch_fits says whether a shape
@@ -130,9 +137,13 @@ cudaError_t launch_route_dispatch(const void* x, const void* W_gate, const float
                                   int32_t* status, cudaStream_t s, int n_groups = 1,
                                   int topk_groups = 1, const void* wsg = nullptr,
                                   float* sg = nullptr);
+// With wsg (bf16 [H]) the shared expert's gate logit x . wsg goes to sg [T] in
+// the same launch; cudaErrorNotSupported when a CTA's slice of H is too long
+// to stage it.
 cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
                             int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
-                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups);
+                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups,
+                            const void* wsg = nullptr, float* sg = nullptr);
 size_t dispatch_ws_bytes(int T, int k, int E);
 cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, int T, int H,
                             int E, int k, int dtype, int32_t* counts, int32_t* offsets,

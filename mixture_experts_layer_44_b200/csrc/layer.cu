@@ -155,9 +155,14 @@ cudaError_t run_layer(moe_layer* L, const void* x, void* out, cudaStream_t s) {
                                         shared ? L->sg_logit : nullptr);
     gate_done = shared;
   } else {
-    e = moe_host::launch_route(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k, d.renormalize != 0,
-                               d.dtype, L->logits, L->ids, L->w, L->status, s, ng,
-                               d.topk_groups);
+    e = shared ? moe_host::launch_route_gated(x, d.W_gate, d.bias, d.w_sg, d.T, d.H, d.E, d.k,
+                                              d.renormalize != 0, d.dtype, L->logits, L->ids,
+                                              L->w, L->sg_logit, L->status, s, ng,
+                                              d.topk_groups)
+               : moe_host::launch_route(x, d.W_gate, d.bias, d.T, d.H, d.E, d.k,
+                                        d.renormalize != 0, d.dtype, L->logits, L->ids, L->w,
+                                        L->status, s, ng, d.topk_groups);
+    gate_done = shared;
     if (e == cudaSuccess)
       e = moe_host::launch_dispatch(L->ids, L->w, x, d.T, d.H, d.E, d.k, d.dtype, L->counts,
                                     L->offsets, L->perm, L->inv_perm, L->packed_tok,

@@ -498,6 +498,33 @@ cudaError_t launch_route(const void* x, const void* W_gate, const float* bias, i
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_route_gated(const void* x, const void* W_gate, const float* bias,
+                               const void* wsg, int T, int H, int E, int k, int renormalize,
+                               int dtype, float* logits, int32_t* ids, float* w, float* sg,
+                               int32_t* status, cudaStream_t s, int n_groups, int topk_groups) {
+  const bool bf = dtype == MOE_BF16;
+  const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
+                           n_groups > 1 ? topk_groups : 1};
+  const bool small = T <= 64 && E <= 64 && H <= 32768;   // launch_route's choice
+  if (small && E + 1 <= 64) {
+    SmallDispatch dd{};
+    dd.wsg = wsg;
+    dd.sg = sg;
+    return launch_small<false>(x, W_gate, bias, T, H, E, k, renormalize, bf, logits, ids, w, gl,
+                               dd, s);
+  }
+  if (bf && !small) {
+    const cudaError_t e = launch_route_tc(x, W_gate, bias, T, H, E, k, renormalize, logits, ids,
+                                          w, status, s, n_groups, topk_groups, wsg, sg);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  // two launches: the routed router, then the gate as one expert with no selection
+  cudaError_t e = launch_route(x, W_gate, bias, T, H, E, k, renormalize, dtype, logits, ids, w,
+                               status, s, n_groups, topk_groups);
+  if (e != cudaSuccess) return e;
+  return launch_route(x, wsg, nullptr, T, H, 1, 0, 0, dtype, sg, nullptr, nullptr, status, s);
+}
+
 bool route_dispatch_fits(int T, int H, int E, int k, bool gate) {
   return T >= 1 && T <= 64 && E >= 1 && E + (gate ? 1 : 0) <= 64 && H <= 32768 && k >= 1 &&
          k <= moe::kMaxTopK && T * k <= (NS / 32) * 32 * kFusedRounds;

@@ -25,6 +25,16 @@
 // CTA = 8 warps: one lane of warp 0 issues the TMA loads, one lane of warp 1
 // owns TMEM and issues the MMAs; then all 8 warps read the accumulators
 // (warp w: TMEM lanes 32*(w%4) .. +31, column half w/4) and finalise tokens.
+// With a shared expert's gate row (wsg, bf16 [H]; diffulex.moe.layer,
+// SharedExpertMLP) its logit x . wsg is contracted in the same launch: the
+// CTA's slice of wsg is staged in shared memory, warps 2-5 (one thread per
+// token row, idle otherwise until the epilogue) read each stage's x tile
+// after the TMA lands it and add 64 products per row in fp32, and the stage
+// is released only once they and the MMAs are done with it.  Each CTA's
+// partial goes into column E of its partial tile (a padding column: E <
+// EPAD), so the cluster sums it with the logits; it takes no part in the
+// selection and goes to sg[t] without bias.
+//
 // Every wait is bounded; one that runs out reports MOE_ERR_TIMEOUT in the
 // status word and the CTA still takes part in both cluster barriers, so its
 // peers finish too.  The stage-ring waits are bounded by `wait_ns` (a test
@@ -50,6 +60,7 @@ constexpr int RNT = 256;                  // threads per CTA
 constexpr int RMAX_S = 8;                 // CTAs per cluster (portable limit)
 constexpr int RMAX_STAGES = 8;
 constexpr size_t RSTAGE_BUDGET = 144 * 1024;   // pipeline bytes: one CTA per SM
+constexpr int RGATE_KB = 256;             // k-blocks of wsg a CTA can stage (32 KB)
 
 template <int EPAD>
 struct RCfg {
@@ -72,11 +83,13 @@ struct RCtl {
   uint64_t accf;          // all MMAs of this CTA have completed
   uint32_t tmem_base;
   int abort;
+  int gstop;              // the gate warps stop (their waiting thread timed out)
 };
 
 template <int EPAD>
-constexpr size_t smem_bytes() {
-  return 1024 + RCfg<EPAD>::BUF_BYTES + (sizeof(RCtl) + 127) / 128 * 128;
+constexpr size_t smem_bytes(bool gate) {
+  return 1024 + RCfg<EPAD>::BUF_BYTES + (sizeof(RCtl) + 127) / 128 * 128 +
+         (gate ? static_cast<size_t>(RGATE_KB) * RBK * 2 : 0);
 }
 
 __device__ __forceinline__ void set_abort(RCtl& c, int32_t* status) {
@@ -90,13 +103,18 @@ __global__ void __launch_bounds__(RNT, 1)
                     const __grid_constant__ CUtensorMap tmW, const float* __restrict__ bias,
                     int T, int E, int k, int renorm, int kblocks, float* __restrict__ logits,
                     int32_t* __restrict__ ids, float* __restrict__ wout, int32_t* status,
-                    moe::GroupLimit gl, uint64_t wait_ns) {
+                    moe::GroupLimit gl, uint64_t wait_ns, const __nv_bfloat16* wsg,
+                    float* __restrict__ sg, int H) {
   using C = RCfg<EPAD>;
   constexpr int LS = C::LS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   RCtl& c = *reinterpret_cast<RCtl*>(smem + C::BUF_BYTES);
+  // the staged slice of the gate row (gate only)
+  __nv_bfloat16* g_s = reinterpret_cast<__nv_bfloat16*>(
+      smem + C::BUF_BYTES + (sizeof(RCtl) + 127) / 128 * 128);
+  const bool gate = wsg != nullptr;
   float* l_s = reinterpret_cast<float*>(smem);   // after the main loop: [RBM][LS] partial logits
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -112,7 +130,7 @@ __global__ void __launch_bounds__(RNT, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       moe::mbar_init(moe::smem_addr(&c.full[s]), 1);
-      moe::mbar_init(moe::smem_addr(&c.empty[s]), 1);
+      moe::mbar_init(moe::smem_addr(&c.empty[s]), gate ? 2 : 1);   // MMAs (+ gate warps)
     }
     moe::mbar_init(moe::smem_addr(&c.accf), 1);
     c.abort = 0;
@@ -123,6 +141,14 @@ __global__ void __launch_bounds__(RNT, 1)
   if (warp == 1) {
     moe::tmem_alloc(moe::smem_addr(&c.tmem_base), C::TMEM_COLS);
     moe::tmem_relinquish();
+  }
+  if (gate && warp >= 2 && warp < 6) {
+    // wsg is a weight (never the previous kernel's output): staged before the wait
+    // (columns past H, in a last partial k-block, stay zero like the x tile's)
+    const uint4* src = reinterpret_cast<const uint4*>(wsg + static_cast<size_t>(kb0) * RBK);
+    uint4* dst = reinterpret_cast<uint4*>(g_s);
+    for (int i = threadIdx.x - 64; i < nkb * RBK / 8; i += 128)
+      dst[i] = kb0 * RBK + i * 8 < H ? moe::ld_nc_v4(src + i) : make_uint4(0, 0, 0, 0);
   }
   moe::grid_dep_wait();        // x may be the previous kernel's output
   moe::tc_fence_before();
@@ -180,6 +206,42 @@ __global__ void __launch_bounds__(RNT, 1)
     }
     moe::tc_commit(moe::smem_addr(&c.accf));   // arrives once every MMA above has completed
   }
+  // Gate: thread r of warps 2-5 adds row r of every landed x tile times the
+  // staged wsg block (chunk j of row r sits at j ^ (r & 7): the 128-byte swizzle).
+  float gacc = 0.f;
+  if (gate && warp >= 2 && warp < 6) {
+    const int r = threadIdx.x - 64;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int i = 0; i < nkb; ++i) {
+      // one thread waits (bounded) and tells the others through the named
+      // barrier, so that all 128 leave the loop together
+      if (r == 0) {
+        const bool landed = moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase, wait_ns);
+        if (!landed) set_abort(c, status);
+        *reinterpret_cast<volatile int*>(&c.gstop) = landed ? 0 : 1;
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+      if (*reinterpret_cast<volatile int*>(&c.gstop) != 0) break;
+      moe::mbar_wait(moe::smem_addr(&c.full[stage]), phase, wait_ns);   // completed: returns
+      const uint4* xr = reinterpret_cast<const uint4*>(smem + stage * C::STAGE_BYTES + r * 128);
+      const uint4* wr = reinterpret_cast<const uint4*>(g_s + i * RBK);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float xf[8], wf[8];
+        moe::unpack8(xr[j ^ (r & 7)], xf);
+        moe::unpack8(wr[j], wf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gacc = fmaf(xf[e], wf[e], gacc);
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");   // the four gate warps have read it
+      if (r == 0) moe::mbar_arrive(moe::smem_addr(&c.empty[stage]));
+      if (++stage == C::STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
   __syncwarp();
 
   // ------------------------------------------- partial logits of this slice ---
@@ -220,6 +282,10 @@ __global__ void __launch_bounds__(RNT, 1)
         l_s[row * LS + c0] = 0.f;
     }
   }
+  if (gate) {
+    __syncthreads();                               // the tile's column E is written
+    if (warp >= 2 && warp < 6) l_s[(threadIdx.x - 64) * LS + E] = ok ? gacc : 0.f;
+  }
   moe::grid_dep_launch();
   moe::tc_fence_before();
   cluster.sync();
@@ -236,11 +302,12 @@ __global__ void __launch_bounds__(RNT, 1)
   const int tl_begin = rank * per_cta;
   const int tl_end = min(min(RBM, tl_begin + per_cta), T - t0);
   float bl[PER];
-  bool live[PER];
+  bool live[PER], gcol[PER];
 #pragma unroll
   for (int j = 0; j < PER; ++j) {
     const int e = lane + 32 * j;
     live[j] = e < E;
+    gcol[j] = gate && e == E;                      // the shared gate's column
     bl[j] = (bias != nullptr && live[j]) ? bias[e] : 0.f;
   }
   for (int tl = tl_begin + warp; tl < tl_end; tl += 2 * NW) {
@@ -259,7 +326,7 @@ __global__ void __launch_bounds__(RNT, 1)
         for (int n = 0; n < 2; ++n)
 #pragma unroll
           for (int j = 0; j < PER; ++j)
-            v[n][j] += live[j] ? rl[rows[n] * LS + lane + 32 * j] : 0.f;
+            v[n][j] += (live[j] || gcol[j]) ? rl[rows[n] * LS + lane + 32 * j] : 0.f;
       }
     }
 #pragma unroll
@@ -267,6 +334,7 @@ __global__ void __launch_bounds__(RNT, 1)
       const size_t t = static_cast<size_t>(t0 + rows[n]);
 #pragma unroll
       for (int j = 0; j < PER; ++j) {
+        if (gcol[j] && (n == 0 || has_b)) sg[t] = v[n][j];
         v[n][j] += bl[j];
         if (live[j] && (n == 0 || has_b)) logits[t * E + lane + 32 * j] = v[n][j];
       }
@@ -285,9 +353,9 @@ __global__ void __launch_bounds__(RNT, 1)
 template <int EPAD>
 cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H, int E, int k,
                      int renorm, float* logits, int32_t* ids, float* w, int32_t* status,
-                     moe::GroupLimit gl, cudaStream_t s) {
+                     moe::GroupLimit gl, cudaStream_t s, const void* wsg, float* sg) {
   auto fn = route_tc_kernel<EPAD>;
-  constexpr size_t smem = smem_bytes<EPAD>();
+  const size_t smem = smem_bytes<EPAD>(wsg != nullptr);
   cudaError_t err = moe_host::ensure_smem(reinterpret_cast<const void*>(fn), (int)smem);
   if (err != cudaSuccess) return err;
   CUtensorMap mx, mw;
@@ -308,9 +376,11 @@ cudaError_t launch_t(const void* x, const void* W, const float* b, int T, int H,
   // One wave: as many H-slices per tile as the SMs allow, at least one block each.
   int S = moe_host::num_sms() / tiles;
   S = std::max(1, std::min({S, RMAX_S, kblocks}));
+  if (wsg != nullptr && (kblocks + S - 1) / S > RGATE_KB) return cudaErrorNotSupported;
   return moe_host::launch_pdl(fn, dim3(S * tiles, 1, 1), dim3(RNT, 1, 1), smem, s, S, mx, mw, b,
                               T, E, k, renorm, kblocks, logits, ids, w, status, gl,
-                              moe_host::main_wait_budget_ns());
+                              moe_host::main_wait_budget_ns(),
+                              static_cast<const __nv_bfloat16*>(wsg), sg, H);
 }
 
 }  // namespace
@@ -319,14 +389,16 @@ namespace moe_host {
 
 cudaError_t launch_route_tc(const void* x, const void* W_gate, const float* bias, int T, int H,
                             int E, int k, int renormalize, float* logits, int32_t* ids, float* w,
-                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups) {
+                            int32_t* status, cudaStream_t s, int n_groups, int topk_groups,
+                            const void* wsg, float* sg) {
   const moe::GroupLimit gl{n_groups > 1 ? E / n_groups : E, n_groups > 1 ? n_groups : 1,
                            n_groups > 1 ? topk_groups : 1};
-  if (E <= 32) return launch_t<32>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
-  if (E <= 64) return launch_t<64>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
-  if (E <= 128) return launch_t<128>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
-  if (E <= 256) return launch_t<256>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s);
-  return cudaErrorInvalidValue;
+  const int Er = E + (wsg != nullptr ? 1 : 0);   // the gate takes column E (a padding column)
+  if (Er <= 32) return launch_t<32>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s, wsg, sg);
+  if (Er <= 64) return launch_t<64>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s, wsg, sg);
+  if (Er <= 128) return launch_t<128>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s, wsg, sg);
+  if (Er <= 256) return launch_t<256>(x, W_gate, bias, T, H, E, k, renormalize, logits, ids, w, status, gl, s, wsg, sg);
+  return cudaErrorNotSupported;
 }
 
 }  // namespace moe_host

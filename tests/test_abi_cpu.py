@@ -31,7 +31,8 @@ def test_header_declares_the_stage_calls():
     names = _declared()
     for n in ("moe_route", "moe_dispatch", "moe_experts", "moe_experts_shared", "moe_combine",
               "moe_dispatch_workspace_bytes", "moe_experts_workspace_bytes", "moe_read_status",
-              "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version", "moe_launch_count"):
+              "moe_probe_wait_timeout", "moe_last_error", "moe_abi_version", "moe_launch_count",
+              "moe_route_gated"):
         assert n in names
 
 
@@ -247,3 +248,16 @@ def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
     # the testing hook's bounds
     assert lib.moe_test_set_wait_budget_ns(10) == M.MOE_ERR_INVALID_ARG
     assert lib.moe_test_set_wait_budget_ns(0) == M.MOE_OK
+
+
+def test_route_gated_rejects_bad_arguments_on_the_host(lib):
+    # x, W, bias, w_sg, T, H, E, k, renorm, G, Mg, dtype, logits, ids, w, sg_logit, status, stream
+    args = [P, P, NULL, P, 4, 64, 8, 2, 1, 1, 1, M.MOE_BF16, P, P, P, P, NULL, NULL]
+    a = list(args); a[3] = NULL           # no gate row
+    assert lib.moe_route_gated(*a) == M.MOE_ERR_INVALID_ARG and "w_gate_shared" in _err(lib)
+    a = list(args); a[15] = NULL          # nowhere to put its logit
+    assert lib.moe_route_gated(*a) == M.MOE_ERR_INVALID_ARG and "shared_gate_logit" in _err(lib)
+    a = list(args); a[3] = ctypes.c_void_p(24)   # gate row not 16-byte aligned
+    assert lib.moe_route_gated(*a) == M.MOE_ERR_INVALID_ARG and "aligned" in _err(lib)
+    a = list(args); a[9] = 3              # the routed part's checks apply as well
+    assert lib.moe_route_gated(*a) == M.MOE_ERR_INVALID_ARG and "n_groups" in _err(lib)

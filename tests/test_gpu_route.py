@@ -222,3 +222,49 @@ def test_grouped_routing_through_the_whole_layer():
     want = O.moe_forward_tokens(p, np.arange(cfg.T), ids, w64)
     from tests.gpu_util import err_bf16_out
     assert err_bf16_out(out.cpu(), want) <= 2e-2
+
+
+# moe_route_gated: the shared expert's gate logit x . w_sg in the router's own
+# launch (row E of the small router; the idle warps of the tensor-core router,
+# from the staged x tiles), or a second launch (fp32 above 64 tokens).  The
+# routed outputs meet the oracle as moe_route's do (and are bit-identical to
+# moe_route's where the gate leaves the router's row block unchanged); the
+# gate logit is within 1e-5 of x . w_sg in fp64.
+def _pow2(n):
+    return 1 << max(0, (n - 1).bit_length())
+
+
+@pytest.mark.parametrize("T,H,E,k,dtype", [
+    (32, 2048, 60, 4, "bf16"),      # small router, row block 64 either way
+    (8192, 2048, 60, 4, "bf16"),    # Qwen1.5 prefill: tensor-core router, column E of 64
+    (300, 200, 64, 2, "bf16"),      # E + 1 = 65: a wider block; H ends in a partial k-block
+    (131, 96, 8, 2, "bf16"),        # E = 8: 32 columns either way
+    (257, 4096, 255, 8, "bf16"),    # the last padding column of the 256-column block
+    (200, 96, 60, 4, "f32"),        # fp32 above 64 tokens: a second launch
+    (7, 72, 3, 2, "f32"),
+])
+def test_route_gated(T, H, E, k, dtype):
+    cfg = LayerConfig("rg", T=T, H=H, E=E, k=k, I=8, dtype=dtype, renormalize=(E % 2 == 0))
+    p = make_layer(cfg, seed=T + E)
+    g = torch.Generator().manual_seed(H)
+    w_sg = (torch.randn(H, generator=g) / H ** 0.5).to(p["x"].dtype)
+    logits = torch.empty(T, E, device=DEV)
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, device=DEV)
+    sg = torch.full((T,), -7.0, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    M.moe_route_gated(dev(p["x"]), dev(p["W_gate"]), None, dev(w_sg), k, cfg.renormalize, logits,
+                      ids, w, sg, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    logits, ids, w, sg = logits.cpu(), ids.cpu(), w.cpu(), sg.cpu()
+    assert rel(logits, O.router_logits(p["x"], p["W_gate"], None)) <= 1e-5
+    ids_o, w_o = O.route_from_logits(logits, k, cfg.renormalize)
+    np.testing.assert_array_equal(ids.numpy(), ids_o)
+    np.testing.assert_allclose(w.numpy(), w_o, rtol=1e-5, atol=0)
+    assert rel(sg, p["x"].double() @ w_sg.double()) <= 1e-5
+    same_block = (_pow2(E + 1) == _pow2(E)) if T <= 64 else \
+        (max(32, _pow2(E + 1)) == max(32, _pow2(E)))
+    if same_block and not (dtype == "f32" and T > 64):
+        l2, i2, w2 = _run(p["x"], p["W_gate"], None, k, cfg.renormalize)
+        assert torch.equal(logits, l2) and torch.equal(ids, i2) and torch.equal(w, w2)
