@@ -268,3 +268,31 @@ def test_route_gated(T, H, E, k, dtype):
     if same_block and not (dtype == "f32" and T > 64):
         l2, i2, w2 = _run(p["x"], p["W_gate"], None, k, cfg.renormalize)
         assert torch.equal(logits, l2) and torch.equal(ids, i2) and torch.equal(w, w2)
+
+
+def test_route_gated_random_shapes():
+    # seeded random shapes over both launches the gate rides in (T <= 64 small
+    # router, tensor-core router above), H tails included
+    rng = np.random.default_rng(11)
+    for _ in range(24):
+        T = int(rng.choice([1, 5, 33, 64, 65, 129, 257, 1000]))
+        E = int(rng.integers(1, 256))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        H = 8 * int(rng.integers(1, 257))
+        cfg = LayerConfig("rgr", T=T, H=H, E=E, k=k, I=8, dtype="bf16", renormalize=True)
+        p = make_layer(cfg, seed=T * 1000 + E)
+        w_sg = (torch.randn(H, generator=torch.Generator().manual_seed(H)) / H ** 0.5).to(
+            torch.bfloat16)
+        logits = torch.empty(T, E, device=DEV)
+        ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+        w = torch.empty(T, k, device=DEV)
+        sg = torch.full((T,), -7.0, device=DEV)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        M.moe_route_gated(dev(p["x"]), dev(p["W_gate"]), None, dev(w_sg), k, True, logits, ids,
+                          w, sg, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0, (T, E, k, H)
+        assert rel(logits.cpu(), O.router_logits(p["x"], p["W_gate"], None)) <= 1e-5, (T, E, H)
+        ids_o, _ = O.route_from_logits(logits.cpu(), k, True)
+        np.testing.assert_array_equal(ids.cpu().numpy(), ids_o)
+        assert rel(sg.cpu(), p["x"].double() @ w_sg.double()) <= 1e-5, (T, E, k, H)
