@@ -9,17 +9,18 @@
 // Small batches (N <= 2048 assignments) take one CTA of 32 warps through
 // count, scan and scatter in a single launch (the same warp-slice algorithm
 // as below), and also gather the rows when they total at most 128 KiB
-// (decode); larger gathers use the bulk-copy kernel.  Larger N takes four launches:
+// (decode); larger gathers use the bulk-copy kernel.  Larger N takes three launches:
 //   count   -- each CTA owns 1024 (N <= 65536) or 2048 consecutive
 //              assignments; each warp owns a contiguous eighth of them and
 //              counts it per expert with
 //              __match_any_sync (one shared-memory add per distinct expert
 //              in a 32-lane round, no atomics); CTA totals go to ws[b][e].
-//   scan    -- one CTA: counts[e] = sum_b ws[b][e], offsets = exclusive scan
-//              over e, and ws[b][e] becomes the first position CTA b writes
-//              for expert e.
-//   scatter -- each CTA recounts its slice per warp, turns the counts into
-//              per-warp bases, and walks its assignments in order; inside a
+//   scatter -- each CTA reads the whole table: counts[e] = sum_b ws[b][e],
+//              offsets = their exclusive scan over e (written by CTA 0), and
+//              its own first position for expert e, offsets[e] +
+//              sum_{b' < b} ws[b'][e]; it recounts its slice per warp, turns
+//              the counts into per-warp bases, and walks its assignments in
+//              order; inside a
 //              round a lane's rank among equal experts is the popcount of
 //              the lower lanes in its match mask.  Positions therefore grow
 //              with f inside an expert: the order is stable (bit-exact).
@@ -106,60 +107,35 @@ __global__ void __launch_bounds__(DNT) dispatch_count_kernel(const int32_t* ids,
   moe::grid_dep_launch();
 }
 
-// One CTA of 256 threads (E <= 256).
-__global__ void __launch_bounds__(256) dispatch_scan_kernel(int32_t* __restrict__ bc, int B,
-                                                            int E, int32_t* __restrict__ counts,
-                                                            int32_t* __restrict__ offsets) {
-  __shared__ int s_scan[256];
-  const int e = threadIdx.x;
-  moe::grid_dep_wait();
-  // The column of CTA counts is read in batches of 16 loads in flight.
-  constexpr int BATCH = 16;
-  int total = 0;
-  if (e < E)
-    for (int b0 = 0; b0 < B; b0 += BATCH) {
-      int c[BATCH];
+// Exclusive prefix of v over the 256 threads of the CTA (a shuffle scan in
+// each warp, then the warp totals); *total gets the sum.  tmp: shared [8].
+__device__ __forceinline__ int cta_excl_scan(int v, int* tmp, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int incl = v;
 #pragma unroll
-      for (int j = 0; j < BATCH; ++j)
-        c[j] = b0 + j < B ? moe::ld_prod(bc + static_cast<size_t>(b0 + j) * E + e) : 0;
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j) total += c[j];
-    }
-  // Exclusive scan over experts (Hillis-Steele on 256 entries).
-  s_scan[e] = total;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) tmp[warp] = incl;
   __syncthreads();
-  for (int o = 1; o < 256; o <<= 1) {
-    const int v = e >= o ? s_scan[e - o] : 0;
-    __syncthreads();
-    s_scan[e] += v;
-    __syncthreads();
-  }
-  const int excl = s_scan[e] - total;
-  if (e < E) {
-    counts[e] = total;
-    offsets[e] = excl;
-    int run = excl;
-    for (int b0 = 0; b0 < B; b0 += BATCH) {
-      int c[BATCH];
+  int before = 0, all = 0;
 #pragma unroll
-      for (int j = 0; j < BATCH; ++j)
-        c[j] = b0 + j < B ? moe::ld_prod(bc + static_cast<size_t>(b0 + j) * E + e) : 0;
-#pragma unroll
-      for (int j = 0; j < BATCH; ++j)
-        if (b0 + j < B) {
-          bc[static_cast<size_t>(b0 + j) * E + e] = run;
-          run += c[j];
-        }
-    }
+  for (int ww = 0; ww < DNT / 32; ++ww) {
+    const int t = tmp[ww];
+    if (ww < warp) before += t;
+    all += t;
   }
-  if (e == 255) offsets[E] = s_scan[255];
-  moe::grid_dep_launch();
+  __syncthreads();                 // tmp may be reused
+  *total = all;
+  return before + incl - v;
 }
 
 template <int CH>
 __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     const int32_t* ids, const float* w, int N, int E, int k,
-    const int32_t* bc, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+    const int32_t* bc, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
     int32_t* __restrict__ packed_tok, float* __restrict__ packed_w, int32_t* status) {
   extern __shared__ int wc[];  // [DWARPS][E] counts, then bases
   // The CTA's assignments in local expert-major order (position, f, weight),
@@ -170,7 +146,7 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
   __shared__ int s_pos[CH], s_f[CH];
   __shared__ float s_w[CH];
   __shared__ int s_shift[moe::kMaxExperts];   // local index - position, per expert
-  __shared__ int s_scan[DNT];
+  __shared__ int s_tmp[DNT / 32];
   const int base = blockIdx.x * CH;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int w0 = base + warp * PER_WARP;
@@ -182,11 +158,41 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     const int f = w0 + 32 * i + lane;
     wv[i] = packed_w != nullptr && f < N ? moe::ld_prod(w + f) : 0.f;
   }
-  // Per-warp global bases, and the CTA's total per expert (E <= DNT).
-  int total = 0, gbase = 0;
+  // Every CTA's count of expert e (the count kernel's table, E <= DNT): the
+  // expert's total and the part of the CTAs before this one, 16 loads in
+  // flight.  Each CTA scans the totals over the experts itself (the offsets;
+  // CTA 0 writes counts and offsets), so no launch sits between the count
+  // and scatter kernels.
   const int e = threadIdx.x;
+  const int B = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  int etot = 0, before = 0;
   if (e < E) {
-    gbase = moe::ld_prod(bc + static_cast<size_t>(blockIdx.x) * E + e);
+    constexpr int BATCH = 16;
+    for (int b0 = 0; b0 < B; b0 += BATCH) {
+      int c[BATCH];
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j)
+        c[j] = b0 + j < B ? moe::ld_prod(bc + static_cast<size_t>(b0 + j) * E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j) {
+        etot += c[j];
+        if (b0 + j < b) before += c[j];
+      }
+    }
+  }
+  int grand = 0;
+  const int eoff = cta_excl_scan(etot, s_tmp, &grand);
+  if (b == 0) {
+    if (e < E) {
+      counts[e] = etot;
+      offsets[e] = eoff;
+    }
+    if (e == 0) offsets[E] = grand;
+  }
+  // Per-warp global bases, and the CTA's total per expert.
+  int total = 0, gbase = 0;
+  if (e < E) {
+    gbase = eoff + before;
     int run = gbase;
 #pragma unroll
     for (int ww = 0; ww < DWARPS; ++ww) {
@@ -197,16 +203,9 @@ __global__ void __launch_bounds__(DNT) dispatch_scatter_kernel(
     total = run - gbase;
   }
   // Local exclusive scan of the totals over the experts.
-  s_scan[e] = total;
-  __syncthreads();
-  for (int o = 1; o < DNT; o <<= 1) {
-    const int v = e >= o ? s_scan[e - o] : 0;
-    __syncthreads();
-    s_scan[e] += v;
-    __syncthreads();
-  }
-  if (e < E) s_shift[e] = s_scan[e] - total - gbase;
-  const int nvalid = s_scan[DNT - 1];
+  int nvalid = 0;
+  const int lexcl = cta_excl_scan(total, s_tmp, &nvalid);
+  if (e < E) s_shift[e] = lexcl - gbase;
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
@@ -404,15 +403,13 @@ cudaError_t launch_dispatch(const int32_t* ids, const float* w, const void* x, i
               : launch_pdl(dispatch_count_kernel<CHUNK>, dim3(B), dim3(DNT), wsm, s, 0, ids, N,
                            E, bc, status);
     if (err == cudaSuccess)
-      err = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(256), 0, s, 0, bc, B, E, counts,
-                       offsets);
-    if (err == cudaSuccess)
       err = small ? launch_pdl(dispatch_scatter_kernel<CHUNK_SMALL>, dim3(B), dim3(DNT), wsm, s,
-                               0, ids, w, N, E, k, static_cast<const int32_t*>(bc), perm,
-                               inv_perm, packed_tok, w ? packed_w : nullptr, status)
+                               0, ids, w, N, E, k, static_cast<const int32_t*>(bc), counts,
+                               offsets, perm, inv_perm, packed_tok, w ? packed_w : nullptr,
+                               status)
                   : launch_pdl(dispatch_scatter_kernel<CHUNK>, dim3(B), dim3(DNT), wsm, s, 0,
-                               ids, w, N, E, k, static_cast<const int32_t*>(bc), perm, inv_perm,
-                               packed_tok, w ? packed_w : nullptr, status);
+                               ids, w, N, E, k, static_cast<const int32_t*>(bc), counts, offsets,
+                               perm, inv_perm, packed_tok, w ? packed_w : nullptr, status);
     if (err != cudaSuccess || x == nullptr) return err;
   }
   return launch_gather(x, packed_tok, offsets, 0, E, N, H, dtype, x_packed, status, s);
